@@ -1,0 +1,516 @@
+"""Benchmark of the CommunityKV decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--budget B]
+    python bench.py --impl reference ...      # the float64 CPU oracle, timed on host cores
+
+One step = ckv_score_select + ckv_sparse_decode (+ the cache append and
+ckv_assign_update when the workload updates) for the whole batch of one
+layer, with inputs resident in HBM.  Every timed step is bracketed by CUDA
+events on the launching stream; L2 is flushed (a 256 MiB write) before each
+step, outside the events.  Rank 0 prints one JSON line.  With N GPUs each rank
+runs its own batch (weak scaling, no collective on the data path); the value
+is N*K steps over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "sparse decode steps/s at 128K ctx; achieved HBM GB/s vs B200 peak"
+DEFAULT_WORKLOAD = "qwen3_8b_128k_head"
+FALLBACK_HBM_GBS = 6650.0
+KERNELS_PER_STEP_UPDATE = 5   # score, select, decode main, decode merge, assign
+KERNELS_PER_STEP_STATIC = 4
+
+
+# ----------------------------------------------------------------------------
+# host logic shared by all ranks (tested on CPU with gloo)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return ws, rank, local
+
+
+def rank_workload(wl: synth.Workload, rank: int) -> tuple:
+    """Weak scaling: every rank decodes its own batch of sequences, drawn from
+    the workload's law with rank-specific seeds (layer index = rank)."""
+    return wl, rank
+
+
+def reduce_max(x: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def job_value(n_ranks: int, steps: int, max_seconds: float) -> float:
+    return n_ranks * steps / max_seconds if max_seconds > 0 else float("nan")
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            d = json.load(open(p))
+            return float(d["hbm_gbs"]), "measured"
+        except Exception:
+            pass
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded by the committed ncu summary for this
+    kernel and workload, valid only while the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        d = json.load(open(path))
+        ent = d[kernel][workload]
+        src = os.path.join(ROOT, "graph_community_sparse_b200", "csrc", ent["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest() != ent["sha256"]:
+            return None
+        return float(ent["bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for r in csv.reader(f):
+                if len(r) >= 9:
+                    rows.append([x.strip() for x in r])
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# the CUDA arm
+# ----------------------------------------------------------------------------
+
+def union_rows(sel, U, G, Hq, Hkv, per_head: bool, T_cap: int) -> torch.Tensor:
+    """Distinct (sequence, KV head, position) rows a step's selection reads."""
+    n_tok = sel.n_tok.long()
+    if not per_head:
+        return n_tok.sum()
+    cap = sel.sel_tok.shape[1]
+    idx = torch.arange(cap, device=n_tok.device)[None, :]
+    valid = idx < n_tok[:, None]
+    gq = Hq // Hkv
+    units = torch.arange(U, device=n_tok.device)
+    group = (units // G) * Hkv + (units % G) // gq
+    key = group[:, None].long() * T_cap + sel.sel_tok.long()
+    return torch.unique(key[valid]).numel() * torch.ones((), dtype=torch.long, device=n_tok.device)
+
+
+def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
+    from graph_community_sparse_b200.layer import LayerState
+
+    K_steps, W_steps = args.steps, args.warmup
+    budget = args.budget if args.budget is not None else wl.budget
+    n_total = W_steps + K_steps + args.e2e_steps
+    extra = n_total + 8 if wl.update else 0
+    T_cap = wl.T + extra
+    layer = rank  # per-rank seeds: each rank owns a different batch of sequences
+    draw = synth.draw_cache(wl, layer=layer, device=device, T_cap=T_cap)
+    C = int(draw.labels.max()) + 1
+    st = LayerState(draw.K, draw.V, wl.Hq, wl.mode, wl.S, C, max(extra, 1))
+    U = st.U
+    labels = torch.from_numpy(draw.labels.reshape(U, wl.T).astype(np.int32)).to(device)
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record()
+    st.build(labels, wl.T)
+    b1.record()
+    torch.cuda.synchronize()
+    build_ms = b0.elapsed_time(b1)
+    if int(st.graph.dev_err.item()) != 0:
+        raise RuntimeError(f"build reported device error {int(st.graph.dev_err.item())}")
+
+    qs = [synth.draw_queries(wl, draw, i, layer) for i in range(n_total)]
+    news = [synth.draw_new_tokens(wl, draw, i, layer) for i in range(n_total)] if wl.update else []
+    flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MiB > L2
+
+    def flush():
+        flush_buf.fill_(1.0)
+
+    esz = 2 if wl.dtype == "bf16" else 4
+    row_bytes = 2 * wl.d * esz
+    per_head = wl.mode == "head"
+    num_comm = st.graph.num_comm.long()
+
+    def one_step(i, ev=None):
+        q = qs[i]
+        if ev:
+            ev[0].record()
+        st.select(q, budget)
+        if ev:
+            ev[1].record()
+        st.attend(q, want_nbr=wl.update)
+        if ev:
+            ev[2].record()
+        if wl.update:
+            k, v = news[i]
+            st.append(k, v)
+        if ev:
+            ev[3].record()
+
+    for i in range(W_steps):
+        flush()
+        one_step(i)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
+    rows_hist, ntok_hist, ncomm_hist = [], [], []
+    barrier(device)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with ClockSampler(device.index) as clk:
+        for j in range(K_steps):
+            flush()
+            one_step(W_steps + j, evs[j])
+            rows_hist.append(union_rows(st.sel, U, wl.G, wl.Hq, wl.Hkv, per_head, T_cap))
+            ntok_hist.append(st.sel.n_tok.long().sum())
+            ncomm_hist.append(num_comm.sum())
+        torch.cuda.synchronize()
+    barrier(device)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clocks = clk.summary()
+    if int(st.graph.dev_err.item()) != 0:
+        raise RuntimeError(f"device error word {int(st.graph.dev_err.item())}")
+
+    sel_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    upd_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    total_s = sum(step_ms) / 1e3
+    max_total_s = reduce_max(total_s, device)
+
+    rows = np.array([int(r.item()) for r in rows_hist], dtype=np.float64)
+    ntok = np.array([int(r.item()) for r in ntok_hist], dtype=np.float64)
+    ncomm = float(ncomm_hist[0].item())
+    q_bytes = wl.B * wl.Hq * wl.d * esz
+    out_bytes = wl.B * wl.Hq * wl.d * 4
+    dec_bytes = rows * row_bytes + ntok * 4 + q_bytes + out_bytes + (U * 8 * 4 if wl.update else 0)
+    sel_bytes = ncomm * wl.d * 4 + q_bytes + ncomm * 4 * 3 + ntok * 4
+    peak, peak_src = measured_peaks()
+
+    def gbs(bytes_, ms):
+        return float(np.mean(bytes_) / (np.mean(ms) * 1e-3) / 1e9)
+
+    dec_gbs = gbs(dec_bytes, dec_ms)
+    sel_gbs = gbs(sel_bytes, sel_ms)
+    kernels = {
+        "ckv_score_select": {"ms": float(np.mean(sel_ms)), "bytes": float(np.mean(sel_bytes)), "GB/s": sel_gbs,
+                             "frac": sel_gbs / peak},
+        "ckv_sparse_decode": {"ms": float(np.mean(dec_ms)), "bytes": float(np.mean(dec_bytes)), "GB/s": dec_gbs,
+                              "frac": dec_gbs / peak, "rows_per_step": float(rows.mean()),
+                              "tokens_per_step": float(ntok.mean())},
+    }
+    if wl.update:
+        kernels["append+ckv_assign_update"] = {"ms": float(np.mean(upd_ms))}
+    dom = max(("ckv_sparse_decode", "ckv_score_select"), key=lambda k: kernels[k]["ms"])
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": peak, "unit": "GB/s",
+                "frac": kernels[dom]["GB/s"] / peak, "peak_source": peak_src,
+                "traffic": profile_traffic(dom, wl.key), "bytes_per_launch": kernels[dom]["bytes"],
+                "timing": "CUDA events around the library call on its stream, mean over the timed steps"}
+
+    # dense comparator on the same cache and queries
+    dense_out = torch.empty_like(st.out)
+    dms = []
+    for j in range(max(3, min(K_steps, 10)) + 2):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        st.dense(qs[j % len(qs)], dense_out)
+        e1.record()
+        dms.append((e0, e1))
+    torch.cuda.synchronize()
+    dms = [a.elapsed_time(b) for a, b in dms[2:]]
+    dense_bytes = wl.B * wl.Hkv * st.T * row_bytes + q_bytes + out_bytes
+    dense_gbs = dense_bytes / (np.mean(dms) * 1e-3) / 1e9
+    dense = {"ms": float(np.mean(dms)), "bytes": float(dense_bytes), "GB/s": float(dense_gbs),
+             "frac": float(dense_gbs / peak), "T": st.T,
+             "sparse_step_speedup": float(np.mean(dms) / np.mean(step_ms))}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        pin = dict(pin_memory=True)
+        q_host = [qs[i].cpu().pin_memory() for i in range(n_total)]
+        kv_host = [(k.cpu().pin_memory(), v.cpu().pin_memory()) for k, v in news] if wl.update else []
+        q_dev = torch.empty_like(qs[0])
+        k_dev = torch.empty_like(news[0][0]) if wl.update else None
+        v_dev = torch.empty_like(news[0][1]) if wl.update else None
+        out_h = torch.empty(st.out.shape, dtype=torch.float32, **pin)
+        nbr_h = torch.empty(st.nbr8.shape, dtype=torch.int32, **pin)
+        asg_h = torch.empty(st.assigned.shape, dtype=torch.int32, **pin)
+        e_ms = []
+        h2d = q_host[0].numel() * q_host[0].element_size()
+        if wl.update:
+            h2d += 2 * kv_host[0][0].numel() * kv_host[0][0].element_size()
+        d2h = out_h.numel() * 4 + (nbr_h.numel() * 4 + asg_h.numel() * 4 if wl.update else 0)
+        for j in range(args.e2e_steps):
+            i = W_steps + K_steps + j
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            q_dev.copy_(q_host[i], non_blocking=True)
+            if wl.update:
+                k_dev.copy_(kv_host[i][0], non_blocking=True)
+                v_dev.copy_(kv_host[i][1], non_blocking=True)
+            st.select(q_dev, budget)
+            st.attend(q_dev, want_nbr=wl.update)
+            out_h.copy_(st.out, non_blocking=True)
+            if wl.update:
+                st.append(k_dev, v_dev)
+                nbr_h.copy_(st.nbr8, non_blocking=True)
+                asg_h.copy_(st.assigned, non_blocking=True)
+            e1.record()
+            e_ms.append((e0, e1))
+        torch.cuda.synchronize()
+        e_ms = [a.elapsed_time(b) for a, b in e_ms]
+        e_total = reduce_max(sum(e_ms) / 1e3, device)
+        e2e = {"value": job_value(n_ranks, len(e_ms), e_total), "unit": "steps/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": float(np.mean(e_ms))}
+
+    value = job_value(n_ranks, K_steps, max_total_s)
+    return {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": n_ranks, "steps": K_steps,
+        "warmup": W_steps, "ms_per_step": max_total_s * 1e3 / K_steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
+        "config": {"workload": wl.key, "title": wl.title, "B_per_gpu": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv,
+                   "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
+                   "communities_per_graph": float(ncomm / U), "budget": budget, "sinks": wl.S,
+                   "update": wl.update, "layout": wl.layout,
+                   "l2": "flushed by a 256 MiB write before every timed step, outside the CUDA events",
+                   "parallelism": f"dp{n_ranks} (independent batches, no collective)"},
+        "tokens_per_s": value * wl.B,
+        "roofline": roofline,
+        "kernels": kernels,
+        "dense": dense,
+        "e2e": e2e,
+        "gpu_launches": K_steps * (KERNELS_PER_STEP_UPDATE if wl.update else KERNELS_PER_STEP_STATIC),
+        "clocks": clocks,
+        "build_ms": build_ms,
+        "wall_s_timed_region": wall,
+    }
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_unit_seconds(wl: synth.Workload, draw: synth.CacheDraw, units, budget: int, step: int,
+                        layer: int = 0) -> float:
+    """Wall time of the oracle's steps for the given (b, g) units of one step,
+    single-threaded, inputs already converted to float64."""
+    import oracle.ckv_oracle as O
+    from threadpoolctl import threadpool_limits
+
+    C = int(draw.labels.max()) + 1
+    q = synth.draw_queries(wl, draw, step, layer).double().cpu().numpy()
+    kvs = {}
+    for (b, g) in units:
+        kvh = O.graph_kv_head(wl.mode, g, wl.Hq, wl.Hkv)
+        if (b, kvh) not in kvs:
+            kvs[(b, kvh)] = (draw.K[b, kvh, : wl.T].double().cpu().numpy(),
+                             draw.V[b, kvh, : wl.T].double().cpu().numpy())
+    if wl.update:
+        kn, _ = synth.draw_new_tokens(wl, draw, step, layer)
+        kn = kn.double().cpu().numpy()
+    t = 0.0
+    with threadpool_limits(1):
+        for (b, g) in units:
+            st = O.GraphState(draw.labels[b, g], wl.T_cap, wl.S, C)
+            kvh = O.graph_kv_head(wl.mode, g, wl.Hq, wl.Hkv)
+            K, V = kvs[(b, kvh)]
+            t0 = time.perf_counter()
+            heads = O.graph_heads(wl.mode, g, wl.Hq, wl.Hkv)
+            members = st.members()
+            cent, cnt = O.centroids(K, members)
+            s = O.community_scores(q[b, heads], cent, cnt)
+            sel = O.select(s, cnt, budget)
+            toks = O.token_set(sel, members, wl.S)
+            for h in heads:
+                O.attention(q[b, h], K, V, toks)
+            nbr = O.neighbours(q[b, heads], K, toks, wl.S)
+            if wl.update:
+                O.assign(kn[b, kvh], cent, [int(st.comm_of[p]) for p in nbr])
+            t += time.perf_counter() - t0
+    return t
+
+
+def sample_units(wl: synth.Workload, n: int, seed: int):
+    rng = np.random.default_rng(seed)
+    allu = [(b, g) for b in range(wl.B) for g in range(wl.G)]
+    idx = rng.choice(len(allu), size=min(n, len(allu)), replace=False)
+    return [allu[i] for i in sorted(idx)]
+
+
+def cpu_baseline(wl: synth.Workload, budget: int, device, n_units: int) -> dict:
+    draw = synth.draw_cache(wl, device=device)
+    units = sample_units(wl, n_units, 1)
+    t = oracle_unit_seconds(wl, draw, units, budget, 0)
+    per_step = t / len(units) * (wl.B * wl.G)
+    del draw
+    return {"value": 1.0 / per_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"{len(units)} of {wl.B * wl.G} graph units of one decode step "
+                      f"({t:.1f} s single-threaded float64 numpy), scaled to the whole step"}
+
+
+def run_reference(args, wl: synth.Workload, device) -> dict:
+    budget = args.budget if args.budget is not None else wl.budget
+    draw = synth.draw_cache(wl, device=device)
+    per_step_units = max(1, args.ref_units)
+    times = []
+    for i in range(args.warmup + args.steps):
+        units = sample_units(wl, per_step_units, 100 + i)
+        t = oracle_unit_seconds(wl, draw, units, budget, i)
+        if i >= args.warmup:
+            times.append(t / len(units) * (wl.B * wl.G))
+    value = args.steps / sum(times)
+    cb = {"value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+          "sample": f"{per_step_units} of {wl.B * wl.G} graph units per step, scaled to the whole step"}
+    return {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.key, "budget": budget},
+            "cpu_baseline": cb, "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------
+
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-units", type=int, default=48, help="graph units the CPU baseline times")
+    ap.add_argument("--ref-units", type=int, default=4, help="graph units per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+def main(argv=None):
+    args = parse(argv)
+    ws, rank, local = dist_env()
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        device = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+        print(json.dumps(run_reference(args, wl, device)), flush=True)
+        return 0
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=device, timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_cuda(args, wl, rank, ws, device)
+        if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+            torch.cuda.empty_cache()
+            res["cpu_baseline"] = cpu_baseline(wl, res["config"]["budget"], device, args.cpu_units)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[local])
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,251 @@
+"""Python binding of libckv, the CommunityKV decode hot path for B200.
+
+Argument marshalling only: every function passes raw device pointers, sizes
+and the current CUDA stream to the C entry point of the same name in
+``libckv.so`` (declared in include/ckv.h) and raises ``CKVError`` on a
+non-zero status.  PyTorch provides device memory and streams; no computation
+of the path happens here.  Importing the package fails loudly when the
+library has not been built: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "CKVError", "lib", "LIB_PATH", "CacheDesc", "GraphDesc", "SelectionDesc",
+    "Graph", "Selection", "cache_desc", "new_graph", "new_selection", "new_workspace",
+    "ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
+    "ckv_assign_update", "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
+    "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
+    "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP",
+    "NEIGHBOURS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckv.so")
+
+DTYPE_F32, DTYPE_BF16 = 0, 1
+PER_GROUP, PER_HEAD = 0, 1
+DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
+NEIGHBOURS = 8
+EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
+            "ckv_assign_update", "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
+            "ckv_abi_version")
+
+
+class CKVError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {ckv_status_string(status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libckv.so not built at {LIB_PATH}; run `python -m graph_community_sparse_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+_i32, _i64, _p, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("dtype", _i32), ("B", _i32), ("Hkv", _i32), ("Hq", _i32), ("d", _i32),
+                ("T_cap", _i32), ("k", _p), ("v", _p), ("stride_b", _i64), ("stride_h", _i64),
+                ("stride_t", _i64)]
+
+
+class GraphDesc(ctypes.Structure):
+    _fields_ = [("mode", _i32), ("S", _i32), ("Cmax", _i32), ("max_tail", _i32), ("T_cap", _i32),
+                ("comm_of", _p), ("offs", _p), ("tok", _p), ("cnt", _p), ("cent", _p),
+                ("num_comm", _p), ("tail_tok", _p), ("tail_comm", _p), ("tail_len", _p),
+                ("dev_err", _p)]
+
+
+class SelectionDesc(ctypes.Structure):
+    _fields_ = [("tok_cap", _i32), ("sel_comm", _p), ("n_sel", _p), ("sel_tok", _p), ("n_tok", _p),
+                ("unit_prefix", _p)]
+
+
+_P = ctypes.POINTER
+lib.ckv_workspace_size.argtypes = [_P(CacheDesc), _P(GraphDesc), _P(SelectionDesc), _P(_sz)]
+lib.ckv_build_centroids.argtypes = [_P(CacheDesc), _p, _i64, _i32, _P(GraphDesc), _p, _sz, _p]
+lib.ckv_score_select.argtypes = [_P(CacheDesc), _P(GraphDesc), _p, _i32, _P(SelectionDesc), _p, _sz, _p]
+lib.ckv_sparse_decode.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p, _sz, _p]
+lib.ckv_assign_update.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p]
+lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
+for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
+           "ckv_assign_update", "ckv_dense_decode"):
+    getattr(lib, _f).restype = ctypes.c_int
+lib.ckv_status_string.argtypes = [ctypes.c_int]
+lib.ckv_status_string.restype = ctypes.c_char_p
+lib.ckv_last_error.argtypes = []
+lib.ckv_last_error.restype = ctypes.c_char_p
+lib.ckv_abi_version.argtypes = []
+lib.ckv_abi_version.restype = ctypes.c_int32
+
+
+def ckv_status_string(status: int) -> str:
+    return lib.ckv_status_string(int(status)).decode()
+
+
+def ckv_last_error() -> str:
+    return lib.ckv_last_error().decode()
+
+
+def ckv_abi_version() -> int:
+    return int(lib.ckv_abi_version())
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise CKVError(status, where, ckv_last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        if not torch.cuda.is_available():
+            return None
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ----------------------------------------------------------------------------
+# descriptors and buffers (device memory comes from PyTorch)
+# ----------------------------------------------------------------------------
+
+def cache_desc(K: torch.Tensor, V: torch.Tensor, Hq: int) -> CacheDesc:
+    """Describe a [B, Hkv, T_cap, d] K/V cache pair (same shape and strides)."""
+    if K.shape != V.shape or K.stride() != V.stride() or K.dtype != V.dtype:
+        raise ValueError("K and V must share shape, strides and dtype")
+    if K.dim() != 4 or K.stride(3) != 1:
+        raise ValueError("K must be [B, Hkv, T_cap, d] with contiguous rows")
+    dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(K.dtype)
+    if dt is None:
+        raise ValueError(f"unsupported dtype {K.dtype}")
+    B, Hkv, T_cap, d = K.shape
+    return CacheDesc(dt, B, Hkv, Hq, d, T_cap, K.data_ptr(), V.data_ptr(),
+                     K.stride(0), K.stride(1), K.stride(2))
+
+
+@dataclass
+class Graph:
+    desc: GraphDesc
+    comm_of: torch.Tensor
+    offs: torch.Tensor
+    tok: torch.Tensor
+    cnt: torch.Tensor
+    cent: torch.Tensor
+    num_comm: torch.Tensor
+    tail_tok: torch.Tensor
+    tail_comm: torch.Tensor
+    tail_len: torch.Tensor
+    dev_err: torch.Tensor
+
+    @property
+    def U(self) -> int:
+        return self.num_comm.shape[0]
+
+
+@dataclass
+class Selection:
+    desc: SelectionDesc
+    sel_comm: torch.Tensor
+    n_sel: torch.Tensor
+    sel_tok: torch.Tensor
+    n_tok: torch.Tensor
+    unit_prefix: torch.Tensor
+
+
+def new_graph(cache: CacheDesc, mode: int, S: int, Cmax: int, max_tail: int, device="cuda") -> Graph:
+    G = cache.Hq if mode == PER_HEAD else cache.Hkv
+    U = cache.B * G
+    i32 = dict(dtype=torch.int32, device=device)
+    t = dict(
+        comm_of=torch.full((U, cache.T_cap), -1, **i32),
+        offs=torch.zeros((U, Cmax + 1), **i32),
+        tok=torch.zeros((U, cache.T_cap), **i32),
+        cnt=torch.zeros((U, Cmax), **i32),
+        cent=torch.zeros((U, Cmax, cache.d), dtype=torch.float32, device=device),
+        num_comm=torch.zeros((U,), **i32),
+        tail_tok=torch.zeros((U, max(max_tail, 1)), **i32),
+        tail_comm=torch.zeros((U, max(max_tail, 1)), **i32),
+        tail_len=torch.zeros((U,), **i32),
+        dev_err=torch.zeros((1,), **i32),
+    )
+    desc = GraphDesc(mode, S, Cmax, max_tail, cache.T_cap, *(t[k].data_ptr() for k in (
+        "comm_of", "offs", "tok", "cnt", "cent", "num_comm", "tail_tok", "tail_comm", "tail_len",
+        "dev_err")))
+    return Graph(desc, **t)
+
+
+def new_selection(cache: CacheDesc, graph: Graph, tok_cap: int, device="cuda") -> Selection:
+    U, Cmax = graph.U, graph.desc.Cmax
+    i32 = dict(dtype=torch.int32, device=device)
+    t = dict(sel_comm=torch.zeros((U, Cmax), **i32), n_sel=torch.zeros((U,), **i32),
+             sel_tok=torch.zeros((U, tok_cap), **i32), n_tok=torch.zeros((U,), **i32),
+             unit_prefix=torch.zeros((U + 1,), **i32))
+    desc = SelectionDesc(tok_cap, *(t[k].data_ptr() for k in ("sel_comm", "n_sel", "sel_tok", "n_tok",
+                                                               "unit_prefix")))
+    return Selection(desc, **t)
+
+
+def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    # torch's caching allocator hands out 512-byte aligned blocks
+    return torch.empty((max(int(nbytes), 256),), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------------------
+# the entry points
+# ----------------------------------------------------------------------------
+
+def ckv_workspace_size(cache: CacheDesc, graph: Optional[Graph] = None,
+                       sel: Optional[Selection] = None) -> int:
+    out = _sz(0)
+    g = ctypes.byref(graph.desc) if graph is not None else None
+    s = ctypes.byref(sel.desc) if sel is not None else None
+    _check(lib.ckv_workspace_size(ctypes.byref(cache), g, s, ctypes.byref(out)), "ckv_workspace_size")
+    return int(out.value)
+
+
+def ckv_build_centroids(cache: CacheDesc, labels: torch.Tensor, T: int, graph: Graph,
+                        ws: torch.Tensor, stream=None) -> None:
+    if labels.dtype != torch.int32 or labels.dim() != 2 or labels.stride(1) != 1:
+        raise ValueError("labels must be int32 [U, >=T] with contiguous rows")
+    _check(lib.ckv_build_centroids(ctypes.byref(cache), labels.data_ptr(), labels.stride(0), T,
+                                   ctypes.byref(graph.desc), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "ckv_build_centroids")
+
+
+def ckv_score_select(cache: CacheDesc, graph: Graph, q: torch.Tensor, budget: int, sel: Selection,
+                     ws: torch.Tensor, stream=None) -> None:
+    _check(lib.ckv_score_select(ctypes.byref(cache), ctypes.byref(graph.desc), q.data_ptr(), budget,
+                                ctypes.byref(sel.desc), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "ckv_score_select")
+
+
+def ckv_sparse_decode(cache: CacheDesc, q: torch.Tensor, graph: Graph, sel: Selection, out: torch.Tensor,
+                      nbr8: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> None:
+    _check(lib.ckv_sparse_decode(ctypes.byref(cache), q.data_ptr(), ctypes.byref(graph.desc),
+                                 ctypes.byref(sel.desc), out.data_ptr(), _ptr(nbr8), ws.data_ptr(),
+                                 ws.numel(), _stream(stream)),
+           "ckv_sparse_decode")
+
+
+def ckv_assign_update(cache: CacheDesc, graph: Graph, pos: int, nbr8: torch.Tensor,
+                      assigned: Optional[torch.Tensor], stream=None) -> None:
+    _check(lib.ckv_assign_update(ctypes.byref(cache), ctypes.byref(graph.desc), pos, nbr8.data_ptr(),
+                                 _ptr(assigned), _stream(stream)),
+           "ckv_assign_update")
+
+
+def ckv_dense_decode(cache: CacheDesc, q: torch.Tensor, T: int, out: torch.Tensor, ws: torch.Tensor,
+                     stream=None) -> None:
+    _check(lib.ckv_dense_decode(ctypes.byref(cache), q.data_ptr(), T, out.data_ptr(), ws.data_ptr(),
+                                ws.numel(), _stream(stream)),
+           "ckv_dense_decode")

@@ -1,0 +1,235 @@
+// Internal declarations and device helpers shared by the libckv kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ckv.h"
+
+namespace ckv {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int MAX_UNITS = 8192;      // B * G
+constexpr int MAX_CMAX = 8192;       // communities per graph
+constexpr int MAX_DECODE_WARPS = 8192;
+constexpr int BUILD_CHUNK = 4096;    // positions per histogram / scatter block
+
+// ---------------------------------------------------------------------------
+// element access: a lane owns E = D/16 consecutive elements of a row
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <typename T> struct ElemBytes;
+template <> struct ElemBytes<float> { static constexpr int v = 4; };
+template <> struct ElemBytes<__nv_bfloat16> { static constexpr int v = 2; };
+
+// Convert E elements at a (shared or global) address to fp32.  Generic loads.
+template <typename T, int E>
+__device__ __forceinline__ void load_row_part(const T* p, float (&x)[E]);
+
+template <>
+__device__ __forceinline__ void load_row_part<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&x)[8]) {
+    uint4 w = *reinterpret_cast<const uint4*>(p);
+    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+}
+template <>
+__device__ __forceinline__ void load_row_part<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&x)[4]) {
+    uint2 w = *reinterpret_cast<const uint2*>(p);
+    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+}
+template <>
+__device__ __forceinline__ void load_row_part<float, 8>(const float* p, float (&x)[8]) {
+    float4 a = reinterpret_cast<const float4*>(p)[0];
+    float4 b = reinterpret_cast<const float4*>(p)[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load_row_part<float, 4>(const float* p, float (&x)[4]) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// ---------------------------------------------------------------------------
+// cp.async (global -> shared, L2 only); size 0 means zero-fill, nothing read
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void cp_async_16(void* smem, const void* gmem, bool pred) {
+    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    int sz = pred ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(sz)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_8(void* smem, const void* gmem, bool pred) {
+    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    int sz = pred ? 8 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(s), "l"(gmem), "r"(sz)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+// Copy `BYTES` bytes (8, 16 or 32) per lane.
+template <int BYTES>
+__device__ __forceinline__ void cp_async_part(void* smem, const void* gmem, bool pred) {
+    if constexpr (BYTES == 8) {
+        cp_async_8(smem, gmem, pred);
+    } else if constexpr (BYTES == 16) {
+        cp_async_16(smem, gmem, pred);
+    } else {
+        static_assert(BYTES == 32, "row part of 8, 16 or 32 bytes");
+        cp_async_16(smem, gmem, pred);
+        cp_async_16(static_cast<char*>(smem) + 16, static_cast<const char*>(gmem) + 16, pred);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// half-warp reduction of GQ per-head partial sums with value exchange:
+// after it, lane l holds the full sum of head (l & 15) >> (4 - log2 GQ).
+// GQ values over 16 lanes cost GQ - 1 + 4 - log2 GQ shuffles instead of 4 GQ.
+// ---------------------------------------------------------------------------
+
+template <int GQ> struct Log2;
+template <> struct Log2<1> { static constexpr int v = 0; };
+template <> struct Log2<2> { static constexpr int v = 1; };
+template <> struct Log2<4> { static constexpr int v = 2; };
+template <> struct Log2<8> { static constexpr int v = 3; };
+
+template <int GQ>
+__device__ __forceinline__ float halfwarp_reduce_heads(float (&v)[GQ], int lane) {
+    float cur[GQ];
+#pragma unroll
+    for (int i = 0; i < GQ; ++i) cur[i] = v[i];
+    int n = GQ;
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) {
+        if (n > 1) {
+            const bool upper = (lane & o) != 0;
+            const int h = n >> 1;
+#pragma unroll
+            for (int i = 0; i < h; ++i) {
+                float send = upper ? cur[i] : cur[i + h];
+                float keep = upper ? cur[i + h] : cur[i];
+                cur[i] = keep + __shfl_xor_sync(FULL, send, o);
+            }
+            n = h;
+        } else {
+            cur[0] += __shfl_xor_sync(FULL, cur[0], o);
+        }
+    }
+    return cur[0];
+}
+
+template <int GQ>
+__device__ __forceinline__ int head_of_lane(int lane) {
+    return (lane & 15) >> (4 - Log2<GQ>::v);
+}
+
+// Max over the lanes of one half-warp that hold different heads.
+template <int GQ>
+__device__ __forceinline__ float halfwarp_max_over_heads(float x) {
+#pragma unroll
+    for (int o = 16 >> Log2<GQ>::v; o <= 8; o <<= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
+    return x;
+}
+
+// ---------------------------------------------------------------------------
+// block-wide exclusive scan of one int per thread (blockDim multiple of 32)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int block_exclusive_scan(int x, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? s_warp[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(FULL, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nw) s_warp[lane] = wi - w;
+        if (lane == 31) s_warp[32] = wi;
+    }
+    __syncthreads();
+    int r = s_warp[warp] + inc - x;
+    if (total) *total = s_warp[32];
+    __syncthreads();
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// launch parameter packs (host builds them after validation)
+// ---------------------------------------------------------------------------
+
+struct CacheView {
+    const void* k;
+    const void* v;
+    int64_t sb, sh, st;
+    int B, Hkv, Hq, d, T_cap, dtype;
+};
+
+struct GraphView {
+    int mode, S, Cmax, max_tail, T_cap, G, gq;
+    int32_t* comm_of;
+    int32_t* offs;
+    int32_t* tok;
+    int32_t* cnt;
+    float* cent;
+    int32_t* num_comm;
+    int32_t* tail_tok;
+    int32_t* tail_comm;
+    int32_t* tail_len;
+    int32_t* dev_err;
+};
+
+struct SelView {
+    int tok_cap;
+    int32_t* sel_comm;
+    int32_t* n_sel;
+    int32_t* sel_tok;
+    int32_t* n_tok;
+    int32_t* unit_prefix;
+};
+
+// workspace carving
+struct DecodeWs {
+    float* m;      // [slots, GQ]
+    float* l;      // [slots, GQ]
+    float* acc;    // [slots, GQ, D]
+    float* tv;     // [slots, 8]
+    int32_t* tp;   // [slots, 8]
+};
+
+size_t build_ws_bytes(int U, int Cmax, int T_cap);
+size_t select_ws_bytes(int U, int Cmax);
+size_t decode_ws_bytes(int U, int gq, int d);
+DecodeWs carve_decode_ws(void* ws, int U, int gq, int d);
+
+cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* labels,
+                         int64_t labels_stride, int T, void* ws, cudaStream_t st);
+cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const void* q, int budget,
+                                const SelView& s, void* ws, cudaStream_t st);
+cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const SelView& s,
+                                 const void* q, float* out, int32_t* nbr8, void* ws, cudaStream_t st);
+cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float* out, void* ws,
+                                cudaStream_t st);
+cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const int32_t* nbr8,
+                                 int32_t* assigned, cudaStream_t st);
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace ckv

@@ -1,0 +1,74 @@
+"""Buffers and call sequence for one layer's CommunityKV decode state.
+
+``LayerState`` owns (through PyTorch) the graph arrays, the selection and the
+workspace for one KV cache, and issues the four library calls in decode
+order.  It computes nothing itself.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import (PER_GROUP, PER_HEAD, Graph, Selection, cache_desc, ckv_assign_update,
+               ckv_build_centroids, ckv_dense_decode, ckv_score_select, ckv_sparse_decode,
+               ckv_workspace_size, new_graph, new_selection, new_workspace, NEIGHBOURS)
+
+
+class LayerState:
+    """K, V: [B, Hkv, T_cap, d] device tensors (bf16 or fp32), read in place.
+
+    mode: "group" (one graph per KV group) or "head" (one graph per query head).
+    tok_cap defaults to T_cap, which can never overflow.
+    """
+
+    def __init__(self, K: torch.Tensor, V: torch.Tensor, Hq: int, mode: str, S: int, Cmax: int,
+                 max_tail: int, tok_cap: Optional[int] = None):
+        self.K, self.V = K, V
+        self.cache = cache_desc(K, V, Hq)
+        self.mode = PER_HEAD if mode == "head" else PER_GROUP
+        self.graph: Graph = new_graph(self.cache, self.mode, S, Cmax, max_tail, device=K.device)
+        self.sel: Selection = new_selection(self.cache, self.graph, tok_cap or self.cache.T_cap,
+                                            device=K.device)
+        self.ws = new_workspace(ckv_workspace_size(self.cache, self.graph, self.sel), device=K.device)
+        B, Hq_, d = self.cache.B, Hq, self.cache.d
+        self.out = torch.empty((B, Hq_, d), dtype=torch.float32, device=K.device)
+        self.nbr8 = torch.full((self.graph.U, NEIGHBOURS), -1, dtype=torch.int32, device=K.device)
+        self.assigned = torch.full((self.graph.U,), -1, dtype=torch.int32, device=K.device)
+        self.T = 0
+
+    @property
+    def U(self) -> int:
+        return self.graph.U
+
+    def build(self, labels: torch.Tensor, T: int, stream=None) -> None:
+        """labels: int32 [U, >=T] on the device."""
+        ckv_build_centroids(self.cache, labels, T, self.graph, self.ws, stream)
+        self.T = T
+
+    def select(self, q: torch.Tensor, budget: int, stream=None) -> None:
+        ckv_score_select(self.cache, self.graph, q, budget, self.sel, self.ws, stream)
+
+    def attend(self, q: torch.Tensor, want_nbr: bool = True, stream=None) -> torch.Tensor:
+        ckv_sparse_decode(self.cache, q, self.graph, self.sel, self.out,
+                          self.nbr8 if want_nbr else None, self.ws, stream)
+        return self.out
+
+    def decode(self, q: torch.Tensor, budget: int, want_nbr: bool = True, stream=None) -> torch.Tensor:
+        self.select(q, budget, stream)
+        return self.attend(q, want_nbr, stream)
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> torch.Tensor:
+        """Write the new token's K/V rows ([B, Hkv, d]) at position T (the
+        model's ordinary cache append) and let it join a community."""
+        pos = self.T
+        self.K[:, :, pos].copy_(k_new)
+        self.V[:, :, pos].copy_(v_new)
+        ckv_assign_update(self.cache, self.graph, pos, self.nbr8, self.assigned, stream)
+        self.T += 1
+        return self.assigned
+
+    def dense(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        out = torch.empty_like(self.out) if out is None else out
+        ckv_dense_decode(self.cache, q, self.T, out, self.ws, stream)
+        return out

@@ -1,0 +1,234 @@
+/*
+ * ckv.h -- C ABI of libckv, the CommunityKV decode-time hot path for NVIDIA
+ * B200 (sm_100a).
+ *
+ * CommunityKV ("CommunityKV: Efficient Long-Context Decoding via Graph
+ * Partitioning", McKenna, Alexandridis, Susanj, Liu, 2026) keeps the whole KV
+ * cache and groups its tokens into communities.  At each decode step a query
+ * is compared with the community centres only; the best communities up to a
+ * token budget, plus the always-kept sink tokens, are read from the full
+ * cache and exact attention runs over them; each new token joins one
+ * neighbouring community and one centre is updated at a cost independent of
+ * the context length.  Sources used below:
+ *   [R-A] rit.work summary of the preprint, section "A graph of tokens
+ *         replaces re-clustering" (paragraphs 3-6);
+ *   [R-B] same page, section "The speed-up depends on how many graphs the
+ *         model stores" (graph per KV group vs per query head, small budget);
+ *   [ABS] the preprint's abstract (omanscience.com listing): constant-time
+ *         local update, one graph per query head or per query group.
+ * The community partition itself (Leiden on the prefill QK^T graph) is not
+ * computed here: callers pass labels.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All pointers in the descriptors and arguments are DEVICE pointers owned
+ *    by the caller, except the descriptors themselves (host structs, read
+ *    during the call only).  The library keeps no pointer after returning.
+ *  - Calls are asynchronous on `stream` and never synchronise the device;
+ *    they may be captured into a CUDA graph after one uncaptured call per
+ *    device and kernel shape (the first call caches device attributes).
+ *  - No call allocates device memory.  Scratch comes from the caller's
+ *    workspace `ws` of `ws_bytes` bytes (256-byte aligned), sized by
+ *    ckv_workspace_size(); a smaller workspace returns CKV_ERR_WORKSPACE.
+ *  - Host-side checks happen before any launch and return a status without
+ *    touching the device; ckv_last_error() then names the failed check.
+ *    Data-dependent faults detected on the device (a label out of range, a
+ *    full tail, a token list longer than its capacity) set bits in the
+ *    caller's `dev_err` word (ckv_graph_desc) and the offending item is
+ *    skipped; kernels never trap and never wait on another block.
+ *  - Graph unit u = b * G + g, with G = Hkv graphs per sequence in
+ *    CKV_GRAPH_PER_GROUP mode (graph g serves query heads g*Hq/Hkv ...) and
+ *    G = Hq in CKV_GRAPH_PER_HEAD mode (graph g serves query head g, whose
+ *    KV head is g / (Hq/Hkv)).  [R-B], [ABS]
+ *  - Supported: d in {64, 128}; Hq/Hkv in {1, 2, 4, 8}; K/V/q in bf16 or
+ *    fp32; 1 <= Cmax <= 8192; B * G <= 8192.
+ */
+#ifndef CKV_H
+#define CKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define CKV_API __attribute__((visibility("default")))
+#else
+#define CKV_API
+#endif
+
+#define CKV_ABI_VERSION 1
+#define CKV_NEIGHBOURS 8
+
+typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
+
+typedef enum {
+    CKV_OK = 0,
+    CKV_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, stride or value  */
+    CKV_ERR_MISALIGNED = 2,   /* K/V rows or q rows not 16-byte aligned    */
+    CKV_ERR_UNSUPPORTED = 3,  /* d, Hq/Hkv, dtype or size not supported     */
+    CKV_ERR_CAPACITY = 4,     /* T or a position beyond T_cap              */
+    CKV_ERR_WORKSPACE = 5,    /* ws too small or misaligned                 */
+    CKV_ERR_CUDA = 6          /* a CUDA launch or attribute call failed     */
+} ckv_status;
+
+typedef enum { CKV_DTYPE_F32 = 0, CKV_DTYPE_BF16 = 1 } ckv_dtype;
+typedef enum { CKV_GRAPH_PER_GROUP = 0, CKV_GRAPH_PER_HEAD = 1 } ckv_graph_mode;
+
+/* Bits of the device error word (ckv_graph_desc.dev_err). */
+#define CKV_DEVERR_SINK_LABEL 1   /* a position < S did not carry label -1            */
+#define CKV_DEVERR_LABEL_RANGE 2  /* a label outside [0, Cmax) at a position >= S      */
+#define CKV_DEVERR_TAIL_FULL 4    /* ckv_assign_update found the tail full; not joined */
+#define CKV_DEVERR_TOKEN_CAP 8    /* a selection longer than tok_cap was truncated     */
+
+/*
+ * The full KV cache of one layer: K and V are [B, Hkv, T_cap, d] with the d
+ * elements of a row contiguous; strides are in elements and their byte
+ * values must be multiples of 16 (as must the base pointers).  The library
+ * only reads it; no call writes K or V.  [R-A] paragraph 5: the cache stays
+ * whole so any fragment can be selected again later.
+ */
+typedef struct {
+    int32_t dtype;  /* ckv_dtype, also the dtype of q */
+    int32_t B, Hkv, Hq, d;
+    int32_t T_cap;  /* rows allocated per (b, kv head) */
+    const void* k;
+    const void* v;
+    int64_t stride_b, stride_h, stride_t;
+} ckv_cache_desc;
+
+/*
+ * Community graph state for all B * G graph units of one layer.
+ *   comm_of  int32 [U, T_cap]   community of each position (-1: sink or none)
+ *   offs     int32 [U, Cmax+1]  CSR offsets of the build-time members
+ *   tok      int32 [U, T_cap]   members sorted by (community, position)
+ *   cnt      int32 [U, Cmax]    member count, including tail members
+ *   cent     fp32  [U, Cmax, d] running-mean centre of each community
+ *   num_comm int32 [U]          1 + largest community id present
+ *   tail_tok, tail_comm int32 [U, max_tail]  tokens joined after the build
+ *   tail_len int32 [U]
+ *   dev_err  int32 [1]          OR of CKV_DEVERR_* bits; the caller zeroes it
+ * S sink positions 0..S-1 belong to no community and are always attended
+ * ([R-A] paragraph 3).  T_cap here must equal the cache's T_cap.
+ */
+typedef struct {
+    int32_t mode;  /* ckv_graph_mode */
+    int32_t S;
+    int32_t Cmax;
+    int32_t max_tail;
+    int32_t T_cap;
+    int32_t* comm_of;
+    int32_t* offs;
+    int32_t* tok;
+    int32_t* cnt;
+    float* cent;
+    int32_t* num_comm;
+    int32_t* tail_tok;
+    int32_t* tail_comm;
+    int32_t* tail_len;
+    int32_t* dev_err;
+} ckv_graph_desc;
+
+/*
+ * One step's selection, written by ckv_score_select, read by
+ * ckv_sparse_decode.
+ *   sel_comm    int32 [U, Cmax]     selected community ids, best first
+ *   n_sel       int32 [U]
+ *   sel_tok     int32 [U, tok_cap]  positions to attend: the S sinks, then the
+ *                                   build-time members of each selected
+ *                                   community in rank order, then its tail
+ *                                   members
+ *   n_tok       int32 [U]           length of each sel_tok row
+ *   unit_prefix int32 [U+1]         exclusive prefix sum of n_tok
+ * tok_cap >= T_cap can never overflow; tok_cap >= S + max(budget, largest
+ * community) + max_tail suffices too.
+ */
+typedef struct {
+    int32_t tok_cap;
+    int32_t* sel_comm;
+    int32_t* n_sel;
+    int32_t* sel_tok;
+    int32_t* n_tok;
+    int32_t* unit_prefix;
+} ckv_selection_desc;
+
+/* Bytes of workspace that any call below needs for these descriptors
+ * (`sel` may be NULL).  Host only; never touches the device. */
+CKV_API ckv_status ckv_workspace_size(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
+                              const ckv_selection_desc* sel, size_t* bytes);
+
+/*
+ * Build the community state from labels, once per sequence and layer
+ * ([R-A] paragraph 4: every community gets a centre).
+ *   labels  int32, row u at labels + u * labels_stride, T entries:
+ *           -1 at positions < S, in [0, Cmax) elsewhere.
+ * Writes comm_of (positions >= T get -1), offs, tok, cnt, cent (fp32 mean of
+ * the member keys, summed in fp64 in position order), num_comm; empties the
+ * tails.  Requires S <= T <= T_cap.
+ */
+CKV_API ckv_status ckv_build_centroids(const ckv_cache_desc* cache, const int32_t* labels,
+                               int64_t labels_stride, int32_t T, const ckv_graph_desc* graph,
+                               void* ws, size_t ws_bytes, ckv_stream_t stream);
+
+/*
+ * Score every community against the step's queries and select the top ones
+ * under the budget ([R-A] paragraph 4; [R-B] on the small active budget).
+ *   q       [B, Hq, d] in the cache dtype, contiguous.
+ *   score   s_c = max over the graph's query heads h of q_h . cent_c / sqrt(d)
+ *   select  rank non-empty communities by (s_c desc, id asc); take the
+ *           longest ranked prefix whose cnt sum is <= budget, and at least the
+ *           top community; the sinks come on top of the budget.
+ * Writes every field of `sel`.  budget >= 0.
+ */
+CKV_API ckv_status ckv_score_select(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
+                            const void* q, int32_t budget, const ckv_selection_desc* sel,
+                            void* ws, size_t ws_bytes, ckv_stream_t stream);
+
+/*
+ * Exact softmax attention over the selected positions only, read in place
+ * from the full cache with no gather copy ([R-A] paragraphs 4-5).
+ *   out   fp32 [B, Hq, d]: o_h = sum_t softmax_t(q_h . k_t / sqrt(d)) v_t over
+ *         sel_tok of head h's graph unit (zero for an empty selection).
+ *   nbr8  int32 [U, 8] or NULL: the 8 non-sink selected positions with the
+ *         largest graph logit (max over the graph's heads), best first, ties
+ *         to the lower position, -1 padded: the neighbours for
+ *         ckv_assign_update.
+ */
+CKV_API ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q,
+                             const ckv_graph_desc* graph, const ckv_selection_desc* sel,
+                             float* out, int32_t* nbr8, void* ws, size_t ws_bytes,
+                             ckv_stream_t stream);
+
+/*
+ * Local update for the token just written at position `pos` (its K/V rows are
+ * already in the cache): in every graph unit it joins the candidate
+ * community (the communities of nbr8) maximising k_new . cent_c / sqrt(d),
+ * ties to the lower id; that centre moves by (k_new - cent)/(cnt + 1), cnt
+ * grows by one, and (pos, c) is appended to the tail.  O(8 d) per graph,
+ * independent of the context length ([R-A] paragraph 6; [ABS]: the
+ * update takes constant time).  assigned int32 [U] or NULL receives the community (-1: no
+ * candidate, or tail full).  0 <= pos < T_cap.
+ */
+CKV_API ckv_status ckv_assign_update(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
+                             int32_t pos, const int32_t* nbr8, int32_t* assigned,
+                             ckv_stream_t stream);
+
+/*
+ * Dense comparator: exact GQA decode attention over positions [0, T) of every
+ * (b, kv head), out fp32 [B, Hq, d].  The pages measure their speed-ups against
+ * dense attention ([R-B], [ABS]).  Workspace: ckv_workspace_size().
+ */
+CKV_API ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t T, float* out,
+                            void* ws, size_t ws_bytes, ckv_stream_t stream);
+
+CKV_API const char* ckv_status_string(ckv_status status);
+/* Message of the last failed call on this host thread ("" if none). */
+CKV_API const char* ckv_last_error(void);
+CKV_API int32_t ckv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CKV_H */

@@ -1,0 +1,185 @@
+"""CUDA path (through the C ABI) against the CPU oracle, on a B200.
+
+Small cases run every unit through the oracle, span many warps' slices and
+ragged tails, and cover both graph modes, both dtypes, d = 64/128 and every
+supported GQA ratio.  Edge cases: budget 0 (the top community is still
+taken), a budget covering everything (equals dense attention), no sinks, a
+single community, empty community ids, a full tail, a token list longer than
+its capacity, and labels the build must reject.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.ckv_oracle as O
+import synth
+from parity_util import BAND, TOL, Case, Report
+
+pytestmark = pytest.mark.gpu
+
+BASE = synth.WORKLOADS["qwen3_8b_32k"]
+
+
+def small(key, index, **kw):
+    args = dict(key=key, title=key, index=index, B=2, T=3000, budgets=(300,), steps=3, update=True)
+    args.update(kw)
+    return BASE.replace(**args)
+
+
+SHAPES = [
+    synth.WORKLOADS["tiny"],
+    small("bf16_group_gq4", 20),
+    small("bf16_head_gq1", 21, mode="head", T=2500, budgets=(200,)),
+    small("bf16_d64_gq2", 22, d=64, Hq=16, Hkv=8),
+    small("f32_d128_gq8", 23, dtype="f32", Hq=32, Hkv=4, budgets=(500,)),
+    small("bf16_gq1_mha", 24, Hq=8, Hkv=8),
+    small("f32_d64_head", 25, dtype="f32", d=64, mode="head", Hq=8, Hkv=4),
+    small("bf16_zipf", 26, sizes="zipf", T=6000, budgets=(700,), update=False),
+    small("bf16_spans", 27, layout="spans"),
+]
+
+
+@pytest.fixture(autouse=True)
+def _free():
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("wl", SHAPES, ids=[w.key for w in SHAPES])
+def test_build_matches_oracle(wl):
+    case = Case(wl)
+    assert case.check_build() <= 1e-5
+    assert int(case.st.graph.dev_err.item()) == 0
+
+
+@pytest.mark.parametrize("wl", SHAPES, ids=[w.key for w in SHAPES])
+def test_steps_match_oracle(wl):
+    case = Case(wl)
+    K0 = case.st.K[:, :, : wl.T].clone()
+    V0 = case.st.V[:, :, : wl.T].clone()
+    rep = Report()
+    for _ in range(wl.steps):
+        case.step(wl.budget, rep=rep)
+    assert rep.units_checked == wl.steps * wl.B * wl.G
+    assert rep.max_out_err <= TOL[wl.dtype]
+    # the library never writes the cache
+    assert torch.equal(case.st.K[:, :, : wl.T], K0) and torch.equal(case.st.V[:, :, : wl.T], V0)
+    assert int(case.st.graph.dev_err.item()) == 0
+    print(f"{wl.key}: {rep}")
+
+
+@pytest.mark.parametrize("wl", SHAPES[:4], ids=[w.key for w in SHAPES[:4]])
+def test_budget_zero_takes_top_community(wl):
+    case = Case(wl)
+    case.step(0, update=False)
+    n_sel = case.st.sel.n_sel.cpu().numpy()
+    assert np.all(n_sel == 1)
+
+
+@pytest.mark.parametrize("wl", SHAPES[:5], ids=[w.key for w in SHAPES[:5]])
+def test_full_budget_equals_dense(wl):
+    case = Case(wl.replace(update=False))
+    q = synth.draw_queries(wl, case.draw, 0)
+    sparse = case.st.decode(q, wl.T).clone()
+    dense = case.st.dense(q)
+    torch.cuda.synchronize()
+    assert float((sparse - dense).abs().max()) <= TOL[wl.dtype]
+    n_tok = case.st.sel.n_tok.cpu().numpy()
+    assert np.all(n_tok == wl.T)
+    # and both match the oracle's dense softmax attention
+    K = case.st.K.double().cpu().numpy()
+    V = case.st.V.double().cpu().numpy()
+    qn = q.double().cpu().numpy()
+    gq = wl.Hq // wl.Hkv
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            o = O.attention(qn[b, h], K[b, h // gq], V[b, h // gq], np.arange(wl.T))
+            assert np.abs(o - dense[b, h].double().cpu().numpy()).max() <= TOL[wl.dtype]
+
+
+@pytest.mark.parametrize("T", [1, 7, 100, 4099, 20000])
+def test_dense_decode_lengths(T):
+    wl = small("dense_len", 30, T=max(T, 8), update=False, B=3)
+    case = Case(wl)
+    q = synth.draw_queries(wl, case.draw, 0)
+    case.st.T = T
+    dense = case.st.dense(q)
+    torch.cuda.synchronize()
+    K = case.st.K.double().cpu().numpy()
+    V = case.st.V.double().cpu().numpy()
+    qn = q.double().cpu().numpy()
+    for b in range(wl.B):
+        for h in range(0, wl.Hq, 5):
+            o = O.attention(qn[b, h], K[b, h // 4], V[b, h // 4], np.arange(T))
+            assert np.abs(o - dense[b, h].double().cpu().numpy()).max() <= TOL[wl.dtype]
+
+
+def test_no_sinks():
+    wl = small("no_sinks", 31, S=0)
+    case = Case(wl)
+    for _ in range(2):
+        case.step(wl.budget)
+
+
+def test_single_community():
+    wl = small("one_comm", 32, update=True)
+    labels = np.zeros((wl.B, wl.G, wl.T), dtype=np.int32)
+    labels[:, :, : wl.S] = -1
+    case = Case(wl, labels=labels)
+    case.check_build()
+    case.step(5)          # budget below the community size: the top community is still taken
+    assert np.all(case.st.sel.n_tok.cpu().numpy() == wl.T)
+    case.step(5)          # the token appended after the first step joined the only community
+    assert np.all(case.st.sel.n_tok.cpu().numpy() == wl.T + 1)
+
+
+def test_empty_ids_and_slack_capacity():
+    wl = small("gaps", 33)
+    labels = np.stack([synth.sequence_labels(wl, 0, b) for b in range(wl.B)])
+    labels = np.where(labels >= 0, labels * 3 + 1, -1).astype(np.int32)   # ids 1, 4, 7, ...
+    case = Case(wl, labels=labels, Cmax=int(labels.max()) + 50)
+    case.check_build()
+    for _ in range(2):
+        case.step(wl.budget)
+
+
+def test_tail_full_sets_error_and_skips():
+    wl = small("tail_full", 34, steps=3)
+    case = Case(wl, max_tail=1)
+    case.step(wl.budget)
+    assert int(case.st.graph.dev_err.item()) == 0
+    cnt0 = case.st.graph.cnt.clone()
+    cent0 = case.st.graph.cent.clone()
+    q = synth.draw_queries(wl, case.draw, 1)
+    case.st.decode(q, wl.budget)
+    kn, vn = synth.draw_new_tokens(wl, case.draw, 1)
+    assigned = case.st.append(kn, vn)
+    torch.cuda.synchronize()
+    assert int(case.st.graph.dev_err.item()) & 4
+    assert bool((assigned == -1).all())
+    assert torch.equal(case.st.graph.cnt, cnt0) and torch.equal(case.st.graph.cent, cent0)
+    assert bool((case.st.graph.comm_of[:, case.st.T - 1] == -1).all())
+
+
+def test_token_capacity_truncates_with_error():
+    wl = small("tok_cap", 35, update=False)
+    case = Case(wl, tok_cap=wl.S + 37)
+    case.step(wl.budget, update=False)
+    assert int(case.st.graph.dev_err.item()) & 8
+    assert np.all(case.st.sel.n_tok.cpu().numpy() == wl.S + 37)
+
+
+def test_bad_labels_are_flagged_and_skipped():
+    wl = small("bad_labels", 36, update=False, B=1)
+    labels = np.stack([synth.sequence_labels(wl, 0, b) for b in range(wl.B)])
+    C = int(labels.max()) + 1
+    bad = labels.copy()
+    bad[0, 0, 1] = 3          # a sink with a label
+    bad[0, 1, 100] = C + 5    # beyond Cmax
+    case = Case(wl, labels=bad, Cmax=C)
+    err = int(case.st.graph.dev_err.item())
+    assert err & 1 and err & 2
+    comm_of = case.st.graph.comm_of.cpu().numpy()
+    assert comm_of[0, 1] == -1 and comm_of[1, 100] == -1
+    assert int(case.st.graph.cnt.sum().item()) == wl.B * wl.G * (wl.T - wl.S) - 1
