@@ -164,19 +164,30 @@ class ClockSampler:
 # the CUDA arm
 # ----------------------------------------------------------------------------
 
-def union_rows(sel, U, G, Hq, Hkv, per_head: bool, T_cap: int) -> torch.Tensor:
-    """Distinct (sequence, KV head, position) rows a step's selection reads."""
-    n_tok = sel.n_tok.long()
-    if not per_head:
-        return n_tok.sum()
-    cap = sel.sel_tok.shape[1]
-    idx = torch.arange(cap, device=n_tok.device)[None, :]
-    valid = idx < n_tok[:, None]
-    gq = Hq // Hkv
-    units = torch.arange(U, device=n_tok.device)
-    group = (units // G) * Hkv + (units % G) // gq
-    key = group[:, None].long() * T_cap + sel.sel_tok.long()
-    return torch.unique(key[valid]).numel() * torch.ones((), dtype=torch.long, device=n_tok.device)
+class RowCounter:
+    """Distinct (sequence, KV head, position) rows a step's selection reads,
+    counted on the device without a host sync (a byte map per KV head)."""
+
+    def __init__(self, wl: synth.Workload, U: int, T_cap: int, cap: int, device):
+        self.per_head = wl.mode == "head"
+        self.T_cap = T_cap
+        units = torch.arange(U, device=device)
+        gq = wl.Hq // wl.Hkv
+        kv = (units // wl.G) * wl.Hkv + ((units % wl.G) // gq if self.per_head else units % wl.G)
+        self.base = (kv.long() * T_cap)[:, None]
+        self.col = torch.arange(cap, device=device)[None, :]
+        self.dummy = wl.B * wl.Hkv * T_cap
+        self.map = torch.zeros(self.dummy + 1, dtype=torch.uint8, device=device)
+
+    def __call__(self, sel) -> torch.Tensor:
+        n_tok = sel.n_tok.long()
+        if not self.per_head:
+            return n_tok.sum()
+        cap = self.col.shape[1]
+        key = torch.where(self.col < n_tok[:, None], self.base + sel.sel_tok[:, :cap].long(), self.dummy)
+        self.map.zero_()
+        self.map.index_fill_(0, key.reshape(-1), 1)
+        return self.map[: self.dummy].sum(dtype=torch.long)
 
 
 def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
@@ -231,6 +242,12 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         if ev:
             ev[3].record()
 
+    # a selection never holds more than S + max(budget, largest community) tokens
+    max_cnt = int(st.graph.cnt.max().item()) + (n_total if wl.update else 0)
+    cap = min(st.sel.sel_tok.shape[1], wl.S + max(budget, max_cnt))
+    count_rows = RowCounter(wl, U, T_cap, cap, device)
+    clock_sampler = ClockSampler(device.index).__enter__()
+    time.sleep(0.5)  # let the sampler start before the warm-up
     for i in range(W_steps):
         flush()
         one_step(i)
@@ -241,17 +258,19 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     barrier(device)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    with ClockSampler(device.index) as clk:
+    clk = clock_sampler
+    if True:
         for j in range(K_steps):
             flush()
             one_step(W_steps + j, evs[j])
-            rows_hist.append(union_rows(st.sel, U, wl.G, wl.Hq, wl.Hkv, per_head, T_cap))
+            rows_hist.append(count_rows(st.sel))
             ntok_hist.append(st.sel.n_tok.long().sum())
             ncomm_hist.append(num_comm.sum())
         torch.cuda.synchronize()
     barrier(device)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    clk.__exit__()
     clocks = clk.summary()
     if int(st.graph.dev_err.item()) != 0:
         raise RuntimeError(f"device error word {int(st.graph.dev_err.item())}")
@@ -463,10 +482,11 @@ def run_reference(args, wl: synth.Workload, device) -> dict:
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget", type=int, default=None)
+    ap.add_argument("--batch", type=int, default=None, help="override the batch (small profiling captures)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-units", type=int, default=48, help="graph units the CPU baseline times")
@@ -482,6 +502,8 @@ def main(argv=None):
     args = parse(argv)
     ws, rank, local = dist_env()
     wl = synth.WORKLOADS[args.workload]
+    if args.batch is not None:
+        wl = wl.replace(B=args.batch)
     if args.impl == "reference":
         if rank != 0:
             return 0

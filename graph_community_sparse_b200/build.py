@@ -1,6 +1,6 @@
 """Compile libckv.so in-tree for sm_100a with nvcc (no GPU needed).
 
-    python -m graph_community_sparse_b200.build [-v]
+    python graph_community_sparse_b200/build.py [-v] [-f]
 
 Objects go to graph_community_sparse_b200/_build/, the library to
 graph_community_sparse_b200/libckv.so.  Only the ckv_* C symbols are exported

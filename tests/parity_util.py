@@ -113,8 +113,17 @@ class Case:
 
     # oracle-side helpers -------------------------------------------------
     def state(self, b: int, g: int) -> O.GraphState:
+        """Oracle membership of one unit.  A unit first checked after some
+        updates starts from the labels plus the joins the GPU made meanwhile
+        (those joins were not checked; later counts and centres are)."""
         if (b, g) not in self.states:
-            self.states[(b, g)] = O.GraphState(self.draw.labels[b, g], self.wl.T_cap, self.wl.S, self.Cmax)
+            st = O.GraphState(self.draw.labels[b, g], self.st.cache.T_cap, self.wl.S, self.Cmax)
+            if self.st.T > self.wl.T:
+                u = b * self.wl.G + g
+                joined = self.st.graph.comm_of[u, self.wl.T: self.st.T].cpu().numpy()
+                for i, c in enumerate(joined):
+                    st.join(self.wl.T + i, int(c))
+            self.states[(b, g)] = st
         return self.states[(b, g)]
 
     def kv(self, b: int, kvh: int):
@@ -210,6 +219,10 @@ class Case:
                     assert abs(sr - sg) <= BAND, f"unit {u}: assignment {got} vs {ref}"
                     rep.resyncs += 1
                 st.join(pos, got)
+            checked = set(units)
+            for (b, g), st in self.states.items():
+                if (b, g) not in checked:       # tracked but not checked this step
+                    st.join(pos, int(assigned[b * wl.G + g]))
             # counts and centres after the update
             cnt_gpu = self.st.graph.cnt.cpu().numpy()
             cent_gpu = self.st.graph.cent.cpu().numpy()
