@@ -20,7 +20,7 @@ __all__ = [
     "CKVError", "lib", "LIB_PATH", "CacheDesc", "GraphDesc", "SelectionDesc",
     "Graph", "Selection", "cache_desc", "new_graph", "new_selection", "new_workspace",
     "ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-    "ckv_assign_update", "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
+    "ckv_sparse_decode_noalloc", "NOALLOC_SCRATCH_BYTES", "ckv_assign_update", "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP",
     "NEIGHBOURS",
@@ -33,8 +33,9 @@ PER_GROUP, PER_HEAD = 0, 1
 DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
 NEIGHBOURS = 8
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-            "ckv_assign_update", "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
-            "ckv_abi_version")
+            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_dense_decode", "ckv_status_string",
+            "ckv_last_error", "ckv_abi_version")
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class CKVError(RuntimeError):
@@ -44,7 +45,7 @@ class CKVError(RuntimeError):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libckv.so not built at {LIB_PATH}; run `python -m graph_community_sparse_b200.build`")
+    raise ImportError(f"libckv.so not built at {LIB_PATH}; run `python graph_community_sparse_b200/build.py`")
 lib = ctypes.CDLL(LIB_PATH)
 
 _i32, _i64, _p, _sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
@@ -73,10 +74,11 @@ lib.ckv_workspace_size.argtypes = [_P(CacheDesc), _P(GraphDesc), _P(SelectionDes
 lib.ckv_build_centroids.argtypes = [_P(CacheDesc), _p, _i64, _i32, _P(GraphDesc), _p, _sz, _p]
 lib.ckv_score_select.argtypes = [_P(CacheDesc), _P(GraphDesc), _p, _i32, _P(SelectionDesc), _p, _sz, _p]
 lib.ckv_sparse_decode.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p, _sz, _p]
+lib.ckv_sparse_decode_noalloc.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p]
 lib.ckv_assign_update.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p]
 lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
 for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-           "ckv_assign_update", "ckv_dense_decode"):
+           "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_dense_decode"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.ckv_status_string.argtypes = [ctypes.c_int]
 lib.ckv_status_string.restype = ctypes.c_char_p
@@ -235,6 +237,16 @@ def ckv_sparse_decode(cache: CacheDesc, q: torch.Tensor, graph: Graph, sel: Sele
                                  ctypes.byref(sel.desc), out.data_ptr(), _ptr(nbr8), ws.data_ptr(),
                                  ws.numel(), _stream(stream)),
            "ckv_sparse_decode")
+
+
+def ckv_sparse_decode_noalloc(cache: CacheDesc, q: torch.Tensor, graph: Graph, sel: Selection,
+                              out: torch.Tensor, nbr8: Optional[torch.Tensor], stream=None) -> None:
+    """ckv_sparse_decode for callers that cannot hand over a workspace: the
+    scratch is a fixed 32 MiB array inside the library (see include/ckv.h).
+    Calls must not overlap on the GPU."""
+    _check(lib.ckv_sparse_decode_noalloc(ctypes.byref(cache), q.data_ptr(), ctypes.byref(graph.desc),
+                                         ctypes.byref(sel.desc), out.data_ptr(), _ptr(nbr8), _stream(stream)),
+           "ckv_sparse_decode_noalloc")
 
 
 def ckv_assign_update(cache: CacheDesc, graph: Graph, pos: int, nbr8: torch.Tensor,

@@ -247,6 +247,34 @@ ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q, const c
                        "ckv_sparse_decode");
 }
 
+// Same validation and kernels as ckv_sparse_decode; the scratch is the
+// library's fixed array instead of a caller workspace, so nothing is
+// allocated.  Sizes whose scratch would not fit are refused up front.
+ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const void* q, const ckv_graph_desc* graph,
+                                     const ckv_selection_desc* sel, float* out, int32_t* nbr8,
+                                     ckv_stream_t stream) {
+    CKV_TRY(check_cache(cache, true));
+    CKV_TRY(check_graph(cache, graph));
+    const int64_t U = (int64_t)cache->B * graphs_per_seq(cache, graph);
+    CKV_TRY(check_sel(graph, sel, U));
+    if (!q || !out) return fail(CKV_ERR_INVALID_ARG, "q or out is NULL");
+    if (!aligned16(q) || !aligned16(out)) return fail(CKV_ERR_MISALIGNED, "q and out must be 16-byte aligned");
+    const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : cache->Hq / cache->Hkv;
+    const size_t need = ckv::decode_ws_bytes((int)U, gq, cache->d);
+    if (need > CKV_NOALLOC_SCRATCH_BYTES)
+        return fail(CKV_ERR_UNSUPPORTED,
+                    "ckv_sparse_decode_noalloc: these shapes need %zu bytes of scratch, above the library's "
+                    "fixed %zu; use ckv_sparse_decode with a workspace",
+                    need, (size_t)CKV_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    size_t have = 0;
+    cudaError_t e = ckv::static_decode_scratch(&scratch, &have);
+    if (e != cudaSuccess) return cuda_status(e, "ckv_sparse_decode_noalloc: scratch address lookup");
+    return cuda_status(ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q,
+                                                 out, nbr8, scratch, reinterpret_cast<cudaStream_t>(stream)),
+                       "ckv_sparse_decode_noalloc");
+}
+
 ckv_status ckv_assign_update(const ckv_cache_desc* cache, const ckv_graph_desc* graph, int32_t pos,
                              const int32_t* nbr8, int32_t* assigned, ckv_stream_t stream) {
     CKV_TRY(check_cache(cache, true));

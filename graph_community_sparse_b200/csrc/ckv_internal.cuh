@@ -227,6 +227,10 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
                                  const void* q, float* out, int32_t* nbr8, void* ws, cudaStream_t st);
 cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float* out, void* ws,
                                 cudaStream_t st);
+// Device address and size of the library's own decode scratch (looked up once
+// per device, with that device current).
+cudaError_t static_decode_scratch(void** ptr, size_t* bytes);
+
 cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const int32_t* nbr8,
                                  int32_t* assigned, cudaStream_t st);
 

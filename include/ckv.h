@@ -202,6 +202,34 @@ CKV_API ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q,
                              ckv_stream_t stream);
 
 /*
+ * ckv_sparse_decode without a workspace argument.  The paper has no
+ * counterpart: this exists for callers that cannot allocate device memory
+ * for scratch, for example a serving engine that has reserved almost all
+ * of HBM for its own KV pools and gives plug-ins no allocator, or a
+ * latency-critical decode loop that must not call cudaMalloc because it can
+ * synchronise the device.  Same arguments and results as ckv_sparse_decode,
+ * computed by the same kernels; the split-K scratch instead lives in a
+ * 32 MiB array inside libckv that every GPU which loads the library keeps
+ * until the process exits.
+ *   - Calls needing more scratch than CKV_NOALLOC_SCRATCH_BYTES (the size
+ *     ckv_workspace_size's attention part reports for these shapes; e.g.
+ *     Hq/Hkv = 8 with d = 128 in per-group mode) return CKV_ERR_UNSUPPORTED
+ *     before touching the device.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.  No call allocates or frees memory.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents (nothing in it needs to start at zero).  Calls that overlap
+ *     on the GPU, e.g. on two streams at once, race on it and give wrong
+ *     results: serialise them.
+ */
+#define CKV_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+CKV_API ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const void* q,
+                                             const ckv_graph_desc* graph,
+                                             const ckv_selection_desc* sel, float* out,
+                                             int32_t* nbr8, ckv_stream_t stream);
+
+/*
  * Local update for the token just written at position `pos` (its K/V rows are
  * already in the cache): in every graph unit it joins the candidate
  * community (the communities of nbr8) maximising k_new . cent_c / sqrt(d),
