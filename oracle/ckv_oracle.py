@@ -26,7 +26,7 @@ in that order:
    full cache, which is never pruned (same section, next paragraph).
 6. A new token joins one neighbouring community and one centre is updated, at
    a cost independent of the context length (same section, last paragraph;
-   abstract: "in constant time").  Rules used: the neighbour set is the
+   the abstract calls the rule constant-time).  Rules used: the neighbour set is the
    communities of the 8 non-sink selected tokens with the largest graph logit
    (max over the graph's heads of q_h . k_t / sqrt(d); ties to the lower
    position); the token joins the candidate c maximising k_new . c / sqrt(d)
