@@ -6,7 +6,7 @@
 One step = ckv_score_select + ckv_sparse_decode (+ the cache append and
 ckv_assign_update when the workload updates) for the whole batch of one
 layer, with inputs resident in HBM.  Every timed step is bracketed by CUDA
-events on the launching stream; L2 is flushed (a 256 MiB write) before each
+events on the launching stream; L2 is flushed (a 1 GiB write) before each
 step, outside the events.  Rank 0 prints one JSON line.  With N GPUs each rank
 runs its own batch (weak scaling, no collective on the data path); the value
 is N*K steps over the slowest rank's time.
@@ -37,7 +37,7 @@ import synth  # noqa: E402
 METRIC = "sparse decode steps/s at 128K ctx; achieved HBM GB/s vs B200 peak"
 DEFAULT_WORKLOAD = "qwen3_8b_128k_head"
 FALLBACK_HBM_GBS = 6650.0
-KERNELS_PER_STEP_UPDATE = 5   # score, select, decode main, decode merge, assign
+KERNELS_PER_STEP_UPDATE = 5   # score, select, attention, merge, assign
 KERNELS_PER_STEP_STATIC = 4
 
 
@@ -196,7 +196,11 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     K_steps, W_steps = args.steps, args.warmup
     budget = args.budget if args.budget is not None else wl.budget
     n_total = W_steps + K_steps + args.e2e_steps
-    extra = n_total + 8 if wl.update else 0
+    # Update workloads run in episodes of the workload's own length (e.g. 64
+    # generated tokens): the graph is rebuilt from the labels and the cache
+    # length reset between episodes, outside the timed events.
+    episode = wl.steps if wl.update else 0
+    extra = episode + 8 if wl.update else 0
     T_cap = wl.T + extra
     layer = rank  # per-rank seeds: each rank owns a different batch of sequences
     draw = synth.draw_cache(wl, layer=layer, device=device, T_cap=T_cap)
@@ -216,7 +220,9 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
 
     qs = [synth.draw_queries(wl, draw, i, layer) for i in range(n_total)]
     news = [synth.draw_new_tokens(wl, draw, i, layer) for i in range(n_total)] if wl.update else []
-    flush_buf = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)  # 256 MiB > L2
+    # 1 GiB > L2; its ~0.3 ms on the GPU also lets the host enqueue a whole step
+    # before the GPU reaches it, so the events time device work, not launch gaps
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.float32, device=device)
 
     def flush():
         flush_buf.fill_(1.0)
@@ -225,6 +231,12 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     row_bytes = 2 * wl.d * esz
     per_head = wl.mode == "head"
     num_comm = st.graph.num_comm.long()
+    episodes = [0]
+
+    def new_episode_if_due():
+        if wl.update and st.T - wl.T >= episode:
+            st.build(labels, wl.T)
+            episodes[0] += 1
 
     def one_step(i, ev=None):
         q = qs[i]
@@ -243,30 +255,34 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
             ev[3].record()
 
     # a selection never holds more than S + max(budget, largest community) tokens
-    max_cnt = int(st.graph.cnt.max().item()) + (n_total if wl.update else 0)
+    max_cnt = int(st.graph.cnt.max().item()) + extra
     cap = min(st.sel.sel_tok.shape[1], wl.S + max(budget, max_cnt))
     count_rows = RowCounter(wl, U, T_cap, cap, device)
     clock_sampler = ClockSampler(device.index).__enter__()
     time.sleep(0.5)  # let the sampler start before the warm-up
     for i in range(W_steps):
+        new_episode_if_due()
         flush()
         one_step(i)
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
     rows_hist, ntok_hist, ncomm_hist = [], [], []
+    host_s = 0.0
     barrier(device)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     clk = clock_sampler
-    if True:
-        for j in range(K_steps):
-            flush()
-            one_step(W_steps + j, evs[j])
-            rows_hist.append(count_rows(st.sel))
-            ntok_hist.append(st.sel.n_tok.long().sum())
-            ncomm_hist.append(num_comm.sum())
-        torch.cuda.synchronize()
+    for j in range(K_steps):
+        new_episode_if_due()
+        flush()
+        h0 = time.perf_counter()
+        one_step(W_steps + j, evs[j])
+        host_s += time.perf_counter() - h0
+        rows_hist.append(count_rows(st.sel))
+        ntok_hist.append(st.sel.n_tok.long().sum())
+        ncomm_hist.append(num_comm.sum())
+    torch.cuda.synchronize()
     barrier(device)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
@@ -348,6 +364,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         d2h = out_h.numel() * 4 + (nbr_h.numel() * 4 + asg_h.numel() * 4 if wl.update else 0)
         for j in range(args.e2e_steps):
             i = W_steps + K_steps + j
+            new_episode_if_due()
             flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -380,7 +397,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
                    "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
                    "communities_per_graph": float(ncomm / U), "budget": budget, "sinks": wl.S,
                    "update": wl.update, "layout": wl.layout,
-                   "l2": "flushed by a 256 MiB write before every timed step, outside the CUDA events",
+                   "l2": "flushed by a 1 GiB write before every timed step, outside the CUDA events",
                    "parallelism": f"dp{n_ranks} (independent batches, no collective)"},
         "tokens_per_s": value * wl.B,
         "roofline": roofline,
@@ -391,6 +408,8 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "clocks": clocks,
         "build_ms": build_ms,
         "wall_s_timed_region": wall,
+        "host_us_per_step": host_s / K_steps * 1e6,
+        "episodes": episodes[0],
     }
 
 

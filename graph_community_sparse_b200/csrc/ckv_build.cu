@@ -204,9 +204,10 @@ cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* 
     p.dev_err = g.dev_err;
     const int U = c.B * g.G;
     const size_t hsm = (size_t)g.Cmax * 4;
-    cudaError_t e = cudaFuncSetAttribute(build_hist, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm);
+    static LaunchCache lc_hist, lc_scatter;
+    cudaError_t e = prepare_launch(build_hist, lc_hist, hsm, 256, nullptr, nullptr);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(build_scatter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsm);
+    e = prepare_launch(build_scatter, lc_scatter, hsm, 32, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     build_hist<<<dim3(p.nchunks, U), 256, hsm, st>>>(p);
     build_scan<<<U, 1024, 0, st>>>(p);

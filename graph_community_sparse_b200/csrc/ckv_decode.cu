@@ -14,16 +14,21 @@
 // community sizes are.  A warp writes one partial (running max m, sum l,
 // unnormalised accumulator, top-8 logits) per unit segment into slot w + u,
 // which is unique because slices and units are both contiguous and ordered.
-// decode_merge then combines each unit's slots in a fixed order.
+// All warps of the persistent grid finish together, so the merge of each
+// unit's slots is a second, small kernel launched as a programmatic
+// dependent: its launch overlaps the attention kernel's tail and it waits
+// (in hardware, griddepcontrol) for that kernel's results; every operand is
+// fetched in one round of independent loads.
 //
 // Inside a warp: each half-warp owns one token row at a time, a lane owns
 // D/16 consecutive elements (16 bytes for bf16, d = 128); K and V rows of
 // 8 tokens per iteration are staged by cp.async into a per-warp ring of
-// DEC_STAGES iterations, so two iterations of loads are always in flight
-// while one is computed.  Logits of the GQA group's heads are reduced with a
-// value-exchanging butterfly; the softmax uses exp2 with log2(e)/sqrt(d)
-// folded into q and a lazily raised running max (raised only when a logit
-// exceeds it by more than 2^8), which is exact after the final division.
+// Stages<GQ> iterations (2 for one head per graph, where more resident warps
+// matter more, 3 otherwise), so loads stay in flight while one is computed.
+// Logits of the GQA group's heads are reduced with a value-exchanging
+// butterfly; the softmax uses exp2 with log2(e)/sqrt(d) folded into q and a
+// lazily raised running max (raised only when a logit exceeds it by more
+// than 2^8), which is exact after the final division.
 #include <math.h>
 
 #include "ckv_internal.cuh"
@@ -31,9 +36,12 @@
 namespace ckv {
 
 constexpr int DEC_WARPS = 4;
-constexpr int DEC_STAGES = 3;
 constexpr int TOK_PER_IT = 8;
 constexpr float RESCALE_THRESH = 8.0f;
+constexpr int MERGE_CHUNK = 128;  // slots whose weights are staged in shared memory at once
+
+template <int GQ> struct Stages { static constexpr int v = GQ == 1 ? 2 : 3; };
+template <int GQ> struct MinBlocks { static constexpr int v = GQ == 1 ? 6 : (GQ == 2 ? 5 : (GQ == 4 ? 4 : 2)); };
 
 template <typename T, int D>
 struct RowGeom {
@@ -46,7 +54,7 @@ struct RowGeom {
 template <typename T, int D, int GQ>
 struct DecSmem {
     static constexpr int PBUF = TOK_PER_IT * GQ * 4;
-    static constexpr int WARP = DEC_STAGES * 2 * RowGeom<T, D>::TILE + ((PBUF + 127) / 128) * 128;
+    static constexpr int WARP = Stages<GQ>::v * 2 * RowGeom<T, D>::TILE + ((PBUF + 127) / 128) * 128;
     static constexpr int CTA_FIXED = DEC_WARPS * WARP;
 };
 
@@ -109,6 +117,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
     using RG = RowGeom<T, D>;
     constexpr int E = RG::E, PART = RG::PART, ROW = RG::ROW, TILE = RG::TILE;
     constexpr int LG = Log2<GQ>::v;
+    constexpr int NS = Stages<GQ>::v;
     const int half = lane >> 4, l16 = lane & 15;
     const int hl = head_of_lane<GQ>(lane);
     const bool owner = (lane & ((16 >> LG) - 1)) == 0;
@@ -129,7 +138,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 
     const int n = hi - lo;
     const int nit = (n + TOK_PER_IT - 1) / TOK_PER_IT;
-    float* pbuf = reinterpret_cast<float*>(wsm + DEC_STAGES * 2 * TILE);
+    float* pbuf = reinterpret_cast<float*>(wsm + NS * 2 * TILE);
 
     int win_cur = 0, win_nxt = 0;
     if constexpr (!DENSE) {
@@ -137,8 +146,10 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
         win_nxt = (32 + lane < n) ? __ldg(toks + lo + 32 + lane) : 0;
     }
 
+    int stage_in = 0;  // ring slot the next issue() fills
     auto issue = [&](int it) {
-        unsigned char* kt = wsm + (it % DEC_STAGES) * 2 * TILE;
+        unsigned char* kt = wsm + stage_in * 2 * TILE;
+        stage_in = (stage_in + 1 == NS) ? 0 : stage_in + 1;
         unsigned char* vt = kt + TILE;
         if constexpr (!DENSE) {
             if (it > 0 && (it & 3) == 0) {
@@ -166,7 +177,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
     };
 
 #pragma unroll
-    for (int s = 0; s < DEC_STAGES - 1; ++s) {
+    for (int s = 0; s < NS - 1; ++s) {
         if (s < nit) issue(s);
         else cp_async_commit();
     }
@@ -180,14 +191,16 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
     float tv = -INFINITY, thr = -INFINITY;
     int tp = 0x7fffffff;
 
+    int stage_out = 0;  // ring slot computed in this iteration
     for (int it = 0; it < nit; ++it) {
         __syncwarp();
-        if (it + DEC_STAGES - 1 < nit) issue(it + DEC_STAGES - 1);
+        if (it + NS - 1 < nit) issue(it + NS - 1);
         else cp_async_commit();
-        cp_async_wait<DEC_STAGES - 1>();
+        cp_async_wait<NS - 1>();
 
-        const unsigned char* kt = wsm + (it % DEC_STAGES) * 2 * TILE;
+        const unsigned char* kt = wsm + stage_out * 2 * TILE;
         const unsigned char* vt = kt + TILE;
+        stage_out = (stage_out + 1 == NS) ? 0 : stage_out + 1;
 
         float s[4];
 #pragma unroll
@@ -317,11 +330,12 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 }
 
 template <typename T, int D, int GQ, bool DENSE>
-__global__ void __launch_bounds__(DEC_WARPS * 32) decode_main(DecodeParams p) {
+__global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(DecodeParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char* wsm = smem + warp * DecSmem<T, D, GQ>::WARP;
     int* s_pre = reinterpret_cast<int*>(smem + DecSmem<T, D, GQ>::CTA_FIXED);
+    const int w = blockIdx.x * DEC_WARPS + warp;
 
     int total;
     if constexpr (!DENSE) {
@@ -333,7 +347,6 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_main(DecodeParams p) {
     }
     if (total <= 0) return;
     const int per = (total + p.W - 1) / p.W;
-    const int w = blockIdx.x * DEC_WARPS + warp;
     const int start = w * per;
     if (start >= total) return;
     const int end = min(start + per, total);
@@ -360,10 +373,18 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_main(DecodeParams p) {
     }
 }
 
-// One block of D threads per unit: combine the unit's slots in slot order.
+// One block per unit: threads 0..D-1 own one output dimension each (all the
+// unit's heads); the extra warp merges the top-8 neighbour lists.  Slots are
+// combined in slot order, MERGE_CHUNK at a time, with every load of a chunk
+// issued before any is used.
 template <int D, int GQ, bool DENSE>
-__global__ void __launch_bounds__(D) decode_merge(DecodeParams p) {
-    const int u = blockIdx.x, d = threadIdx.x;
+__global__ void __launch_bounds__(D + 32) decode_merge(DecodeParams p) {
+    __shared__ float s_f[MERGE_CHUNK][GQ];
+    __shared__ float s_red[(D + 32) / 32][GQ];
+    __shared__ float s_M[GQ];
+    // wait until the attention kernel's partials are complete and visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int u = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     int b, kvh, h0;
     unit_heads(p, u, GQ, DENSE, b, kvh, h0);
     int ubeg, uend, total;
@@ -376,68 +397,144 @@ __global__ void __launch_bounds__(D) decode_merge(DecodeParams p) {
         uend = p.unit_prefix[u + 1];
         total = p.unit_prefix[p.U];
     }
+    float* outu = p.out + ((size_t)b * p.Hq + h0) * D;
     if (uend <= ubeg) {
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) p.out[((size_t)b * p.Hq + h0 + h) * D + d] = 0.f;
-        if (!DENSE && p.want_nbr && d < 8) p.nbr8[(size_t)u * 8 + d] = -1;
+        for (int i = t; i < GQ * D; i += blockDim.x) outu[i] = 0.f;
+        if (!DENSE && p.want_nbr && t < 8) p.nbr8[(size_t)u * 8 + t] = -1;
         return;
     }
     const int per = (total + p.W - 1) / p.W;
-    const int wf = ubeg / per, wl = (uend - 1) / per;
+    const int wf = ubeg / per, nslots = (uend - 1) / per - wf + 1;
+    const size_t s0 = (size_t)wf + u;
     const DecodeWs& ws = p.ws;
+
+    if (!DENSE && p.want_nbr && warp == D / 32) {
+        // candidates: 8 per slot; each lane keeps its best 8 in registers
+        // (value desc, position asc), then 8 warp-wide rounds pick the winners
+        float cv[8];
+        int cp[8];
 #pragma unroll
-    for (int h = 0; h < GQ; ++h) {
-        float M = -INFINITY;
-        for (int w = wf; w <= wl; ++w) M = fmaxf(M, ws.m[(size_t)(w + u) * GQ + h]);
-        float L = 0.f, A = 0.f;
-        for (int w = wf; w <= wl; ++w) {
-            const size_t s = (size_t)(w + u) * GQ + h;
-            const float f = exp2f(ws.m[s] - M);
-            L = fmaf(ws.l[s], f, L);
-            A = fmaf(ws.acc[s * D + d], f, A);
+        for (int r = 0; r < 8; ++r) {
+            cv[r] = -INFINITY;
+            cp[r] = 0x7fffffff;
         }
-        p.out[((size_t)b * p.Hq + h0 + h) * D + d] = A / L;
-    }
-    if constexpr (!DENSE) {
-        if (p.want_nbr && d < 32) {
-            const int lane = d;
-            const int ncand = (wl - wf + 1) * 8;
-            float pv = INFINITY;
-            int pp = -1;  // previous pick; the next pick ranks strictly below it
-            for (int r = 0; r < 8; ++r) {
-                float bv = -INFINITY;
-                int bp = 0x7fffffff;
-                for (int i = lane; i < ncand; i += 32) {
-                    const size_t s = (size_t)(wf + (i >> 3) + u) * 8 + (i & 7);
-                    const int cp = ws.tp[s];
-                    if (cp < 0) continue;
-                    const float cv = ws.tv[s];
-                    const bool below_prev = (cv < pv) || (cv == pv && cp > pp);
-                    const bool better = (cv > bv) || (cv == bv && cp < bp);
-                    if (below_prev && better) {
-                        bv = cv;
-                        bp = cp;
-                    }
-                }
+        for (int i = lane; i < nslots * 8; i += 32) {
+            const size_t sl = (s0 + (i >> 3)) * 8 + (i & 7);
+            float v = ws.tv[sl];
+            int q = ws.tp[sl];
+            if (q < 0) continue;
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    const float ov = __shfl_xor_sync(FULL, bv, o);
-                    const int op = __shfl_xor_sync(FULL, bp, o);
-                    if (ov > bv || (ov == bv && op < bp)) {
-                        bv = ov;
-                        bp = op;
-                    }
+            for (int r = 0; r < 8; ++r) {
+                const bool better = (v > cv[r]) || (v == cv[r] && q < cp[r]);
+                const float v2 = better ? cv[r] : v;
+                const int q2 = better ? cp[r] : q;
+                if (better) {
+                    cv[r] = v;
+                    cp[r] = q;
                 }
-                const int outp = (bp == 0x7fffffff) ? -1 : bp;
-                if (lane == 0) p.nbr8[(size_t)u * 8 + r] = outp;
-                if (outp >= 0) {
-                    pv = bv;
-                    pp = bp;
-                } else {
-                    pv = -INFINITY;
-                    pp = 0x7fffffff;
+                v = v2;
+                q = q2;
+            }
+        }
+        int head = 0;  // this lane's best remaining candidate
+        for (int r = 0; r < 8; ++r) {
+            float bv = -INFINITY;
+            int bp = 0x7fffffff;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k == head) {
+                    bv = cv[k];
+                    bp = cp[k];
+                }
+            float wv = bv;
+            int wp = bp;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const float ov = __shfl_xor_sync(FULL, wv, o);
+                const int op = __shfl_xor_sync(FULL, wp, o);
+                if (ov > wv || (ov == wv && op < wp)) {
+                    wv = ov;
+                    wp = op;
                 }
             }
+            const bool valid = wp != 0x7fffffff;
+            if (lane == 0) p.nbr8[(size_t)u * 8 + r] = valid ? wp : -1;
+            if (valid && bp == wp) ++head;  // positions are unique: only the owner advances
+        }
+    }
+
+    // running max per head over all slots
+    float M[GQ];
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) M[h] = -INFINITY;
+    for (int sl = t; sl < nslots; sl += blockDim.x)
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) M[h] = fmaxf(M[h], ws.m[(s0 + sl) * GQ + h]);
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(FULL, M[h], o));
+        if (lane == 0) s_red[warp][h] = M[h];
+    }
+    __syncthreads();
+    if (t < GQ) {
+        float m = -INFINITY;
+        for (int w2 = 0; w2 < (int)(blockDim.x >> 5); ++w2) m = fmaxf(m, s_red[w2][t]);
+        s_M[t] = m;
+    }
+    __syncthreads();
+
+    float A[GQ], Lp[GQ];
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) {
+        A[h] = 0.f;
+        Lp[h] = 0.f;
+    }
+    for (int c0 = 0; c0 < nslots; c0 += MERGE_CHUNK) {
+        const int cnt = min(MERGE_CHUNK, nslots - c0);
+        for (int i = t; i < cnt; i += blockDim.x) {
+#pragma unroll
+            for (int h = 0; h < GQ; ++h) {
+                const size_t sl = (s0 + c0 + i) * GQ + h;
+                const float f = exp2f(ws.m[sl] - s_M[h]);
+                s_f[i][h] = f;
+                Lp[h] = fmaf(ws.l[sl], f, Lp[h]);
+            }
+        }
+        __syncthreads();
+        if (t < D) {
+            int j = 0;
+            for (; j + 8 <= cnt; j += 8) {
+                float x[8][GQ];
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int h = 0; h < GQ; ++h) x[r][h] = ws.acc[((s0 + c0 + j + r) * GQ + h) * D + t];
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int h = 0; h < GQ; ++h) A[h] = fmaf(x[r][h], s_f[j + r][h], A[h]);
+            }
+            for (; j < cnt; ++j)
+#pragma unroll
+                for (int h = 0; h < GQ; ++h) A[h] = fmaf(ws.acc[((s0 + c0 + j) * GQ + h) * D + t], s_f[j][h], A[h]);
+        }
+        __syncthreads();
+    }
+    // sum of the weights per head
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) Lp[h] += __shfl_xor_sync(FULL, Lp[h], o);
+        if (lane == 0) s_red[warp][h] = Lp[h];
+    }
+    __syncthreads();
+    if (t < D) {
+#pragma unroll
+        for (int h = 0; h < GQ; ++h) {
+            float L = 0.f;
+            for (int w2 = 0; w2 < (int)(blockDim.x >> 5); ++w2) L += s_red[w2][h];
+            outu[h * D + t] = A[h] / L;
         }
     }
 }
@@ -469,32 +566,14 @@ DecodeWs carve_decode_ws(void* ws, int U, int gq, int d) {
 
 namespace {
 
-struct DevInfo {
-    int sms = 0;
-};
-
-int device_sms() {
-    static DevInfo info[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (info[dev].sms == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        info[dev].sms = n;
-    }
-    return info[dev].sms;
-}
-
 template <typename T, int D, int GQ, bool DENSE>
 cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
+    static LaunchCache lc;
     auto kern = decode_main<T, D, GQ, DENSE>;
     const size_t smem = DecSmem<T, D, GQ>::CTA_FIXED + (DENSE ? 0 : (size_t)(p.U + 1) * 4);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int per_sm = 0, sms = 0;
+    cudaError_t e = prepare_launch(kern, lc, smem, DEC_WARPS * 32, &per_sm, &sms);
     if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, DEC_WARPS * 32, smem);
-    if (e != cudaSuccess) return e;
-    const int sms = device_sms();
     if (sms <= 0 || per_sm <= 0) return cudaErrorInvalidConfiguration;
     int blocks = sms * per_sm;
     if (blocks * DEC_WARPS > MAX_DECODE_WARPS) blocks = MAX_DECODE_WARPS / DEC_WARPS;
@@ -502,8 +581,18 @@ cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
     kern<<<blocks, DEC_WARPS * 32, smem, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    decode_merge<D, GQ, DENSE><<<p.U, D, 0, st>>>(p);
-    return cudaGetLastError();
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.U);
+    cfg.blockDim = dim3(D + 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_merge<D, GQ, DENSE>, p);
 }
 
 template <bool DENSE>

@@ -236,4 +236,46 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Launch-shape cache for one kernel: the dynamic shared memory limit it was
+// raised to and its resident blocks per SM, per device, so that steady-state
+// calls make no attribute or occupancy queries (only launches).
+struct LaunchCache {
+    int smem_set[64] = {};   // largest dynamic smem the attribute allows (bytes)
+    int occ_smem[64] = {};   // smem the occupancy below was computed for (+1)
+    int occ_blocks[64] = {};
+    int sms[64] = {};
+};
+
+template <typename Kern>
+inline cudaError_t prepare_launch(Kern kern, LaunchCache& lc, size_t smem, int threads, int* blocks_per_sm,
+                                  int* sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (lc.sms[dev] == 0) {
+        int n = 0;
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        lc.sms[dev] = n;
+    }
+    if ((int)smem > lc.smem_set[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        lc.smem_set[dev] = (int)smem;
+    }
+    if (blocks_per_sm) {
+        if (lc.occ_smem[dev] != (int)smem + 1) {
+            int nb = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, threads, smem);
+            if (e != cudaSuccess) return e;
+            lc.occ_blocks[dev] = nb;
+            lc.occ_smem[dev] = (int)smem + 1;
+        }
+        *blocks_per_sm = lc.occ_blocks[dev];
+    }
+    if (sms) *sms = lc.sms[dev];
+    return cudaSuccess;
+}
+
 }  // namespace ckv

@@ -6,49 +6,119 @@
 // re-clustering", paragraph 4); the active token budget is small (section
 // "The speed-up depends on how many graphs the model stores").
 //
-// score_kernel: s_c = max over the graph's query heads of q_h . cent_c /
-//   sqrt(d).  A streaming matrix-vector product over the fp32 centres: one
-//   half-warp per centre row, 16-byte loads, the same value-exchanging
-//   butterfly as the attention kernel for the head sums.
-// select_kernel: one block per graph unit.  Keys (orderable score << 32 |
-//   ~id) are sorted descending in shared memory (bitonic), the sizes are
-//   prefix-summed in rank order and the longest prefix within the budget is
-//   kept (at least the top community).  The block then writes the unit's
-//   token list: sinks, build-time members of each selected community (copied
-//   from the community-contiguous CSR), then the selected tail members.  The
-//   last block to finish (atomic ticket; no block ever waits) writes the
-//   exclusive prefix of the token counts over units for the attention
-//   kernel's work split.
+// Two kernels, 8 warps per block:
+//  * score_kernel, grid (centre blocks of 64, units): s_c = max over the
+//    graph's query heads of q_h . cent_c / sqrt(d), a streaming
+//    matrix-vector product over the fp32 centres (one half-warp per row,
+//    16-byte loads, the value-exchanging butterfly of the attention kernel
+//    for the head sums).  Each score is stored and its community size is
+//    added, with a global atomic, to a per-unit histogram over the top 12
+//    bits of its key, key = (orderable score << 32) | ~id (unique; orders
+//    communities by score desc, id asc);
+//  * select_kernel, one block per unit, launched as a programmatic
+//    dependent (its launch overlaps the scoring; it waits in hardware for the
+//    scores): the histogram gives the bin the budget cut falls in; only the
+//    keys from that bin up (typically a few dozen) are sorted, in registers;
+//    a scan of their sizes gives the cut (at least the top community).  Then
+//    the unit's token list: sinks, build-time members of each selected
+//    community (from the community-contiguous CSR), then the selected tail
+//    members.  The last unit done (arrival counter; no block ever waits)
+//    writes the exclusive prefix of the token counts over units for the
+//    attention kernel's work split.
+// Histograms and the counter are zeroed by one memset issued in the same call.
 #include <math.h>
 
 #include "ckv_internal.cuh"
 
 namespace ckv {
 
-constexpr int SCORE_ROWS = 64;      // centres per block (8 warps x 8 rows)
-constexpr int SEL_THREADS = 1024;
+constexpr int SEL_WARPS = 8;
+constexpr int SEL_THREADS = SEL_WARPS * 32;
+constexpr int SCORE_ROWS = SEL_WARPS * 8;  // centres per block
+constexpr int SEL_HBITS = 12;
+constexpr int SEL_HBINS = 1 << SEL_HBITS;
+constexpr int SEL_FAST = SEL_THREADS;       // candidates sorted in registers
 
-struct ScoreParams {
+struct SelectParams {
     const void* q;
     const float* cent;
+    float* scores;              // [U, Cmax]
+    int32_t* hist;              // [U, SEL_HBINS]
+    int32_t* tickets;           // [U + 1]
+    unsigned long long* gkey;   // [U, npow_max] scratch for large candidate sets
+    int32_t* gw;                // [U, npow_max]
+    const int32_t* cnt;
+    const int32_t* offs;
+    const int32_t* tok;
     const int32_t* num_comm;
-    float* scores;
-    int32_t* counter;
-    int Hq, Hkv, G, per_head, Cmax;
+    const int32_t* tail_tok;
+    const int32_t* tail_comm;
+    const int32_t* tail_len;
+    int32_t* dev_err;
+    int32_t* sel_comm;
+    int32_t* n_sel;
+    int32_t* sel_tok;
+    int32_t* n_tok;
+    int32_t* unit_prefix;
+    int Hq, G, per_head;
     float inv_sqrt_d;
+    int U, Cmax, npow_max, S, T_cap, max_tail, tok_cap, budget;
 };
 
+__device__ __forceinline__ unsigned long long score_key(float s, int c) {
+    unsigned int b = __float_as_uint(s);
+    b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)b << 32) | (unsigned long long)(0xffffffffu - (unsigned)c);
+}
+
+__device__ __forceinline__ int key_id(unsigned long long k) {
+    return (int)(0xffffffffu - (unsigned)(k & 0xffffffffull));
+}
+
+// In-place inclusive scan of n ints (shared or global memory, visible to the
+// whole block); returns the total.
+__device__ int block_scan_inplace(int* a, int n, int* s_warp) {
+    const int nt = blockDim.x;
+    const int seg = (n + nt - 1) / nt;
+    const int b0 = min(n, threadIdx.x * seg), b1 = min(n, b0 + seg);
+    int sum = 0;
+    for (int i = b0; i < b1; ++i) sum += a[i];
+    int total;
+    int run = block_exclusive_scan(sum, s_warp, &total);
+    for (int i = b0; i < b1; ++i) {
+        run += a[i];
+        a[i] = run;
+    }
+    __syncthreads();
+    return total;
+}
+
+// Bitonic sort of one (key, weight) pair per lane across a warp, keys descending.
+__device__ __forceinline__ void warp_sort_desc(unsigned long long& v, int& w, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(FULL, v, j);
+            const int ow = __shfl_xor_sync(FULL, w, j);
+            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+            const bool take = keep_max ? (o > v) : (o < v);
+            if (take) {
+                v = o;
+                w = ow;
+            }
+        }
+    }
+}
+
+// Scores of this block's (up to) SCORE_ROWS centres of unit u.
 template <typename T, int D, int GQ>
-__global__ void __launch_bounds__(256) score_kernel(ScoreParams p) {
+__device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) {
     constexpr int E = D / 16;
-    const int u = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int half = lane >> 4, l16 = lane & 15;
-    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.counter = 0;
-    const int C = p.num_comm[u];
     const int row0 = blockIdx.x * SCORE_ROWS + warp * 8;
     if (row0 >= C) return;
-
     const int b = u / p.G, g = u - b * p.G;
     const int h0 = p.per_head ? g : g * GQ;
     float qr[GQ][E];
@@ -67,6 +137,8 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreParams p) {
             for (int e = 0; e < E; ++e) x[j][e] = 0.f;
         }
     }
+    const int wc = (lane < 8 && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
+    int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         float part[GQ];
@@ -78,129 +150,183 @@ __global__ void __launch_bounds__(256) score_kernel(ScoreParams p) {
             part[h] = a;
         }
         float s = halfwarp_reduce_heads<GQ>(part, lane);
-        s = halfwarp_max_over_heads<GQ>(s);
+        s = halfwarp_max_over_heads<GQ>(s) * p.inv_sqrt_d;
         const int c = row0 + 2 * j + half;
-        if (l16 == 0 && c < C) p.scores[(size_t)u * p.Cmax + c] = s * p.inv_sqrt_d;
+        const int w = __shfl_sync(FULL, wc, 2 * j + half);
+        if (l16 == 0 && c < C) {
+            p.scores[(size_t)u * p.Cmax + c] = s;
+            if (w > 0) atomicAdd(hist + (int)(score_key(s, c) >> (64 - SEL_HBITS)), w);
+        }
     }
 }
 
-struct SelectParams {
-    const float* scores;
-    const int32_t* cnt;
-    const int32_t* offs;
-    const int32_t* tok;
-    const int32_t* num_comm;
-    const int32_t* tail_tok;
-    const int32_t* tail_comm;
-    const int32_t* tail_len;
-    int32_t* dev_err;
-    int32_t* sel_comm;
-    int32_t* n_sel;
-    int32_t* sel_tok;
-    int32_t* n_tok;
-    int32_t* unit_prefix;
-    int32_t* counter;
-    int U, Cmax, npow_max, S, T_cap, max_tail, tok_cap, budget;
-};
-
-__device__ __forceinline__ unsigned long long score_key(float s, int c) {
-    unsigned int b = __float_as_uint(s);
-    b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-    return ((unsigned long long)b << 32) | (unsigned long long)(0xffffffffu - (unsigned)c);
-}
-
-// In-place inclusive scan of n ints in shared memory; returns the total.
-__device__ int block_scan_inplace(int* a, int n, int* s_warp) {
-    const int nt = blockDim.x;
-    const int seg = (n + nt - 1) / nt;
-    const int b0 = min(n, threadIdx.x * seg), b1 = min(n, b0 + seg);
-    int sum = 0;
-    for (int i = b0; i < b1; ++i) sum += a[i];
-    int total;
-    int run = block_exclusive_scan(sum, s_warp, &total);
-    for (int i = b0; i < b1; ++i) {
-        run += a[i];
-        a[i] = run;
-    }
-    __syncthreads();
-    return total;
-}
-
-__global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    unsigned long long* key = reinterpret_cast<unsigned long long*>(smem);
-    int* sz = reinterpret_cast<int*>(key + p.npow_max);
-    unsigned* mask = reinterpret_cast<unsigned*>(sz + p.npow_max);
+// Selection for unit u after all its scores are in (see the file comment).
+// Scores and the histogram were written by other blocks: read through L2.
+__device__ void select_unit(const SelectParams& p, int u, int C) {
+    __shared__ unsigned long long s_key[SEL_FAST];
+    __shared__ int s_w[SEL_FAST];
+    __shared__ unsigned long long s_runs[SEL_FAST];
+    __shared__ int s_bsz[SEL_FAST];
+    __shared__ int s_ofs[SEL_FAST];
+    __shared__ unsigned s_mask[MAX_CMAX / 32];
     __shared__ int s_warp[33];
-    __shared__ int s_kstar, s_last;
+    __shared__ int s_bstar, s_nc, s_nt, s_cnt;
 
-    const int u = blockIdx.x;
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
-    const int C = min(p.num_comm[u], p.Cmax);
-    int np = 1;
-    while (np < C) np <<= 1;
-
     const float* sc = p.scores + (size_t)u * p.Cmax;
     const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
-    for (int i = tid; i < np; i += nt) key[i] = (i < C && cn[i] > 0) ? score_key(sc[i], i) : 0ull;
-    for (int i = tid; i < (p.Cmax + 31) / 32; i += nt) mask[i] = 0u;
-    if (tid == 0) s_kstar = 0;
-    __syncthreads();
+    const int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
+    for (int i = tid; i < (p.Cmax + 31) / 32; i += nt) s_mask[i] = 0u;
+    if (tid == 0) {
+        s_bstar = -1;
+        s_nc = 0;
+        s_cnt = 0;
+    }
 
-    // bitonic sort, descending
-    for (int k = 2; k <= np; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int pi = tid; pi < (np >> 1); pi += nt) {
-                const int i = ((pi / j) * 2 * j) + (pi % j);
-                const int ixj = i + j;
-                const unsigned long long a = key[i], bb = key[ixj];
-                const bool desc = (i & k) == 0;
-                if (desc ? (a < bb) : (a > bb)) {
-                    key[i] = bb;
-                    key[ixj] = a;
+    // 1. crossing bin: thread t owns bins [per*t, per*t + per)
+    {
+        constexpr int per = SEL_HBINS / SEL_THREADS;
+        int hw[per];
+        int own = 0;
+#pragma unroll
+        for (int i = 0; i < per; ++i) {
+            hw[i] = __ldcg(hist + per * tid + i);
+            own += hw[i];
+        }
+        int total;
+        const int pre = block_exclusive_scan(own, s_warp, &total);  // also orders the inits above
+        int above = total - pre - own;  // weight of every bin above this thread's
+#pragma unroll
+        for (int i = per - 1; i >= 0; --i) {
+            if (above + hw[i] > p.budget) {
+                atomicMax(&s_bstar, per * tid + i);
+                break;
+            }
+            above += hw[i];
+        }
+    }
+    __syncthreads();
+    const int bstar = max(s_bstar, 0);  // no crossing: every key is a candidate
+
+    // 2. candidates: keys from the crossing bin up, with their sizes (the
+    //    loads of a round are all issued before any is used)
+    constexpr int RND = 8;
+    for (int c0 = tid; c0 < C; c0 += RND * nt) {
+        int wv[RND];
+        float sv[RND];
+#pragma unroll
+        for (int r = 0; r < RND; ++r) {
+            const int c = c0 + r * nt;
+            wv[r] = c < C ? cn[c] : 0;
+            sv[r] = c < C ? __ldcg(sc + c) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < RND; ++r) {
+            const int c = c0 + r * nt;
+            if (wv[r] <= 0) continue;
+            const unsigned long long k = score_key(sv[r], c);
+            if ((int)(k >> (64 - SEL_HBITS)) >= bstar) {
+                const int i = atomicAdd(&s_nc, 1);
+                if (i < SEL_FAST) {
+                    s_key[i] = k;
+                    s_w[i] = wv[r];
                 }
             }
-            __syncthreads();
         }
     }
-
-    // sizes in rank order, inclusive prefix, cut
-    for (int i = tid; i < np; i += nt) {
-        const unsigned long long kk = key[i];
-        sz[i] = kk ? cn[0xffffffffu - (unsigned)(kk & 0xffffffffull)] : 0;
-    }
     __syncthreads();
-    block_scan_inplace(sz, np, s_warp);
-    for (int i = tid; i < np; i += nt) {
-        const bool in_i = key[i] != 0ull && sz[i] <= p.budget;
-        const bool in_n = (i + 1 < np) && key[i + 1] != 0ull && sz[i + 1] <= p.budget;
-        if (in_i && !in_n) s_kstar = i + 1;
-    }
-    __syncthreads();
-    int kstar = s_kstar;
-    if (kstar == 0 && np > 0 && key[0] != 0ull) kstar = 1;
+    const int nc = s_nc;
 
+    int kstar;
+    const unsigned long long* sorted;
+    if (nc <= SEL_FAST) {
+        unsigned long long v = tid < nc ? s_key[tid] : 0ull;
+        int w = tid < nc ? s_w[tid] : 0;
+        warp_sort_desc(v, w, lane);
+        s_runs[tid] = v;
+        __syncthreads();
+        if (v) {
+            int r = lane;
+            for (int w2 = 0; w2 < nw; ++w2) {
+                if (w2 == warp) continue;
+                const unsigned long long* run = s_runs + 32 * w2;
+                int lo = 0, hi = 32;  // count of entries > v (runs are descending)
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (run[mid] > v) lo = mid + 1;
+                    else hi = mid;
+                }
+                r += lo;
+            }
+            s_key[r] = v;  // every s_key read happened before the barrier
+            s_w[r] = w;
+        }
+        __syncthreads();
+        const int ws = tid < nc ? s_w[tid] : 0;
+        int tot;
+        const int inc = block_exclusive_scan(ws, s_warp, &tot) + ws;
+        kstar = __syncthreads_count(tid < nc && inc <= p.budget);
+        sorted = s_key;
+    } else {
+        // rare: more candidates than one register sort holds; sort them in
+        // global scratch (block-wide bitonic, barriers between stages)
+        unsigned long long* gk = p.gkey + (size_t)u * p.npow_max;
+        int* gw = p.gw + (size_t)u * p.npow_max;
+        if (tid == 0) s_nc = 0;
+        __syncthreads();
+        for (int c = tid; c < C; c += nt) {
+            const int w = cn[c];
+            if (w <= 0) continue;
+            const unsigned long long k = score_key(__ldcg(sc + c), c);
+            if ((int)(k >> (64 - SEL_HBITS)) >= bstar) gk[atomicAdd(&s_nc, 1)] = k;
+        }
+        __syncthreads();
+        int np2 = 1;
+        while (np2 < nc) np2 <<= 1;
+        for (int i = nc + tid; i < np2; i += nt) gk[i] = 0ull;
+        __syncthreads();
+        for (int k = 2; k <= np2; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int pi = tid; pi < (np2 >> 1); pi += nt) {
+                    const int i = ((pi / j) * 2 * j) + (pi % j);
+                    const int ixj = i + j;
+                    const unsigned long long a = gk[i], bb = gk[ixj];
+                    if (((i & k) == 0) ? (a < bb) : (a > bb)) {
+                        gk[i] = bb;
+                        gk[ixj] = a;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        for (int i = tid; i < nc; i += nt) gw[i] = cn[key_id(gk[i])];
+        __syncthreads();
+        block_scan_inplace(gw, nc, s_warp);
+        int mine = 0;
+        for (int i = tid; i < nc; i += nt) mine += gw[i] <= p.budget;
+        atomicAdd(&s_cnt, mine);
+        __syncthreads();
+        kstar = s_cnt;
+        sorted = gk;
+    }
+    if (kstar == 0 && nc > 0) kstar = 1;  // the top community alone exceeds the budget: take it
+
+    // 3. ranked ids, membership mask, build-time run sizes in rank order
     int32_t* selc = p.sel_comm + (size_t)u * p.Cmax;
-    for (int i = tid; i < kstar; i += nt) {
-        const int c = (int)(0xffffffffu - (unsigned)(key[i] & 0xffffffffull));
-        selc[i] = c;
-        atomicOr(&mask[c >> 5], 1u << (c & 31));
-    }
-    __syncthreads();
-
-    // build-time member counts in rank order -> exclusive offsets
     const int32_t* of = p.offs + (size_t)u * (p.Cmax + 1);
-    for (int i = tid; i < np; i += nt) {
-        int v = 0;
-        if (i < kstar) {
-            const int c = selc[i];
-            v = of[c + 1] - of[c];
-        }
-        sz[i] = v;
+    const bool small = kstar <= SEL_FAST;
+    int* bsz = small ? s_bsz : p.gw + (size_t)u * p.npow_max;
+    for (int i = tid; i < kstar; i += nt) {
+        const int c = key_id(sorted[i]);
+        selc[i] = c;
+        atomicOr(&s_mask[c >> 5], 1u << (c & 31));
+        const int o0 = of[c];
+        bsz[i] = of[c + 1] - o0;
+        if (small) s_ofs[i] = o0;
     }
     __syncthreads();
-    const int nb = block_scan_inplace(sz, np, s_warp);  // inclusive
+    const int nb = block_scan_inplace(bsz, kstar, s_warp);  // inclusive
 
     int32_t* out = p.sel_tok + (size_t)u * p.tok_cap;
     const int32_t* tk = p.tok + (size_t)u * p.T_cap;
@@ -209,64 +335,111 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
         if (i < p.tok_cap) out[i] = i;
         else overflow = true;
     }
-    for (int k = warp; k < kstar; k += nw) {
-        const int c = selc[k];
-        const int len = of[c + 1] - of[c];
-        const int dst = p.S + sz[k] - len;
-        const int src = of[c];
-        for (int i = lane; i < len; i += 32) {
-            if (dst + i < p.tok_cap) out[dst + i] = tk[src + i];
-            else overflow = true;
+    if (small) {
+        // one token per thread per round: its run is found by binary search in
+        // the inclusive run prefix; a round's loads are issued before its stores
+        for (int t0 = tid; t0 < nb; t0 += RND * nt) {
+            int val[RND];
+#pragma unroll
+            for (int r = 0; r < RND; ++r) {
+                const int t = t0 + r * nt;
+                val[r] = 0;
+                if (t < nb) {
+                    int lo = 0, hi = kstar - 1;  // first k with bsz[k] > t
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        if (bsz[mid] > t) hi = mid;
+                        else lo = mid + 1;
+                    }
+                    const int start = lo ? bsz[lo - 1] : 0;
+                    val[r] = tk[s_ofs[lo] + (t - start)];
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RND; ++r) {
+                const int t = t0 + r * nt;
+                if (t < nb) {
+                    if (p.S + t < p.tok_cap) out[p.S + t] = val[r];
+                    else overflow = true;
+                }
+            }
+        }
+    } else {
+        for (int k = warp; k < kstar; k += nw) {
+            const int c = key_id(sorted[k]);
+            const int len = of[c + 1] - of[c];
+            const int dst = p.S + bsz[k] - len;
+            const int src = of[c];
+            for (int i = lane; i < len; i += 32) {
+                if (dst + i < p.tok_cap) out[dst + i] = tk[src + i];
+                else overflow = true;
+            }
         }
     }
-    __shared__ int s_nt;
-    if (warp == 0) {
+    {
+        // tail members of the selected communities, in tail order: the whole
+        // block flags one entry per thread per round and compacts by a scan
         const int tl = min(p.tail_len[u], p.max_tail);
         const int32_t* tt = p.tail_tok + (size_t)u * p.max_tail;
         const int32_t* tc = p.tail_comm + (size_t)u * p.max_tail;
         int base = p.S + nb;
-        for (int c0 = 0; c0 < tl; c0 += 32) {
-            const int i = c0 + lane;
-            bool in = false;
+        for (int c0 = 0; c0 < tl; c0 += nt) {
+            const int i = c0 + tid;
+            int in = 0;
             if (i < tl) {
                 const int c = tc[i];
-                in = c >= 0 && c < p.Cmax && ((mask[c >> 5] >> (c & 31)) & 1u);
+                in = c >= 0 && c < p.Cmax && ((s_mask[c >> 5] >> (c & 31)) & 1u);
             }
-            const unsigned bal = __ballot_sync(FULL, in);
+            int total;
+            const int off = block_exclusive_scan(in, s_warp, &total);
             if (in) {
-                const int dst = base + __popc(bal & ((1u << lane) - 1u));
+                const int dst = base + off;
                 if (dst < p.tok_cap) out[dst] = tt[i];
                 else overflow = true;
             }
-            base += __popc(bal);
+            base += total;
         }
-        if (lane == 0) s_nt = base;
+        if (tid == 0) s_nt = base;
     }
     if (__syncthreads_or(overflow) && tid == 0) atomicOr(p.dev_err, CKV_DEVERR_TOKEN_CAP);
-
     if (tid == 0) {
         p.n_sel[u] = kstar;
         p.n_tok[u] = min(s_nt, p.tok_cap);
-        __threadfence();
-        const int t = atomicAdd(p.counter, 1);
-        s_last = (t == (int)gridDim.x - 1);
     }
+}
+
+template <typename T, int D, int GQ>
+__global__ void __launch_bounds__(SEL_THREADS) score_kernel(SelectParams p) {
+    const int u = blockIdx.y;
+    const int C = min(p.num_comm[u], p.Cmax);
+    score_rows<T, D, GQ>(p, u, C);
+}
+
+__global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
+    __shared__ int s_last;
+    __shared__ int s_warp2[33];
+    // wait until every score and histogram update of the scoring kernel is visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int u = blockIdx.x, tid = threadIdx.x;
+    const int C = min(p.num_comm[u], p.Cmax);
+    select_unit(p, u, C);
+
+    // the last unit selected writes the prefix of token counts over units
+    __threadfence();
     __syncthreads();
-    if (s_last) {
-        __threadfence();
-        int carry = 0;
-        for (int base = 0; base < p.U; base += nt) {
-            const int x = (base + tid < p.U) ? __ldcg(p.n_tok + base + tid) : 0;
-            int tot;
-            const int ex = block_exclusive_scan(x, s_warp, &tot);
-            if (base + tid < p.U) p.unit_prefix[base + tid] = carry + ex;
-            carry += tot;
-        }
-        if (tid == 0) {
-            p.unit_prefix[p.U] = carry;
-            *p.counter = 0;
-        }
+    if (tid == 0) s_last = atomicAdd(p.tickets + p.U, 1) == p.U - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    int carry = 0;
+    for (int base = 0; base < p.U; base += blockDim.x) {
+        const int x = (base + tid < p.U) ? __ldcg(p.n_tok + base + tid) : 0;
+        int tot;
+        const int ex = block_exclusive_scan(x, s_warp2, &tot);
+        if (base + tid < p.U) p.unit_prefix[base + tid] = carry + ex;
+        carry += tot;
     }
+    if (tid == 0) p.unit_prefix[p.U] = carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -279,85 +452,100 @@ static int next_pow2(int x) {
     return n;
 }
 
-size_t select_ws_bytes(int U, int Cmax) { return align256((size_t)U * Cmax * 4) + 256; }
-
 namespace {
+struct SelWs {
+    size_t scores, hist, tickets, gkey, gw, total;
+};
+SelWs sel_ws_layout(int U, int Cmax) {
+    SelWs l;
+    const size_t np = (size_t)next_pow2(Cmax);
+    l.scores = 0;
+    l.hist = l.scores + align256((size_t)U * Cmax * 4);
+    l.tickets = l.hist + align256((size_t)U * SEL_HBINS * 4);
+    l.gkey = l.tickets + align256((size_t)(U + 1) * 4);
+    l.gw = l.gkey + align256((size_t)U * np * 8);
+    l.total = l.gw + align256((size_t)U * np * 4);
+    return l;
+}
+
 template <typename T, int D, int GQ>
-cudaError_t launch_score_t(const ScoreParams& p, int U, cudaStream_t st) {
-    dim3 grid((p.Cmax + SCORE_ROWS - 1) / SCORE_ROWS, U);
-    score_kernel<T, D, GQ><<<grid, 256, 0, st>>>(p);
-    return cudaGetLastError();
+cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
+    dim3 grid((p.Cmax + SCORE_ROWS - 1) / SCORE_ROWS, p.U);
+    score_kernel<T, D, GQ><<<grid, SEL_THREADS, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.U);
+    cfg.blockDim = dim3(SEL_THREADS);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, select_kernel, p);
 }
 }  // namespace
+
+size_t select_ws_bytes(int U, int Cmax) { return sel_ws_layout(U, Cmax).total; }
 
 cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const void* q, int budget,
                                 const SelView& s, void* ws, cudaStream_t st) {
     const int U = c.B * g.G;
+    const SelWs l = sel_ws_layout(U, g.Cmax);
     char* w = static_cast<char*>(ws);
-    float* scores = reinterpret_cast<float*>(w);
-    int32_t* counter = reinterpret_cast<int32_t*>(w + align256((size_t)U * g.Cmax * 4));
+    SelectParams p{};
+    p.q = q;
+    p.cent = g.cent;
+    p.scores = reinterpret_cast<float*>(w + l.scores);
+    p.hist = reinterpret_cast<int32_t*>(w + l.hist);
+    p.tickets = reinterpret_cast<int32_t*>(w + l.tickets);
+    p.gkey = reinterpret_cast<unsigned long long*>(w + l.gkey);
+    p.gw = reinterpret_cast<int32_t*>(w + l.gw);
+    p.cnt = g.cnt;
+    p.offs = g.offs;
+    p.tok = g.tok;
+    p.num_comm = g.num_comm;
+    p.tail_tok = g.tail_tok;
+    p.tail_comm = g.tail_comm;
+    p.tail_len = g.tail_len;
+    p.dev_err = g.dev_err;
+    p.sel_comm = s.sel_comm;
+    p.n_sel = s.n_sel;
+    p.sel_tok = s.sel_tok;
+    p.n_tok = s.n_tok;
+    p.unit_prefix = s.unit_prefix;
+    p.Hq = c.Hq;
+    p.G = g.G;
+    p.per_head = g.mode == CKV_GRAPH_PER_HEAD;
+    p.inv_sqrt_d = 1.0f / sqrtf((float)c.d);
+    p.U = U;
+    p.Cmax = g.Cmax;
+    p.npow_max = next_pow2(g.Cmax);
+    p.S = g.S;
+    p.T_cap = g.T_cap;
+    p.max_tail = g.max_tail;
+    p.tok_cap = s.tok_cap;
+    p.budget = budget;
+    // histograms and counters are contiguous: one memset clears both
+    cudaError_t e = cudaMemsetAsync(p.hist, 0, l.gkey - l.hist, st);
+    if (e != cudaSuccess) return e;
 
-    ScoreParams sp{};
-    sp.q = q;
-    sp.cent = g.cent;
-    sp.num_comm = g.num_comm;
-    sp.scores = scores;
-    sp.counter = counter;
-    sp.Hq = c.Hq;
-    sp.Hkv = c.Hkv;
-    sp.G = g.G;
-    sp.per_head = g.mode == CKV_GRAPH_PER_HEAD;
-    sp.Cmax = g.Cmax;
-    sp.inv_sqrt_d = 1.0f / sqrtf((float)c.d);
-
-    cudaError_t e = cudaErrorInvalidValue;
 #define CKV_SC_CASE(TT, DD, GG) \
-    else if (c.d == DD && g.gq == GG) e = launch_score_t<TT, DD, GG>(sp, U, st);
+    if (c.d == DD && g.gq == GG) return launch_t<TT, DD, GG>(p, st);
     if (c.dtype == CKV_DTYPE_BF16) {
-        if (false) {}
         CKV_SC_CASE(__nv_bfloat16, 128, 1) CKV_SC_CASE(__nv_bfloat16, 128, 2)
         CKV_SC_CASE(__nv_bfloat16, 128, 4) CKV_SC_CASE(__nv_bfloat16, 128, 8)
         CKV_SC_CASE(__nv_bfloat16, 64, 1) CKV_SC_CASE(__nv_bfloat16, 64, 2)
         CKV_SC_CASE(__nv_bfloat16, 64, 4) CKV_SC_CASE(__nv_bfloat16, 64, 8)
     } else {
-        if (false) {}
         CKV_SC_CASE(float, 128, 1) CKV_SC_CASE(float, 128, 2)
         CKV_SC_CASE(float, 128, 4) CKV_SC_CASE(float, 128, 8)
         CKV_SC_CASE(float, 64, 1) CKV_SC_CASE(float, 64, 2)
         CKV_SC_CASE(float, 64, 4) CKV_SC_CASE(float, 64, 8)
     }
 #undef CKV_SC_CASE
-    if (e != cudaSuccess) return e;
-
-    SelectParams pp{};
-    pp.scores = scores;
-    pp.cnt = g.cnt;
-    pp.offs = g.offs;
-    pp.tok = g.tok;
-    pp.num_comm = g.num_comm;
-    pp.tail_tok = g.tail_tok;
-    pp.tail_comm = g.tail_comm;
-    pp.tail_len = g.tail_len;
-    pp.dev_err = g.dev_err;
-    pp.sel_comm = s.sel_comm;
-    pp.n_sel = s.n_sel;
-    pp.sel_tok = s.sel_tok;
-    pp.n_tok = s.n_tok;
-    pp.unit_prefix = s.unit_prefix;
-    pp.counter = counter;
-    pp.U = U;
-    pp.Cmax = g.Cmax;
-    pp.npow_max = next_pow2(g.Cmax);
-    pp.S = g.S;
-    pp.T_cap = g.T_cap;
-    pp.max_tail = g.max_tail;
-    pp.tok_cap = s.tok_cap;
-    pp.budget = budget;
-    const size_t smem = (size_t)pp.npow_max * 12 + ((g.Cmax + 31) / 32) * 4;
-    e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    select_kernel<<<U, SEL_THREADS, smem, st>>>(pp);
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace ckv

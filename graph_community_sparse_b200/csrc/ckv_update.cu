@@ -6,10 +6,10 @@
 // rit.work summary, section "A graph of tokens replaces re-clustering",
 // paragraph 6; the abstract describes the rule as constant-time).
 //
-// One warp per graph unit: the candidate communities are those of the 8
-// neighbour positions found by the attention kernel; each distinct candidate
-// costs one d-long dot product with the new key; the winner's centre moves
-// by (k - c)/(n + 1) and its count grows by one.  O(8 d) work per graph.
+// The candidate communities are those of the 8 neighbour positions found by
+// the attention kernel; each distinct candidate costs one d-long dot product
+// with the new key; the winner's centre moves by (k - c)/(n + 1) and its
+// count grows by one.  O(8 d) work per graph.
 #include <math.h>
 
 #include "ckv_internal.cuh"
@@ -32,81 +32,96 @@ struct AssignParams {
     int32_t* assigned;
 };
 
+// One block per graph unit; warp i scores candidate i (the community of
+// neighbour i, skipped when empty or already seen), so all candidate centres
+// are fetched at once.  Thread 0 picks the winner; the block updates its
+// centre row.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) assign_kernel(AssignParams p) {
+__global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParams p) {
     constexpr int E = D / 32;
-    const int lane = threadIdx.x & 31;
-    const int u = blockIdx.x * 4 + (threadIdx.x >> 5);
-    if (u >= p.U) return;
+    __shared__ int s_cand[CKV_NEIGHBOURS];
+    __shared__ float s_score[CKV_NEIGHBOURS];
+    __shared__ int s_best, s_n, s_tl;
+    const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = u / p.G, g = u - b * p.G;
     const int kvh = p.per_head ? g / (p.Hq / p.Hkv) : g;
+    if (tid < CKV_NEIGHBOURS) {
+        int c = -1;
+        const int np = p.nbr8[(size_t)u * CKV_NEIGHBOURS + tid];
+        if (np >= 0 && np < p.T_cap) {
+            const int cc = p.comm_of[(size_t)u * p.T_cap + np];
+            if (cc >= 0 && cc < p.Cmax) c = cc;
+        }
+        s_cand[tid] = c;
+    }
+    if (tid == 0) {
+        s_tl = p.tail_len[u];
+    }
     const T* krow = static_cast<const T*>(p.k) + b * p.sb + kvh * p.sh + (int64_t)p.pos * p.st + lane * E;
     float kx[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) kx[e] = to_f32(krow[e]);
+    __syncthreads();
 
-    int cand = -1;
-    if (lane < CKV_NEIGHBOURS) {
-        const int np = p.nbr8[(size_t)u * CKV_NEIGHBOURS + lane];
-        if (np >= 0 && np < p.T_cap) {
-            const int c = p.comm_of[(size_t)u * p.T_cap + np];
-            if (c >= 0 && c < p.Cmax) cand = c;
-        }
-    }
-    int best = -1;
-    float best_s = -INFINITY;
-    for (int i = 0; i < CKV_NEIGHBOURS; ++i) {
-        const int ci = __shfl_sync(FULL, cand, i);
-        if (ci < 0) continue;
-        if (__ballot_sync(FULL, lane < i && cand == ci)) continue;  // seen already
-        const float* cr = p.cent + ((size_t)u * p.Cmax + ci) * D + lane * E;
-        float a = 0.f;
+    // warp i: score of candidate i (-inf when absent or a repeat)
+    {
+        const int ci = s_cand[warp];
+        bool use = ci >= 0;
+        for (int j = 0; j < warp; ++j) use = use && s_cand[j] != ci;
+        float s = -INFINITY;
+        if (use) {
+            const float* cr = p.cent + ((size_t)u * p.Cmax + ci) * D + lane * E;
+            float a = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) a = fmaf(kx[e], cr[e], a);
+            for (int e = 0; e < E; ++e) a = fmaf(kx[e], cr[e], a);
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
-        const float s = a * p.inv_sqrt_d;
-        if (best < 0 || s > best_s || (s == best_s && ci < best)) {
-            best = ci;
-            best_s = s;
+            for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+            s = a * p.inv_sqrt_d;
         }
+        if (lane == 0) s_score[warp] = use ? s : -INFINITY;
     }
-    int32_t* cpos = p.comm_of + (size_t)u * p.T_cap + p.pos;
-    if (best < 0) {
-        if (lane == 0) {
-            *cpos = -1;
-            if (p.assigned) p.assigned[u] = -1;
+    __syncthreads();
+    if (tid == 0) {
+        int best = -1;
+        float bs = -INFINITY;
+        for (int i = 0; i < CKV_NEIGHBOURS; ++i) {
+            const int ci = s_cand[i];
+            if (ci < 0 || s_score[i] == -INFINITY) continue;
+            if (best < 0 || s_score[i] > bs || (s_score[i] == bs && ci < best)) {
+                best = ci;
+                bs = s_score[i];
+            }
         }
-        return;
-    }
-    int tl = 0;
-    if (lane == 0) tl = p.tail_len[u];
-    tl = __shfl_sync(FULL, tl, 0);
-    if (tl >= p.max_tail) {
-        if (lane == 0) {
-            *cpos = -1;
+        int32_t* cpos = p.comm_of + (size_t)u * p.T_cap + p.pos;
+        if (best >= 0 && s_tl >= p.max_tail) {
             atomicOr(p.dev_err, CKV_DEVERR_TAIL_FULL);
-            if (p.assigned) p.assigned[u] = -1;
+            best = -1;
         }
-        return;
+        s_best = best;
+        if (best < 0) {
+            *cpos = -1;
+            if (p.assigned) p.assigned[u] = -1;
+        } else {
+            const int n = p.cnt[(size_t)u * p.Cmax + best];
+            s_n = n;
+            p.cnt[(size_t)u * p.Cmax + best] = n + 1;
+            *cpos = best;
+            p.tail_tok[(size_t)u * p.max_tail + s_tl] = p.pos;
+            p.tail_comm[(size_t)u * p.max_tail + s_tl] = best;
+            p.tail_len[u] = s_tl + 1;
+            if (p.assigned) p.assigned[u] = best;
+        }
     }
-    int n = 0;
-    if (lane == 0) n = p.cnt[(size_t)u * p.Cmax + best];
-    n = __shfl_sync(FULL, n, 0);
+    __syncthreads();
+    const int best = s_best;
+    if (best < 0 || warp != 0) return;
+    // running mean: c <- c + (k - c) / (n + 1)
     float* cr = p.cent + ((size_t)u * p.Cmax + best) * D + lane * E;
-    const float denom = (float)(n + 1);
+    const float denom = (float)(s_n + 1);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const float c0 = cr[e];
         cr[e] = c0 + (kx[e] - c0) / denom;
-    }
-    if (lane == 0) {
-        p.cnt[(size_t)u * p.Cmax + best] = n + 1;
-        *cpos = best;
-        p.tail_tok[(size_t)u * p.max_tail + tl] = p.pos;
-        p.tail_comm[(size_t)u * p.max_tail + tl] = best;
-        p.tail_len[u] = tl + 1;
-        if (p.assigned) p.assigned[u] = best;
     }
 }
 
@@ -136,13 +151,13 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
     p.tail_len = g.tail_len;
     p.dev_err = g.dev_err;
     p.assigned = assigned;
-    const int blocks = (p.U + 3) / 4;
+    const int threads = CKV_NEIGHBOURS * 32;
     if (c.dtype == CKV_DTYPE_BF16) {
-        if (c.d == 128) assign_kernel<__nv_bfloat16, 128><<<blocks, 128, 0, st>>>(p);
-        else assign_kernel<__nv_bfloat16, 64><<<blocks, 128, 0, st>>>(p);
+        if (c.d == 128) assign_kernel<__nv_bfloat16, 128><<<p.U, threads, 0, st>>>(p);
+        else assign_kernel<__nv_bfloat16, 64><<<p.U, threads, 0, st>>>(p);
     } else {
-        if (c.d == 128) assign_kernel<float, 128><<<blocks, 128, 0, st>>>(p);
-        else assign_kernel<float, 64><<<blocks, 128, 0, st>>>(p);
+        if (c.d == 128) assign_kernel<float, 128><<<p.U, threads, 0, st>>>(p);
+        else assign_kernel<float, 64><<<p.U, threads, 0, st>>>(p);
     }
     return cudaGetLastError();
 }
