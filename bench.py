@@ -6,8 +6,8 @@
 One step = ckv_score_select + ckv_sparse_decode (+ the cache append and
 ckv_assign_update when the workload updates) for the whole batch of one
 layer, with inputs resident in HBM.  Every timed step is bracketed by CUDA
-events on the launching stream; L2 is flushed (a 1 GiB write) before each
-step, outside the events.  Rank 0 prints one JSON line.  With N GPUs each rank
+events on the launching stream; L2 is flushed (a 1 GiB write, then a 512 MiB
+read so no dirty lines are left) before each step, outside the events.  Rank 0 prints one JSON line.  With N GPUs each rank
 runs its own batch (weak scaling, no collective on the data path); the value
 is N*K steps over the slowest rank's time.
 """
@@ -224,8 +224,14 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     # before the GPU reaches it, so the events time device work, not launch gaps
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.float32, device=device)
 
+    # then reading another 512 MiB leaves L2 clean: the dirty lines of the
+    # write are written back here, not charged to the step's first kernel
+    clean_buf = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device=device)
+    sink = torch.zeros((), dtype=torch.float32, device=device)
+
     def flush():
         flush_buf.fill_(1.0)
+        torch.sum(clean_buf, dim=0, out=sink)
 
     esz = 2 if wl.dtype == "bf16" else 4
     row_bytes = 2 * wl.d * esz
@@ -397,7 +403,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
                    "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
                    "communities_per_graph": float(ncomm / U), "budget": budget, "sinks": wl.S,
                    "update": wl.update, "layout": wl.layout,
-                   "l2": "flushed by a 1 GiB write before every timed step, outside the CUDA events",
+                   "l2": "flushed by a 1 GiB write then a 512 MiB read before every timed step, outside the CUDA events",
                    "parallelism": f"dp{n_ranks} (independent batches, no collective)"},
         "tokens_per_s": value * wl.B,
         "roofline": roofline,

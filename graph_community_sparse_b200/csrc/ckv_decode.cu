@@ -68,7 +68,8 @@ struct DecodeParams {
     int S;
     const int32_t* sel_tok;
     int tok_cap;
-    const int32_t* unit_prefix;
+    int32_t* unit_prefix;   // written by block 0 of the attention kernel
+    const int32_t* n_tok;
     int T;                  // dense only: tokens per unit
     float scale_log2;
     DecodeWs ws;
@@ -339,8 +340,28 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(
 
     int total;
     if constexpr (!DENSE) {
-        for (int i = threadIdx.x; i <= p.U; i += blockDim.x) s_pre[i] = p.unit_prefix[i];
+        // exclusive prefix of the units' token counts, computed by every block
+        // (each thread scans a contiguous chunk); block 0 also publishes it
+        __shared__ int s_warp[33];
+        const int seg = (p.U + blockDim.x - 1) / blockDim.x;
+        const int b0 = min(p.U, (int)threadIdx.x * seg), b1 = min(p.U, b0 + seg);
+        int own = 0;
+        for (int i = b0; i < b1; ++i) {
+            const int x = p.n_tok[i];
+            s_pre[i] = x;
+            own += x;
+        }
+        int all;
+        int run = block_exclusive_scan(own, s_warp, &all);
+        for (int i = b0; i < b1; ++i) {
+            const int x = s_pre[i];
+            s_pre[i] = run;
+            run += x;
+        }
+        if (threadIdx.x == 0) s_pre[p.U] = all;
         __syncthreads();
+        if (blockIdx.x == 0)
+            for (int i = threadIdx.x; i <= p.U; i += blockDim.x) p.unit_prefix[i] = s_pre[i];
         total = s_pre[p.U];
     } else {
         total = p.U * p.T;
@@ -634,6 +655,7 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
     p.sel_tok = s.sel_tok;
     p.tok_cap = s.tok_cap;
     p.unit_prefix = s.unit_prefix;
+    p.n_tok = s.n_tok;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
     p.ws = carve_decode_ws(ws, p.U, g.gq, c.d);
     p.want_nbr = nbr8 != nullptr;

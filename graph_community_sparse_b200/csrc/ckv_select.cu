@@ -22,10 +22,8 @@
 //    a scan of their sizes gives the cut (at least the top community).  Then
 //    the unit's token list: sinks, build-time members of each selected
 //    community (from the community-contiguous CSR), then the selected tail
-//    members.  The last unit done (arrival counter; no block ever waits)
-//    writes the exclusive prefix of the token counts over units for the
-//    attention kernel's work split.
-// Histograms and the counter are zeroed by one memset issued in the same call.
+//    members.
+// The histograms are zeroed by a memset issued in the same call.
 #include <math.h>
 
 #include "ckv_internal.cuh"
@@ -44,7 +42,6 @@ struct SelectParams {
     const float* cent;
     float* scores;              // [U, Cmax]
     int32_t* hist;              // [U, SEL_HBINS]
-    int32_t* tickets;           // [U + 1]
     unsigned long long* gkey;   // [U, npow_max] scratch for large candidate sets
     int32_t* gw;                // [U, npow_max]
     const int32_t* cnt;
@@ -416,30 +413,11 @@ __global__ void __launch_bounds__(SEL_THREADS) score_kernel(SelectParams p) {
 }
 
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
-    __shared__ int s_last;
-    __shared__ int s_warp2[33];
     // wait until every score and histogram update of the scoring kernel is visible
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int u = blockIdx.x, tid = threadIdx.x;
+    const int u = blockIdx.x;
     const int C = min(p.num_comm[u], p.Cmax);
     select_unit(p, u, C);
-
-    // the last unit selected writes the prefix of token counts over units
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.tickets + p.U, 1) == p.U - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    int carry = 0;
-    for (int base = 0; base < p.U; base += blockDim.x) {
-        const int x = (base + tid < p.U) ? __ldcg(p.n_tok + base + tid) : 0;
-        int tot;
-        const int ex = block_exclusive_scan(x, s_warp2, &tot);
-        if (base + tid < p.U) p.unit_prefix[base + tid] = carry + ex;
-        carry += tot;
-    }
-    if (tid == 0) p.unit_prefix[p.U] = carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -454,15 +432,14 @@ static int next_pow2(int x) {
 
 namespace {
 struct SelWs {
-    size_t scores, hist, tickets, gkey, gw, total;
+    size_t scores, hist, gkey, gw, total;
 };
 SelWs sel_ws_layout(int U, int Cmax) {
     SelWs l;
     const size_t np = (size_t)next_pow2(Cmax);
     l.scores = 0;
     l.hist = l.scores + align256((size_t)U * Cmax * 4);
-    l.tickets = l.hist + align256((size_t)U * SEL_HBINS * 4);
-    l.gkey = l.tickets + align256((size_t)(U + 1) * 4);
+    l.gkey = l.hist + align256((size_t)U * SEL_HBINS * 4);
     l.gw = l.gkey + align256((size_t)U * np * 8);
     l.total = l.gw + align256((size_t)U * np * 4);
     return l;
@@ -499,7 +476,6 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     p.cent = g.cent;
     p.scores = reinterpret_cast<float*>(w + l.scores);
     p.hist = reinterpret_cast<int32_t*>(w + l.hist);
-    p.tickets = reinterpret_cast<int32_t*>(w + l.tickets);
     p.gkey = reinterpret_cast<unsigned long long*>(w + l.gkey);
     p.gw = reinterpret_cast<int32_t*>(w + l.gw);
     p.cnt = g.cnt;
@@ -527,7 +503,7 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     p.max_tail = g.max_tail;
     p.tok_cap = s.tok_cap;
     p.budget = budget;
-    // histograms and counters are contiguous: one memset clears both
+    // the per-unit histograms start at zero
     cudaError_t e = cudaMemsetAsync(p.hist, 0, l.gkey - l.hist, st);
     if (e != cudaSuccess) return e;
 

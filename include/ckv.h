@@ -141,7 +141,8 @@ typedef struct {
  *                                   community in rank order, then its tail
  *                                   members
  *   n_tok       int32 [U]           length of each sel_tok row
- *   unit_prefix int32 [U+1]         exclusive prefix sum of n_tok
+ *   unit_prefix int32 [U+1]         exclusive prefix sum of n_tok, written by
+ *                                   ckv_sparse_decode (its work split)
  * tok_cap >= T_cap can never overflow; tok_cap >= S + max(budget, largest
  * community) + max_tail suffices too.
  */
