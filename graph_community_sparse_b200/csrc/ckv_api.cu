@@ -179,18 +179,17 @@ const char* ckv_last_error(void) { return g_last_error.c_str(); }
 
 ckv_status ckv_workspace_size(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
                               const ckv_selection_desc* sel, size_t* bytes) {
-    (void)sel;
     if (!bytes) return fail(CKV_ERR_INVALID_ARG, "bytes is NULL");
     CKV_TRY(check_cache(cache, false));
     const int gq_dense = cache->Hq / cache->Hkv;
-    size_t need = ckv::decode_ws_bytes(cache->B * cache->Hkv, gq_dense, cache->d);
+    size_t need = ckv::decode_ws_bytes(cache->B * cache->Hkv, gq_dense, cache->d, 0);
     if (graph) {
         CKV_TRY(check_graph(cache, graph));
         const int U = cache->B * graphs_per_seq(cache, graph);
         const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : gq_dense;
         const size_t a = ckv::build_ws_bytes(U, graph->Cmax, graph->T_cap);
         const size_t b = ckv::select_ws_bytes(U, graph->Cmax);
-        const size_t c = ckv::decode_ws_bytes(U, gq, cache->d);
+        const size_t c = ckv::decode_ws_bytes(U, gq, cache->d, sel ? sel->tok_cap : graph->T_cap);
         need = need > a ? need : a;
         need = need > b ? need : b;
         need = need > c ? need : c;
@@ -241,7 +240,7 @@ ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q, const c
     if (!q || !out) return fail(CKV_ERR_INVALID_ARG, "q or out is NULL");
     if (!aligned16(q) || !aligned16(out)) return fail(CKV_ERR_MISALIGNED, "q and out must be 16-byte aligned");
     const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : cache->Hq / cache->Hkv;
-    CKV_TRY(check_ws(ws, ws_bytes, ckv::decode_ws_bytes((int)U, gq, cache->d)));
+    CKV_TRY(check_ws(ws, ws_bytes, ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap)));
     return cuda_status(ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q,
                                                  out, nbr8, ws, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_sparse_decode");
@@ -260,7 +259,7 @@ ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const void* q,
     if (!q || !out) return fail(CKV_ERR_INVALID_ARG, "q or out is NULL");
     if (!aligned16(q) || !aligned16(out)) return fail(CKV_ERR_MISALIGNED, "q and out must be 16-byte aligned");
     const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : cache->Hq / cache->Hkv;
-    const size_t need = ckv::decode_ws_bytes((int)U, gq, cache->d);
+    const size_t need = ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap);
     if (need > CKV_NOALLOC_SCRATCH_BYTES)
         return fail(CKV_ERR_UNSUPPORTED,
                     "ckv_sparse_decode_noalloc: these shapes need %zu bytes of scratch, above the library's "
@@ -294,7 +293,7 @@ ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t 
     if (T < 1 || T > cache->T_cap) return fail(CKV_ERR_CAPACITY, "T = %d outside [1, T_cap]", T);
     const int64_t U = (int64_t)cache->B * cache->Hkv;
     if (U * T > (int64_t)1 << 30) return fail(CKV_ERR_UNSUPPORTED, "B*Hkv*T above 2^30");
-    CKV_TRY(check_ws(ws, ws_bytes, ckv::decode_ws_bytes((int)U, cache->Hq / cache->Hkv, cache->d)));
+    CKV_TRY(check_ws(ws, ws_bytes, ckv::decode_ws_bytes((int)U, cache->Hq / cache->Hkv, cache->d, 0)));
     return cuda_status(ckv::launch_dense_decode(cache_view(cache), q, T, out, ws,
                                                 reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_dense_decode");

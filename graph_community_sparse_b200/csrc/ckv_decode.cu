@@ -30,6 +30,7 @@
 // lazily raised running max (raised only when a logit exceeds it by more
 // than 2^8), which is exact after the final division.
 #include <math.h>
+#include <type_traits>
 
 #include "ckv_internal.cuh"
 
@@ -38,7 +39,6 @@ namespace ckv {
 constexpr int DEC_WARPS = 4;
 constexpr int TOK_PER_IT = 8;
 constexpr float RESCALE_THRESH = 8.0f;
-constexpr int MERGE_CHUNK = 128;  // slots whose weights are staged in shared memory at once
 
 template <int GQ> struct Stages { static constexpr int v = GQ == 1 ? 2 : 3; };
 template <int GQ> struct MinBlocks { static constexpr int v = GQ == 1 ? 6 : (GQ == 2 ? 5 : (GQ == 4 ? 4 : 2)); };
@@ -92,26 +92,19 @@ __device__ __forceinline__ void unit_heads(const DecodeParams& p, int u, int gq,
     }
 }
 
-// Insert (cv, cpos) into the warp's sorted top-8 list held by lanes 0..7
-// (value descending, position ascending).
-__device__ __forceinline__ void top8_insert(float cv, int cpos, float& tv, int& tp, float& thr, int lane) {
-    const bool above = lane < 8 && (tv > cv || (tv == cv && tp < cpos));
-    const int k = __popc(__ballot_sync(FULL, above));
-    if (k < 8) {
-        const float uv = __shfl_up_sync(FULL, tv, 1);
-        const int up = __shfl_up_sync(FULL, tp, 1);
-        if (lane < 8 && lane > k) {
-            tv = uv;
-            tp = up;
-        }
-        if (lane == k) {
-            tv = cv;
-            tp = cpos;
-        }
-        thr = __shfl_sync(FULL, tv, 7);
-    }
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32, relative error
+// about 2^-22).  Arguments here are <= 8; results below 2^-126 flush to zero,
+// which only drops weights below 1e-38 of the running maximum.
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
+// One warp, one unit, list positions [lo, hi) of the unit's selection (or
+// cache positions, dense).  Full iterations (all 8 tokens valid, past the
+// sinks) take a path without per-token masks; only the last, partial
+// iteration and the one holding the sinks test each token.
 template <typename T, int D, int GQ, bool DENSE>
 __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, int lo, int hi, int slot,
                                                 unsigned char* wsm, int lane) {
@@ -122,6 +115,8 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
     const int half = lane >> 4, l16 = lane & 15;
     const int hl = head_of_lane<GQ>(lane);
     const bool owner = (lane & ((16 >> LG) - 1)) == 0;
+    const int64_t st = p.st;
+    const bool want_nbr = !DENSE && p.want_nbr;
 
     int b, kvh, h0;
     unit_heads(p, u, GQ, DENSE, b, kvh, h0);
@@ -139,6 +134,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 
     const int n = hi - lo;
     const int nit = (n + TOK_PER_IT - 1) / TOK_PER_IT;
+    const int nfull = n / TOK_PER_IT;
     float* pbuf = reinterpret_cast<float*>(wsm + NS * 2 * TILE);
 
     int win_cur = 0, win_nxt = 0;
@@ -147,8 +143,9 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
         win_nxt = (32 + lane < n) ? __ldg(toks + lo + 32 + lane) : 0;
     }
 
-    int stage_in = 0;  // ring slot the next issue() fills
-    auto issue = [&](int it) {
+    int stage_in = 0;  // ring slot the next issue fills
+    auto issue = [&](int it, auto full_tag) {
+        constexpr bool ALL_VALID = decltype(full_tag)::value;
         unsigned char* kt = wsm + stage_in * 2 * TILE;
         stage_in = (stage_in + 1 == NS) ? 0 : stage_in + 1;
         unsigned char* vt = kt + TILE;
@@ -162,26 +159,29 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int i = it * TOK_PER_IT + 2 * j + half;
-            const bool valid = i < n;
+            const bool valid = ALL_VALID || i < n;
             int pos;
             if constexpr (DENSE) {
-                pos = valid ? lo + i : 0;
+                pos = lo + i;
             } else {
-                const int pp = __shfl_sync(FULL, win_cur, ((it & 3) << 3) + 2 * j + half);
-                pos = valid ? pp : 0;
+                pos = __shfl_sync(ckv::FULL, win_cur, ((it & 3) << 3) + 2 * j + half);
             }
+            if (!ALL_VALID) pos = valid ? pos : 0;
+            const int64_t off = (int64_t)pos * st;
             const int r = 2 * j + half;
-            cp_async_part<PART>(kt + r * ROW + l16 * PART, Kb + (int64_t)pos * p.st, valid);
-            cp_async_part<PART>(vt + r * ROW + l16 * PART, Vb + (int64_t)pos * p.st, valid);
+            cp_async_part<PART>(kt + r * ROW + l16 * PART, Kb + off, valid);
+            cp_async_part<PART>(vt + r * ROW + l16 * PART, Vb + off, valid);
         }
         cp_async_commit();
     };
+    auto issue_any = [&](int it) {
+        if (it < nfull) issue(it, std::true_type{});
+        else if (it < nit) issue(it, std::false_type{});
+        else cp_async_commit();
+    };
 
 #pragma unroll
-    for (int s = 0; s < NS - 1; ++s) {
-        if (s < nit) issue(s);
-        else cp_async_commit();
-    }
+    for (int s = 0; s < NS - 1; ++s) issue_any(s);
 
     float m_run = -INFINITY, l_run = 0.f;
     float acc[GQ][E];
@@ -189,16 +189,11 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
     for (int h = 0; h < GQ; ++h)
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
-    float tv = -INFINITY, thr = -INFINITY;
-    int tp = 0x7fffffff;
+    float* lamu = DENSE ? nullptr : p.ws.lam + (size_t)u * p.ws.lam_cap;
+    int stage_out = 0;  // ring slot computed next
 
-    int stage_out = 0;  // ring slot computed in this iteration
-    for (int it = 0; it < nit; ++it) {
-        __syncwarp();
-        if (it + NS - 1 < nit) issue(it + NS - 1);
-        else cp_async_commit();
-        cp_async_wait<NS - 1>();
-
+    auto compute = [&](int it, auto full_tag) {
+        constexpr bool ALL_VALID = decltype(full_tag)::value;
         const unsigned char* kt = wsm + stage_out * 2 * TILE;
         const unsigned char* vt = kt + TILE;
         stage_out = (stage_out + 1 == NS) ? 0 : stage_out + 1;
@@ -217,20 +212,20 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
                 part[h] = a;
             }
             s[j] = halfwarp_reduce_heads<GQ>(part, lane);
-            if (it * TOK_PER_IT + 2 * j + half >= n) s[j] = -INFINITY;
+            if (!ALL_VALID && it * TOK_PER_IT + 2 * j + half >= n) s[j] = -INFINITY;
         }
 
         float mx = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[2], s[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+        mx = fmaxf(mx, __shfl_xor_sync(ckv::FULL, mx, 16));
         const bool need = mx > m_run + RESCALE_THRESH;
-        if (__any_sync(FULL, need)) {
+        if (__any_sync(ckv::FULL, need)) {
             const float m_new = need ? mx : m_run;
-            const float f = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
+            const float f = (m_run == -INFINITY) ? 0.f : exp2_approx(m_run - m_new);
             l_run *= f;
             m_run = m_new;
 #pragma unroll
             for (int h = 0; h < GQ; ++h) {
-                const float fh = __shfl_sync(FULL, f, (lane & 16) | (h << (4 - LG)));
+                const float fh = __shfl_sync(ckv::FULL, f, (lane & 16) | (h << (4 - LG)));
 #pragma unroll
                 for (int e = 0; e < E; ++e) acc[h][e] *= fh;
             }
@@ -238,7 +233,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 
         float pj[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) pj[j] = exp2f(s[j] - m_run);
+        for (int j = 0; j < 4; ++j) pj[j] = exp2_approx(s[j] - m_run);
         l_run += (pj[0] + pj[1]) + (pj[2] + pj[3]);
 
         if constexpr (GQ > 1) {
@@ -270,35 +265,24 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
                 for (int e = 0; e < E; ++e) acc[h][e] = fmaf(ph[h], vf[e], acc[h][e]);
         }
 
-        if constexpr (!DENSE) {
-            if (p.want_nbr) {
-                bool f[4];
-                bool anyf = false;
+        if (want_nbr) {
+            // graph logit of each token (max over the group's heads) for the
+            // neighbour search in the merge kernel
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int i = it * TOK_PER_IT + 2 * j + half;
-                    f[j] = (i < n) && (lo + i >= p.S) && (s[j] >= thr);
-                    anyf |= f[j];
-                }
-                if (__any_sync(FULL, anyf)) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const unsigned bj = __ballot_sync(FULL, f[j]);
-                        if (bj) {
-                            const float lam = halfwarp_max_over_heads<GQ>(s[j]);
-#pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                if (bj & (0xffffu << (16 * hh))) {
-                                    const float cv = __shfl_sync(FULL, lam, 16 * hh);
-                                    const int cpos = __ldg(toks + lo + it * TOK_PER_IT + 2 * j + hh);
-                                    top8_insert(cv, cpos, tv, tp, thr, lane);
-                                }
-                            }
-                        }
-                    }
-                }
+            for (int j = 0; j < 4; ++j) {
+                const float lam = halfwarp_max_over_heads<GQ>(s[j]);
+                const int i = it * TOK_PER_IT + 2 * j + half;
+                if (l16 == 0 && (ALL_VALID || i < n)) lamu[lo + i] = lam;
             }
         }
+    };
+
+    for (int it = 0; it < nit; ++it) {
+        __syncwarp();
+        issue_any(it + NS - 1);
+        cp_async_wait<NS - 1>();
+        if (it < nfull) compute(it, std::true_type{});
+        else compute(it, std::false_type{});
     }
     cp_async_wait<0>();
 
@@ -320,12 +304,6 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
         if (owner) {
             ws.m[(size_t)slot * GQ + hl] = m_run;
             ws.l[(size_t)slot * GQ + hl] = l_run;
-        }
-    }
-    if constexpr (!DENSE) {
-        if (p.want_nbr && lane < 8) {
-            ws.tv[(size_t)slot * 8 + lane] = tv;
-            ws.tp[(size_t)slot * 8 + lane] = (tv == -INFINITY) ? -1 : tp;
         }
     }
 }
@@ -394,15 +372,57 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(
     }
 }
 
+// Warps of the merge block that search the neighbours (sparse decode only).
+constexpr int NBR_WARPS = 4;
+// Spare partial slots after the last one: a merge chunk (<= 32 slots) may
+// read past a unit's last slot without leaving the arrays.
+constexpr int MERGE_PAD = 32;
+constexpr int NBR_THREADS = NBR_WARPS * 32;
+constexpr int NBR_KEEP = 16;  // list entries per thread held in registers
+constexpr int NBR_CAP = 256;  // candidate slots in shared memory
+
+// Neighbour ranking key: graph logit descending, then position ascending, as
+// one unsigned 64-bit number (larger is better; 0 = no entry).  The logit is
+// mapped to an order-preserving unsigned integer.
+__device__ __forceinline__ unsigned long long nbr_key(float lam, int pos) {
+    unsigned b = __float_as_uint(lam + 0.0f);  // -0 ranks as +0
+    b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)b << 32) | (unsigned)(0x7fffffff - pos);
+}
+__device__ __forceinline__ int nbr_pos(unsigned long long k) {
+    return 0x7fffffff - (int)(unsigned)(k & 0xffffffffu);
+}
+
+// Bitonic sort of one key per lane, descending across the warp.
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(FULL, x, j);
+            const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
+            x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+        }
+    }
+    return x;
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(FULL, x, o);
+        x = x > y ? x : y;
+    }
+    return x;
+}
+
 // One block per unit: threads 0..D-1 own one output dimension each (all the
-// unit's heads); the extra warp merges the top-8 neighbour lists.  Slots are
-// combined in slot order, MERGE_CHUNK at a time, with every load of a chunk
-// issued before any is used.
+// unit's heads); the NBR_WARPS extra warps search the top-8 neighbours.  Slots are
+// combined in slot order, a chunk of slots at a time, by a per-thread online
+// merge: no shared memory and no barriers, so the merge costs about two
+// dependent rounds of loads.
 template <int D, int GQ, bool DENSE>
-__global__ void __launch_bounds__(D + 32) decode_merge(DecodeParams p) {
-    __shared__ float s_f[MERGE_CHUNK][GQ];
-    __shared__ float s_red[(D + 32) / 32][GQ];
-    __shared__ float s_M[GQ];
+__global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_merge(DecodeParams p) {
     // wait until the attention kernel's partials are complete and visible
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int u = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -429,148 +449,169 @@ __global__ void __launch_bounds__(D + 32) decode_merge(DecodeParams p) {
     const size_t s0 = (size_t)wf + u;
     const DecodeWs& ws = p.ws;
 
-    if (!DENSE && p.want_nbr && warp == D / 32) {
-        // candidates: 8 per slot; each lane keeps its best 8 in registers
-        // (value desc, position asc), then 8 warp-wide rounds pick the winners
-        float cv[8];
-        int cp[8];
+    if (!DENSE && p.want_nbr && warp >= D / 32) {
+        // neighbour search over the graph logits the attention kernel stored,
+        // for the unit's non-sink list entries [S, n).  Threshold filter:
+        // theta = the 8th largest of the NBR_THREADS per-thread maxima is a
+        // distinct entry's key with 7 larger ones, so every top-8 entry has
+        // key >= theta; those few candidates are collected in shared memory
+        // and sorted by one warp.
+        __shared__ unsigned long long s_top[NBR_THREADS / 4];
+        __shared__ unsigned long long s_cand[NBR_CAP];
+        __shared__ int s_cnt;
+        const int xt = t - D, xw = xt >> 5;
+        const int n = uend - ubeg;
+        const float* lamu = ws.lam + (size_t)u * ws.lam_cap;
+        const int32_t* toks = p.sel_tok + (size_t)u * p.tok_cap;
+        auto key_at = [&](int i) { return nbr_key(lamu[i], __ldg(toks + i)); };
+        // all loads first (clamped in-range indices, no branches), so the
+        // 2 x NBR_KEEP loads are in flight together
+        float lv[NBR_KEEP];
+        int pv[NBR_KEEP];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            cv[r] = -INFINITY;
-            cp[r] = 0x7fffffff;
+        for (int k = 0; k < NBR_KEEP; ++k) {
+            const int i = min(p.S + xt + k * NBR_THREADS, n - 1);
+            lv[k] = lamu[i];
+            pv[k] = __ldg(toks + i);
         }
-        for (int i = lane; i < nslots * 8; i += 32) {
-            const size_t sl = (s0 + (i >> 3)) * 8 + (i & 7);
-            float v = ws.tv[sl];
-            int q = ws.tp[sl];
-            if (q < 0) continue;
+        unsigned long long kk[NBR_KEEP];
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const bool better = (v > cv[r]) || (v == cv[r] && q < cp[r]);
-                const float v2 = better ? cv[r] : v;
-                const int q2 = better ? cp[r] : q;
-                if (better) {
-                    cv[r] = v;
-                    cp[r] = q;
+        for (int k = 0; k < NBR_KEEP; ++k)
+            kk[k] = p.S + xt + k * NBR_THREADS < n ? nbr_key(lv[k], pv[k]) : 0ull;
+        unsigned long long mx = 0;
+#pragma unroll
+        for (int k = 0; k < NBR_KEEP; ++k) mx = kk[k] > mx ? kk[k] : mx;
+        for (int i = p.S + xt + NBR_KEEP * NBR_THREADS; i < n; i += NBR_THREADS) {
+            const unsigned long long k2 = key_at(i);
+            mx = k2 > mx ? k2 : mx;
+        }
+        if (xt == 0) s_cnt = 0;
+        const unsigned long long srt = warp_sort_desc(mx, lane);
+        if (lane < 8) s_top[xw * 8 + lane] = srt;
+        asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory");
+        // every warp sorts the NBR_WARPS x 8 warp leaders itself (no extra barrier)
+        const unsigned long long theta =
+            __shfl_sync(FULL, warp_sort_desc(lane < NBR_WARPS * 8 ? s_top[lane] : 0ull, lane), 7);
+        auto offer = [&](unsigned long long k2) {
+            if (k2 != 0ull && k2 >= theta) {
+                const int slot = atomicAdd(&s_cnt, 1);
+                if (slot < NBR_CAP) s_cand[slot] = k2;
+            }
+        };
+#pragma unroll
+        for (int k = 0; k < NBR_KEEP; ++k) offer(kk[k]);
+        for (int i = p.S + xt + NBR_KEEP * NBR_THREADS; i < n; i += NBR_THREADS) offer(key_at(i));
+        asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory");
+        if (xw == 0) {
+            const int cnt = s_cnt;
+            int32_t* outn = p.nbr8 + (size_t)u * 8;
+            if (cnt <= 32) {
+                const unsigned long long x = warp_sort_desc(lane < cnt ? s_cand[lane] : 0ull, lane);
+                if (lane < 8) outn[lane] = x ? nbr_pos(x) : -1;
+            } else {
+                // many candidates (ties in the logits): 8 rounds, each taking
+                // the best key below the previous winner, from the shared
+                // list or, past its capacity, from the whole list
+                unsigned long long prev = ~0ull;
+                for (int r = 0; r < 8; ++r) {
+                    unsigned long long best = 0;
+                    if (cnt <= NBR_CAP) {
+                        for (int c = lane; c < cnt; c += 32) {
+                            const unsigned long long k2 = s_cand[c];
+                            if (k2 < prev && k2 > best) best = k2;
+                        }
+                    } else {
+                        for (int i = p.S + lane; i < n; i += 32) {
+                            const unsigned long long k2 = key_at(i);
+                            if (k2 < prev && k2 > best) best = k2;
+                        }
+                    }
+                    best = warp_max_u64(best);
+                    if (lane == 0) outn[r] = best ? nbr_pos(best) : -1;
+                    prev = best;  // 0 once the entries run out: every later round finds none
                 }
-                v = v2;
-                q = q2;
             }
         }
-        int head = 0;  // this lane's best remaining candidate
-        for (int r = 0; r < 8; ++r) {
-            float bv = -INFINITY;
-            int bp = 0x7fffffff;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                if (k == head) {
-                    bv = cv[k];
-                    bp = cp[k];
-                }
-            float wv = bv;
-            int wp = bp;
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                const float ov = __shfl_xor_sync(FULL, wv, o);
-                const int op = __shfl_xor_sync(FULL, wp, o);
-                if (ov > wv || (ov == wv && op < wp)) {
-                    wv = ov;
-                    wp = op;
-                }
-            }
-            const bool valid = wp != 0x7fffffff;
-            if (lane == 0) p.nbr8[(size_t)u * 8 + r] = valid ? wp : -1;
-            if (valid && bp == wp) ++head;  // positions are unique: only the owner advances
-        }
+        return;
     }
 
-    // running max per head over all slots
-    float M[GQ];
-#pragma unroll
-    for (int h = 0; h < GQ; ++h) M[h] = -INFINITY;
-    for (int sl = t; sl < nslots; sl += blockDim.x)
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) M[h] = fmaxf(M[h], ws.m[(s0 + sl) * GQ + h]);
-#pragma unroll
-    for (int h = 0; h < GQ; ++h) {
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(FULL, M[h], o));
-        if (lane == 0) s_red[warp][h] = M[h];
-    }
-    __syncthreads();
-    if (t < GQ) {
-        float m = -INFINITY;
-        for (int w2 = 0; w2 < (int)(blockDim.x >> 5); ++w2) m = fmaxf(m, s_red[w2][t]);
-        s_M[t] = m;
-    }
-    __syncthreads();
-
-    float A[GQ], Lp[GQ];
+    if (t >= D) return;
+    // online merge, in slot order, of this thread's output dimension for every
+    // head: running max, rescaled sum and accumulator; all loads of a chunk of
+    // slots are issued before any is used
+    constexpr int CH = GQ >= 8 ? 4 : 32 / GQ;
+    float M[GQ], Ls[GQ], A[GQ];
 #pragma unroll
     for (int h = 0; h < GQ; ++h) {
+        M[h] = -INFINITY;
+        Ls[h] = 0.f;
         A[h] = 0.f;
-        Lp[h] = 0.f;
     }
-    for (int c0 = 0; c0 < nslots; c0 += MERGE_CHUNK) {
-        const int cnt = min(MERGE_CHUNK, nslots - c0);
-        for (int i = t; i < cnt; i += blockDim.x) {
+    for (int c0 = 0; c0 < nslots; c0 += CH) {
+        float xm[CH][GQ], xl[CH][GQ], xa[CH][GQ];
+        // unconditional loads at constant offsets from one base (the slot
+        // arrays carry MERGE_PAD spare slots, so a chunk never reads past
+        // them), masked afterwards by selects: every load of the chunk is in
+        // flight before the first is used
+        const float* mb = ws.m + (s0 + c0) * GQ;
+        const float* lb = ws.l + (s0 + c0) * GQ;
+        const float* ab = ws.acc + (s0 + c0) * GQ * D + t;
+#pragma unroll
+        for (int r = 0; r < CH; ++r) {
 #pragma unroll
             for (int h = 0; h < GQ; ++h) {
-                const size_t sl = (s0 + c0 + i) * GQ + h;
-                const float f = exp2f(ws.m[sl] - s_M[h]);
-                s_f[i][h] = f;
-                Lp[h] = fmaf(ws.l[sl], f, Lp[h]);
+                xm[r][h] = mb[r * GQ + h];
+                xl[r][h] = lb[r * GQ + h];
+                xa[r][h] = ab[(r * GQ + h) * D];
             }
         }
-        __syncthreads();
-        if (t < D) {
-            int j = 0;
-            for (; j + 8 <= cnt; j += 8) {
-                float x[8][GQ];
 #pragma unroll
-                for (int r = 0; r < 8; ++r)
+        for (int r = 0; r < CH; ++r) {
+            const bool ok = c0 + r < nslots;
 #pragma unroll
-                    for (int h = 0; h < GQ; ++h) x[r][h] = ws.acc[((s0 + c0 + j + r) * GQ + h) * D + t];
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-#pragma unroll
-                    for (int h = 0; h < GQ; ++h) A[h] = fmaf(x[r][h], s_f[j + r][h], A[h]);
+            for (int h = 0; h < GQ; ++h) {
+                xm[r][h] = ok ? xm[r][h] : -INFINITY;
+                xl[r][h] = ok ? xl[r][h] : 0.f;
+                xa[r][h] = ok ? xa[r][h] : 0.f;
             }
-            for (; j < cnt; ++j)
-#pragma unroll
-                for (int h = 0; h < GQ; ++h) A[h] = fmaf(ws.acc[((s0 + c0 + j) * GQ + h) * D + t], s_f[j][h], A[h]);
         }
-        __syncthreads();
-    }
-    // sum of the weights per head
-#pragma unroll
-    for (int h = 0; h < GQ; ++h) {
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) Lp[h] += __shfl_xor_sync(FULL, Lp[h], o);
-        if (lane == 0) s_red[warp][h] = Lp[h];
-    }
-    __syncthreads();
-    if (t < D) {
+        // the chunk's maximum first, then independent weights: the dependent
+        // chain per chunk is one rescale instead of one per slot
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
-            float L = 0.f;
-            for (int w2 = 0; w2 < (int)(blockDim.x >> 5); ++w2) L += s_red[w2][h];
-            outu[h * D + t] = A[h] / L;
+            float mc = -INFINITY;
+#pragma unroll
+            for (int r = 0; r < CH; ++r) mc = fmaxf(mc, xm[r][h]);
+            if (mc == -INFINITY) continue;
+            const float mn = fmaxf(M[h], mc);
+            const float fo = exp2_approx(M[h] - mn);
+            float ls = 0.f, a = 0.f;
+#pragma unroll
+            for (int r = 0; r < CH; ++r) {
+                const float f = exp2_approx(xm[r][h] - mn);
+                ls = fmaf(xl[r][h], f, ls);
+                a = fmaf(xa[r][h], f, a);
+            }
+            Ls[h] = fmaf(Ls[h], fo, ls);
+            A[h] = fmaf(A[h], fo, a);
+            M[h] = mn;
         }
     }
+#pragma unroll
+    for (int h = 0; h < GQ; ++h) outu[h * D + t] = A[h] / Ls[h];
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 
-size_t decode_ws_bytes(int U, int gq, int d) {
-    const size_t slots = (size_t)MAX_DECODE_WARPS + U;
-    return align256(slots * gq * 4) * 2 + align256(slots * gq * d * 4) + align256(slots * 8 * 4) * 2;
+size_t decode_ws_bytes(int U, int gq, int d, int lam_cap) {
+    const size_t slots = (size_t)MAX_DECODE_WARPS + U + MERGE_PAD;
+    return align256(slots * gq * 4) * 2 + align256(slots * gq * d * 4) + align256((size_t)U * lam_cap * 4);
 }
 
-DecodeWs carve_decode_ws(void* ws, int U, int gq, int d) {
-    const size_t slots = (size_t)MAX_DECODE_WARPS + U;
+DecodeWs carve_decode_ws(void* ws, int U, int gq, int d, int lam_cap) {
+    const size_t slots = (size_t)MAX_DECODE_WARPS + U + MERGE_PAD;
     char* p = static_cast<char*>(ws);
     DecodeWs w;
     w.m = reinterpret_cast<float*>(p);
@@ -579,9 +620,8 @@ DecodeWs carve_decode_ws(void* ws, int U, int gq, int d) {
     p += align256(slots * gq * 4);
     w.acc = reinterpret_cast<float*>(p);
     p += align256(slots * gq * d * 4);
-    w.tv = reinterpret_cast<float*>(p);
-    p += align256(slots * 8 * 4);
-    w.tp = reinterpret_cast<int32_t*>(p);
+    w.lam = reinterpret_cast<float*>(p);
+    w.lam_cap = lam_cap;
     return w;
 }
 
@@ -605,7 +645,7 @@ cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.U);
-    cfg.blockDim = dim3(D + 32);
+    cfg.blockDim = dim3(D + (DENSE ? 0 : 32 * NBR_WARPS));
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -657,7 +697,7 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
     p.unit_prefix = s.unit_prefix;
     p.n_tok = s.n_tok;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
-    p.ws = carve_decode_ws(ws, p.U, g.gq, c.d);
+    p.ws = carve_decode_ws(ws, p.U, g.gq, c.d, s.tok_cap);
     p.want_nbr = nbr8 != nullptr;
     p.out = out;
     p.nbr8 = nbr8;
@@ -681,7 +721,7 @@ cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float*
     p.T = T;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
     const int gq = c.Hq / c.Hkv;
-    p.ws = carve_decode_ws(ws, p.U, gq, c.d);
+    p.ws = carve_decode_ws(ws, p.U, gq, c.d, 0);
     p.out = out;
     return dispatch<true>(c, gq, p, st);
 }

@@ -210,14 +210,16 @@ struct DecodeWs {
     float* m;      // [slots, GQ]
     float* l;      // [slots, GQ]
     float* acc;    // [slots, GQ, D]
-    float* tv;     // [slots, 8]
-    int32_t* tp;   // [slots, 8]
+    float* lam;    // [U * lam_cap] graph logit of every selected token (sparse only)
+    int lam_cap;   // list entries per unit
 };
 
 size_t build_ws_bytes(int U, int Cmax, int T_cap);
 size_t select_ws_bytes(int U, int Cmax);
-size_t decode_ws_bytes(int U, int gq, int d);
-DecodeWs carve_decode_ws(void* ws, int U, int gq, int d);
+// lam_cap: selection entries per unit whose graph logits are kept (the
+// selection's tok_cap; 0 for the dense comparator)
+size_t decode_ws_bytes(int U, int gq, int d, int lam_cap);
+DecodeWs carve_decode_ws(void* ws, int U, int gq, int d, int lam_cap);
 
 cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* labels,
                          int64_t labels_stride, int T, void* ws, cudaStream_t st);

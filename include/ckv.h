@@ -212,10 +212,14 @@ CKV_API ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q,
  * computed by the same kernels; the split-K scratch instead lives in a
  * 32 MiB array inside libckv that every GPU which loads the library keeps
  * until the process exits.
- *   - Calls needing more scratch than CKV_NOALLOC_SCRATCH_BYTES (the size
- *     ckv_workspace_size's attention part reports for these shapes; e.g.
- *     Hq/Hkv = 8 with d = 128 in per-group mode) return CKV_ERR_UNSUPPORTED
- *     before touching the device.
+ *   - Calls needing more scratch than CKV_NOALLOC_SCRATCH_BYTES return
+ *     CKV_ERR_UNSUPPORTED before touching the device.  The need is the size
+ *     ckv_workspace_size's attention part reports for these shapes: about
+ *     4 * (8192 + U) * gq * (d + 2) bytes of split-K partials (gq query
+ *     heads per graph, U = B * graphs per sequence) plus 4 * U * sel->tok_cap
+ *     bytes of neighbour logits.  Per-head graphs with d = 128 need about
+ *     4.3 MiB + the logits; Hq/Hkv = 8 with d = 128 in per-group mode needs
+ *     over 32 MiB and is refused.
  *   - The first call on each device looks up the array's device address
  *     (with that device current); make that first call before any stream
  *     capture.  No call allocates or frees memory.

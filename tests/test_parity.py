@@ -183,3 +183,22 @@ def test_bad_labels_are_flagged_and_skipped():
     comm_of = case.st.graph.comm_of.cpu().numpy()
     assert comm_of[0, 1] == -1 and comm_of[1, 100] == -1
     assert int(case.st.graph.cnt.sum().item()) == wl.B * wl.G * (wl.T - wl.S) - 1
+
+
+@pytest.mark.parametrize("T", [6000, 40000])
+def test_neighbours_crowded_threshold(T):
+    """Tokens planted with identical keys, all in one thread's share of the
+    list (every 128th entry of a single community), crowd the neighbour
+    search's candidate set past one warp (T = 6000) and past its shared-memory
+    capacity (T = 40000).  The exact ties resolve to the lowest positions."""
+    wl = small(f"crowded_{T}", 37, B=1, Hq=1, Hkv=1, T=T, budgets=(64,), steps=1)
+    labels = np.zeros((wl.B, wl.G, wl.T), dtype=np.int32)
+    labels[:, :, : wl.S] = -1
+    case = Case(wl, labels=labels)
+    q = synth.draw_queries(wl, case.draw, 0)
+    planted = np.arange(wl.S, wl.T, 128)
+    case.st.K[0, 0, torch.from_numpy(planted).cuda()] = (3.0 * q[0, 0].float()).to(case.st.K.dtype)
+    case.st.build(torch.from_numpy(labels.reshape(case.U, wl.T)).cuda(), wl.T)
+    rep = case.step(wl.budget)
+    assert rep.band_neighbours == 0
+    assert case.st.nbr8[0].cpu().tolist() == planted[:8].tolist()
