@@ -20,7 +20,8 @@ __all__ = [
     "CKVError", "lib", "LIB_PATH", "CacheDesc", "GraphDesc", "SelectionDesc",
     "Graph", "Selection", "cache_desc", "new_graph", "new_selection", "new_workspace",
     "ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-    "ckv_sparse_decode_noalloc", "NOALLOC_SCRATCH_BYTES", "ckv_assign_update", "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
+    "ckv_sparse_decode_noalloc", "NOALLOC_SCRATCH_BYTES", "ckv_assign_update", "ckv_append_assign",
+    "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP",
     "NEIGHBOURS",
@@ -35,8 +36,8 @@ PER_GROUP, PER_HEAD = 0, 1
 DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
 NEIGHBOURS = 8
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_dense_decode", "ckv_status_string",
-            "ckv_last_error", "ckv_abi_version")
+            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_dense_decode",
+            "ckv_status_string", "ckv_last_error", "ckv_abi_version")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -78,9 +79,10 @@ lib.ckv_score_select.argtypes = [_P(CacheDesc), _P(GraphDesc), _p, _i32, _P(Sele
 lib.ckv_sparse_decode.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p, _sz, _p]
 lib.ckv_sparse_decode_noalloc.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p]
 lib.ckv_assign_update.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p]
+lib.ckv_append_assign.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p, _p, _p]
 lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
 for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-           "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_dense_decode"):
+           "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_dense_decode"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.ckv_status_string.argtypes = [ctypes.c_int]
 lib.ckv_status_string.restype = ctypes.c_char_p
@@ -256,6 +258,19 @@ def ckv_assign_update(cache: CacheDesc, graph: Graph, pos: int, nbr8: torch.Tens
     _check(lib.ckv_assign_update(ctypes.byref(cache), ctypes.byref(graph.desc), pos, nbr8.data_ptr(),
                                  _ptr(assigned), _stream(stream)),
            "ckv_assign_update")
+
+
+def ckv_append_assign(cache: CacheDesc, graph: Graph, pos: int, k_new: torch.Tensor, v_new: torch.Tensor,
+                      nbr8: torch.Tensor, assigned: Optional[torch.Tensor], stream=None) -> None:
+    """k_new, v_new: [B, Hkv, d] contiguous in the cache dtype; written to
+    row ``pos`` of K and V by the library, then the update runs."""
+    shape = (cache.B, cache.Hkv, cache.d)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {shape} tensor, got {tuple(t.shape)}")
+    _check(lib.ckv_append_assign(ctypes.byref(cache), ctypes.byref(graph.desc), pos, k_new.data_ptr(),
+                                 v_new.data_ptr(), nbr8.data_ptr(), _ptr(assigned), _stream(stream)),
+           "ckv_append_assign")
 
 
 def ckv_dense_decode(cache: CacheDesc, q: torch.Tensor, T: int, out: torch.Tensor, ws: torch.Tensor,

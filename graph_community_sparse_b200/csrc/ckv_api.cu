@@ -280,9 +280,24 @@ ckv_status ckv_assign_update(const ckv_cache_desc* cache, const ckv_graph_desc* 
     CKV_TRY(check_graph(cache, graph));
     if (!nbr8) return fail(CKV_ERR_INVALID_ARG, "nbr8 is NULL");
     if (pos < 0 || pos >= cache->T_cap) return fail(CKV_ERR_CAPACITY, "pos = %d outside [0, T_cap)", pos);
-    return cuda_status(ckv::launch_assign_update(cache_view(cache), graph_view(cache, graph), pos, nbr8, assigned,
-                                                 reinterpret_cast<cudaStream_t>(stream)),
+    return cuda_status(ckv::launch_assign_update(cache_view(cache), graph_view(cache, graph), pos, nullptr,
+                                                 nullptr, nbr8, assigned, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_assign_update");
+}
+
+ckv_status ckv_append_assign(const ckv_cache_desc* cache, const ckv_graph_desc* graph, int32_t pos,
+                             const void* k_new, const void* v_new, const int32_t* nbr8, int32_t* assigned,
+                             ckv_stream_t stream) {
+    CKV_TRY(check_cache(cache, true));
+    CKV_TRY(check_graph(cache, graph));
+    if (!nbr8) return fail(CKV_ERR_INVALID_ARG, "nbr8 is NULL");
+    if (!k_new || !v_new) return fail(CKV_ERR_INVALID_ARG, "k_new or v_new is NULL");
+    if ((reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(v_new)) & 15)
+        return fail(CKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+    if (pos < 0 || pos >= cache->T_cap) return fail(CKV_ERR_CAPACITY, "pos = %d outside [0, T_cap)", pos);
+    return cuda_status(ckv::launch_assign_update(cache_view(cache), graph_view(cache, graph), pos, k_new, v_new,
+                                                 nbr8, assigned, reinterpret_cast<cudaStream_t>(stream)),
+                       "ckv_append_assign");
 }
 
 ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t T, float* out, void* ws,

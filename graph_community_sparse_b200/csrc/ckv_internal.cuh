@@ -233,8 +233,10 @@ cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float*
 // per device, with that device current).
 cudaError_t static_decode_scratch(void** ptr, size_t* bytes);
 
-cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const int32_t* nbr8,
-                                 int32_t* assigned, cudaStream_t st);
+// k_new/v_new NULL: the new key is read from the cache at pos; otherwise it
+// comes from k_new and both rows are first written to the cache at pos.
+cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const void* k_new,
+                                 const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 

@@ -17,9 +17,16 @@
 namespace ckv {
 
 struct AssignParams {
-    const void* k;
-    int64_t sb, sh, st;
-    int U, G, Hq, Hkv, per_head, Cmax, T_cap, max_tail, pos;
+    const void* k;      // new key rows: the cache at pos, or the caller's k_new
+    int64_t sb, sh;     // element strides of k between sequences / KV heads
+    // fused append (ckv_append_assign): copy the caller's rows into the cache
+    const void* k_new;
+    const void* v_new;
+    void* k_dst;        // K row (b = 0, kv head 0) at pos; NULL: no append
+    void* v_dst;
+    int64_t csb, csh;   // cache element strides between sequences / KV heads
+    int row_vec;        // 16-byte vectors per row
+    int U, G, Hq, Hkv, d, per_head, Cmax, T_cap, max_tail, pos;
     float inv_sqrt_d;
     const int32_t* nbr8;
     int32_t* comm_of;
@@ -42,9 +49,25 @@ __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParam
     __shared__ int s_cand[CKV_NEIGHBOURS];
     __shared__ float s_score[CKV_NEIGHBOURS];
     __shared__ int s_best, s_n, s_tl;
+    // everything this kernel reads may come from the kernel before it
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = u / p.G, g = u - b * p.G;
-    const int kvh = p.per_head ? g / (p.Hq / p.Hkv) : g;
+    const int gq = p.Hq / p.Hkv;
+    const int kvh = p.per_head ? g / gq : g;
+    if (p.k_dst && (!p.per_head || g % gq == 0) && warp == CKV_NEIGHBOURS - 1) {
+        // the first graph of each (sequence, KV head) appends its K and V rows
+        const uint4* ks = static_cast<const uint4*>(p.k_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
+        const uint4* vs = static_cast<const uint4*>(p.v_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
+        const size_t eoff = (size_t)(b * p.csb + kvh * p.csh);  // elements
+        const size_t esz = p.row_vec * 16 / (size_t)p.d;
+        uint4* kd = reinterpret_cast<uint4*>(static_cast<char*>(p.k_dst) + eoff * esz);
+        uint4* vd = reinterpret_cast<uint4*>(static_cast<char*>(p.v_dst) + eoff * esz);
+        for (int i = lane; i < p.row_vec; i += 32) {
+            kd[i] = ks[i];
+            vd[i] = vs[i];
+        }
+    }
     if (tid < CKV_NEIGHBOURS) {
         int c = -1;
         const int np = p.nbr8[(size_t)u * CKV_NEIGHBOURS + tid];
@@ -57,7 +80,7 @@ __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParam
     if (tid == 0) {
         s_tl = p.tail_len[u];
     }
-    const T* krow = static_cast<const T*>(p.k) + b * p.sb + kvh * p.sh + (int64_t)p.pos * p.st + lane * E;
+    const T* krow = static_cast<const T*>(p.k) + b * p.sb + kvh * p.sh + lane * E;
     float kx[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) kx[e] = to_f32(krow[e]);
@@ -125,17 +148,33 @@ __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParam
     }
 }
 
-cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const int32_t* nbr8,
-                                 int32_t* assigned, cudaStream_t st) {
+cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const void* k_new,
+                                 const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st) {
     AssignParams p{};
-    p.k = c.k;
-    p.sb = c.sb;
-    p.sh = c.sh;
-    p.st = c.st;
+    const size_t esz = c.dtype == CKV_DTYPE_BF16 ? 2 : 4;
+    if (k_new) {
+        // new key from the caller's contiguous [B, Hkv, d] rows; append them
+        p.k = k_new;
+        p.sb = (int64_t)c.Hkv * c.d;
+        p.sh = c.d;
+        p.k_new = k_new;
+        p.v_new = v_new;
+        p.k_dst = const_cast<char*>(static_cast<const char*>(c.k)) + (size_t)pos * c.st * esz;
+        p.v_dst = const_cast<char*>(static_cast<const char*>(c.v)) + (size_t)pos * c.st * esz;
+    } else {
+        // new key already in the cache at pos
+        p.k = static_cast<const char*>(c.k) + (size_t)pos * c.st * esz;
+        p.sb = c.sb;
+        p.sh = c.sh;
+    }
+    p.csb = c.sb;
+    p.csh = c.sh;
+    p.row_vec = (int)(c.d * esz / 16);
     p.U = c.B * g.G;
     p.G = g.G;
     p.Hq = c.Hq;
     p.Hkv = c.Hkv;
+    p.d = c.d;
     p.per_head = g.mode == CKV_GRAPH_PER_HEAD;
     p.Cmax = g.Cmax;
     p.T_cap = g.T_cap;
@@ -151,15 +190,25 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
     p.tail_len = g.tail_len;
     p.dev_err = g.dev_err;
     p.assigned = assigned;
-    const int threads = CKV_NEIGHBOURS * 32;
+    if (p.U <= 0) return cudaSuccess;
+    // programmatic dependent launch: the block launch overlaps the previous
+    // kernel's tail; the kernel waits for it before its first load
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.U);
+    cfg.blockDim = dim3(CKV_NEIGHBOURS * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (c.dtype == CKV_DTYPE_BF16) {
-        if (c.d == 128) assign_kernel<__nv_bfloat16, 128><<<p.U, threads, 0, st>>>(p);
-        else assign_kernel<__nv_bfloat16, 64><<<p.U, threads, 0, st>>>(p);
-    } else {
-        if (c.d == 128) assign_kernel<float, 128><<<p.U, threads, 0, st>>>(p);
-        else assign_kernel<float, 64><<<p.U, threads, 0, st>>>(p);
+        if (c.d == 128) return cudaLaunchKernelEx(&cfg, assign_kernel<__nv_bfloat16, 128>, p);
+        return cudaLaunchKernelEx(&cfg, assign_kernel<__nv_bfloat16, 64>, p);
     }
-    return cudaGetLastError();
+    if (c.d == 128) return cudaLaunchKernelEx(&cfg, assign_kernel<float, 128>, p);
+    return cudaLaunchKernelEx(&cfg, assign_kernel<float, 64>, p);
 }
 
 }  // namespace ckv

@@ -10,7 +10,7 @@ from typing import Optional
 
 import torch
 
-from . import (PER_GROUP, PER_HEAD, Graph, Selection, cache_desc, ckv_assign_update,
+from . import (PER_GROUP, PER_HEAD, Graph, Selection, cache_desc, ckv_append_assign, ckv_assign_update,
                ckv_build_centroids, ckv_dense_decode, ckv_score_select, ckv_sparse_decode,
                ckv_workspace_size, new_graph, new_selection, new_workspace, NEIGHBOURS)
 
@@ -59,8 +59,17 @@ class LayerState:
         return self.attend(q, want_nbr, stream)
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> torch.Tensor:
-        """Write the new token's K/V rows ([B, Hkv, d]) at position T (the
-        model's ordinary cache append) and let it join a community."""
+        """Write the new token's K/V rows ([B, Hkv, d]) at position T and let
+        it join a community: one library call (ckv_append_assign)."""
+        pos = self.T
+        ckv_append_assign(self.cache, self.graph, pos, k_new.contiguous(), v_new.contiguous(), self.nbr8,
+                          self.assigned, stream)
+        self.T += 1
+        return self.assigned
+
+    def append_external(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> torch.Tensor:
+        """Same result for a caller that writes the cache itself: the rows are
+        copied with PyTorch, then ckv_assign_update reads the key from K."""
         pos = self.T
         self.K[:, :, pos].copy_(k_new)
         self.V[:, :, pos].copy_(v_new)

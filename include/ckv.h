@@ -87,8 +87,9 @@ typedef enum { CKV_GRAPH_PER_GROUP = 0, CKV_GRAPH_PER_HEAD = 1 } ckv_graph_mode;
  * The full KV cache of one layer: K and V are [B, Hkv, T_cap, d] with the d
  * elements of a row contiguous; strides are in elements and their byte
  * values must be multiples of 16 (as must the base pointers).  The library
- * only reads it; no call writes K or V.  [R-A] paragraph 5: the cache stays
- * whole so any fragment can be selected again later.
+ * only reads it, except ckv_append_assign, which writes row `pos` of K and V
+ * and nothing else.  [R-A] paragraph 5: the cache stays whole so any
+ * fragment can be selected again later.
  */
 typedef struct {
     int32_t dtype;  /* ckv_dtype, also the dtype of q */
@@ -247,6 +248,19 @@ CKV_API ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const 
 CKV_API ckv_status ckv_assign_update(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
                              int32_t pos, const int32_t* nbr8, int32_t* assigned,
                              ckv_stream_t stream);
+
+/*
+ * The decode step's cache append fused with ckv_assign_update: writes the new
+ * token's rows k_new and v_new (each [B, Hkv, d] in the cache dtype,
+ * contiguous, 16-byte aligned) at position `pos` of K and V, then updates
+ * every graph unit exactly as ckv_assign_update does, taking the new key from
+ * k_new.  One launch; the only call that writes the cache, and only row pos
+ * (the selection of the step that produced nbr8 never holds pos, so no
+ * read of this step races with the write).  0 <= pos < T_cap.
+ */
+CKV_API ckv_status ckv_append_assign(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
+                                     int32_t pos, const void* k_new, const void* v_new,
+                                     const int32_t* nbr8, int32_t* assigned, ckv_stream_t stream);
 
 /*
  * Dense comparator: exact GQA decode attention over positions [0, T) of every

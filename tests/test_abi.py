@@ -148,6 +148,14 @@ CASES = [
                                                      FAKE, FAKE, None), CAPACITY),
     ("assign null nbr", lambda: ckv.lib.ckv_assign_update(ctypes.byref(_cache()), ctypes.byref(_graph()), 5,
                                                           None, FAKE, None), INVALID),
+    ("append pos", lambda: ckv.lib.ckv_append_assign(ctypes.byref(_cache()), ctypes.byref(_graph()), -1,
+                                                     FAKE, FAKE, FAKE, FAKE, None), CAPACITY),
+    ("append null k_new", lambda: ckv.lib.ckv_append_assign(ctypes.byref(_cache()), ctypes.byref(_graph()), 5,
+                                                            None, FAKE, FAKE, FAKE, None), INVALID),
+    ("append misaligned v_new", lambda: ckv.lib.ckv_append_assign(ctypes.byref(_cache()), ctypes.byref(_graph()),
+                                                                  5, FAKE, FAKE + 8, FAKE, FAKE, None), INVALID),
+    ("append null nbr", lambda: ckv.lib.ckv_append_assign(ctypes.byref(_cache()), ctypes.byref(_graph()), 5,
+                                                          FAKE, FAKE, None, FAKE, None), INVALID),
     ("dense T", lambda: ckv.lib.ckv_dense_decode(ctypes.byref(_cache()), FAKE, 0, FAKE, FAKE, 1 << 40, None),
      CAPACITY),
     ("dense ws", lambda: ckv.lib.ckv_dense_decode(ctypes.byref(_cache()), FAKE, 100, FAKE, FAKE, 8, None),

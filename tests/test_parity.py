@@ -202,3 +202,25 @@ def test_neighbours_crowded_threshold(T):
     rep = case.step(wl.budget)
     assert rep.band_neighbours == 0
     assert case.st.nbr8[0].cpu().tolist() == planted[:8].tolist()
+
+
+def test_append_assign_matches_external_append():
+    """ckv_append_assign (the library writes row pos, key from k_new) leaves
+    the cache and graph exactly as a PyTorch append + ckv_assign_update."""
+    wl = small("append", 38, steps=3)
+    a, b = Case(wl), Case(wl)
+    for i in range(wl.steps):
+        q = synth.draw_queries(wl, a.draw, i)
+        a.st.decode(q, wl.budget)
+        b.st.decode(q, wl.budget)
+        kn, vn = synth.draw_new_tokens(wl, a.draw, i)
+        kn, vn = kn.to(a.st.K.dtype), vn.to(a.st.V.dtype)
+        ga = a.st.append(kn, vn).clone()
+        gb = b.st.append_external(kn, vn).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(ga, gb)
+        pos = a.st.T - 1
+        assert torch.equal(a.st.K[:, :, pos], kn) and torch.equal(a.st.V[:, :, pos], vn)
+        assert torch.equal(a.st.K, b.st.K) and torch.equal(a.st.V, b.st.V)
+        for name in ("comm_of", "cnt", "cent", "tail_tok", "tail_comm", "tail_len", "dev_err"):
+            assert torch.equal(getattr(a.st.graph, name), getattr(b.st.graph, name)), name
