@@ -12,7 +12,8 @@
 // [w*per, (w+1)*per) with per = ceil(total/W), whatever units it crosses, so
 // every warp reads the same number of K/V rows regardless of how skewed the
 // community sizes are.  A warp writes one partial (running max m, sum l,
-// unnormalised accumulator, top-8 logits) per unit segment into slot w + u,
+// unnormalised accumulator) per unit segment into slot w + u, and, when
+// neighbours are wanted, each list entry's graph logit;
 // which is unique because slices and units are both contiguous and ordered.
 // All warps of the persistent grid finish together, so the merge of each
 // unit's slots is a second, small kernel launched as a programmatic
@@ -311,6 +312,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 template <typename T, int D, int GQ, bool DENSE>
 __global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(DecodeParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
+    pdl_wait();  // the selection comes from the kernel before
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned char* wsm = smem + warp * DecSmem<T, D, GQ>::WARP;
     int* s_pre = reinterpret_cast<int*>(smem + DecSmem<T, D, GQ>::CTA_FIXED);
@@ -423,8 +425,7 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x)
 // dependent rounds of loads.
 template <int D, int GQ, bool DENSE>
 __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_merge(DecodeParams p) {
-    // wait until the attention kernel's partials are complete and visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();  // the attention kernel's partials are complete and visible
     const int u = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     int b, kvh, h0;
     unit_heads(p, u, GQ, DENSE, b, kvh, h0);
@@ -639,21 +640,9 @@ cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
     int blocks = sms * per_sm;
     if (blocks * DEC_WARPS > MAX_DECODE_WARPS) blocks = MAX_DECODE_WARPS / DEC_WARPS;
     p.W = blocks * DEC_WARPS;
-    kern<<<blocks, DEC_WARPS * 32, smem, st>>>(p);
-    e = cudaGetLastError();
+    e = launch_pdl(kern, dim3(blocks), dim3(DEC_WARPS * 32), smem, st, p);
     if (e != cudaSuccess) return e;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.U);
-    cfg.blockDim = dim3(D + (DENSE ? 0 : 32 * NBR_WARPS));
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_merge<D, GQ, DENSE>, p);
+    return launch_pdl(decode_merge<D, GQ, DENSE>, dim3(p.U), dim3(D + (DENSE ? 0 : 32 * NBR_WARPS)), 0, st, p);
 }
 
 template <bool DENSE>

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <utility>
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -239,6 +240,32 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
                                  const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Programmatic dependent launch.  Kernels launched by launch_pdl() start
+// with pdl_wait(), so they read and write nothing before the previous kernel
+// in the stream has completed and its memory is visible; what overlaps is
+// the launch itself (block scheduling) with that kernel's tail.  No kernel
+// signals its dependents early: measured on the step, letting the next
+// kernel's blocks take SM slots before the previous kernel ends slowed the
+// scoring and selection and did not speed up the attention.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 
 // Launch-shape cache for one kernel: the dynamic shared memory limit it was
 // raised to and its resident blocks per SM, per device, so that steady-state

@@ -18,8 +18,9 @@
 //  * select_kernel, one block per unit, launched as a programmatic
 //    dependent (its launch overlaps the scoring; it waits in hardware for the
 //    scores): the histogram gives the bin the budget cut falls in; only the
-//    keys from that bin up (typically a few dozen) are sorted, in registers;
-//    a scan of their sizes gives the cut (at least the top community).  Then
+//    keys from that bin up (typically a few dozen) are ranked, each against
+//    all the others in shared memory, which also gives the size above it and
+//    so the cut (at least the top community), with no sort.  Then
 //    the unit's token list: sinks, build-time members of each selected
 //    community (from the community-contiguous CSR), then the selected tail
 //    members.
@@ -90,24 +91,6 @@ __device__ int block_scan_inplace(int* a, int n, int* s_warp) {
     return total;
 }
 
-// Bitonic sort of one (key, weight) pair per lane across a warp, keys descending.
-__device__ __forceinline__ void warp_sort_desc(unsigned long long& v, int& w, int lane) {
-#pragma unroll
-    for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            const unsigned long long o = __shfl_xor_sync(FULL, v, j);
-            const int ow = __shfl_xor_sync(FULL, w, j);
-            const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
-            const bool take = keep_max ? (o > v) : (o < v);
-            if (take) {
-                v = o;
-                w = ow;
-            }
-        }
-    }
-}
-
 // Scores of this block's (up to) SCORE_ROWS centres of unit u.
 template <typename T, int D, int GQ>
 __device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) {
@@ -174,6 +157,16 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     const float* sc = p.scores + (size_t)u * p.Cmax;
     const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
     const int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
+    // The pages this block writes or reads late (token list, members, CSR
+    // offsets, ranked ids) are touched now by prefetches, so their address
+    // translations overlap the first loads instead of stalling the copy.
+    if (tid < 4) {
+        const void* pg = tid == 0 ? (const void*)(p.sel_tok + (size_t)u * p.tok_cap)
+                       : tid == 1 ? (const void*)(p.tok + (size_t)u * p.T_cap)
+                       : tid == 2 ? (const void*)(p.offs + (size_t)u * (p.Cmax + 1))
+                                  : (const void*)(p.sel_comm + (size_t)u * p.Cmax);
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pg));
+    }
     for (int i = tid; i < (p.Cmax + 31) / 32; i += nt) s_mask[i] = 0u;
     if (tid == 0) {
         s_bstar = -1;
@@ -181,16 +174,35 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         s_cnt = 0;
     }
 
+    // Every load that depends on nothing but u is issued first, together:
+    // the histogram (16 bins per thread as four 16-byte loads) and the first
+    // round of community sizes and scores (from clamped in-range ids, masked
+    // by c < C later).
+    constexpr int RND = 8;
+    constexpr int per = SEL_HBINS / SEL_THREADS;
+    static_assert(per == 16, "four int4 histogram loads per thread");
+    int4 hv[4];
+    {
+        const int4* h4 = reinterpret_cast<const int4*>(hist + per * tid);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) hv[i] = __ldcg(h4 + i);
+    }
+    int wv[RND];
+    float sv[RND];
+#pragma unroll
+    for (int r = 0; r < RND; ++r) {
+        const int c = min(tid + r * nt, p.Cmax - 1);
+        wv[r] = cn[c];
+        sv[r] = __ldcg(sc + c);
+    }
+
     // 1. crossing bin: thread t owns bins [per*t, per*t + per)
     {
-        constexpr int per = SEL_HBINS / SEL_THREADS;
-        int hw[per];
+        const int hw[per] = {hv[0].x, hv[0].y, hv[0].z, hv[0].w, hv[1].x, hv[1].y, hv[1].z, hv[1].w,
+                             hv[2].x, hv[2].y, hv[2].z, hv[2].w, hv[3].x, hv[3].y, hv[3].z, hv[3].w};
         int own = 0;
 #pragma unroll
-        for (int i = 0; i < per; ++i) {
-            hw[i] = __ldcg(hist + per * tid + i);
-            own += hw[i];
-        }
+        for (int i = 0; i < per; ++i) own += hw[i];
         int total;
         const int pre = block_exclusive_scan(own, s_warp, &total);  // also orders the inits above
         int above = total - pre - own;  // weight of every bin above this thread's
@@ -206,67 +218,66 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     __syncthreads();
     const int bstar = max(s_bstar, 0);  // no crossing: every key is a candidate
 
-    // 2. candidates: keys from the crossing bin up, with their sizes (the
-    //    loads of a round are all issued before any is used)
-    constexpr int RND = 8;
-    for (int c0 = tid; c0 < C; c0 += RND * nt) {
-        int wv[RND];
-        float sv[RND];
-#pragma unroll
-        for (int r = 0; r < RND; ++r) {
-            const int c = c0 + r * nt;
-            wv[r] = c < C ? cn[c] : 0;
-            sv[r] = c < C ? __ldcg(sc + c) : 0.f;
-        }
-#pragma unroll
-        for (int r = 0; r < RND; ++r) {
-            const int c = c0 + r * nt;
-            if (wv[r] <= 0) continue;
-            const unsigned long long k = score_key(sv[r], c);
-            if ((int)(k >> (64 - SEL_HBITS)) >= bstar) {
-                const int i = atomicAdd(&s_nc, 1);
-                if (i < SEL_FAST) {
-                    s_key[i] = k;
-                    s_w[i] = wv[r];
-                }
+    // 2. candidates: keys from the crossing bin up, with their sizes
+    auto offer = [&](int c, int w, float sval) {
+        if (c >= C || w <= 0) return;
+        const unsigned long long k = score_key(sval, c);
+        if ((int)(k >> (64 - SEL_HBITS)) >= bstar) {
+            const int i = atomicAdd(&s_nc, 1);
+            if (i < SEL_FAST) {
+                s_key[i] = k;
+                s_w[i] = w;
             }
         }
+    };
+#pragma unroll
+    for (int r = 0; r < RND; ++r) offer(tid + r * nt, wv[r], sv[r]);
+    for (int c0 = tid + RND * nt; c0 < C; c0 += RND * nt) {
+#pragma unroll
+        for (int r = 0; r < RND; ++r) {
+            const int c = min(c0 + r * nt, p.Cmax - 1);
+            wv[r] = cn[c];
+            sv[r] = __ldcg(sc + c);
+        }
+#pragma unroll
+        for (int r = 0; r < RND; ++r) offer(c0 + r * nt, wv[r], sv[r]);
     }
     __syncthreads();
     const int nc = s_nc;
 
+    // 3. the cut.  Few candidates (the usual case): no sort; candidate i's
+    //    rank is the number of larger keys and the weight above it their size
+    //    sum, so it is selected iff that sum plus its own size fits the budget
+    //    (sizes are positive, so the selected set is a prefix of the ranking).
+    //    Each candidate's CSR run is looked up meanwhile and stored at its rank.
     int kstar;
     const unsigned long long* sorted;
-    if (nc <= SEL_FAST) {
-        unsigned long long v = tid < nc ? s_key[tid] : 0ull;
-        int w = tid < nc ? s_w[tid] : 0;
-        warp_sort_desc(v, w, lane);
-        s_runs[tid] = v;
-        __syncthreads();
-        if (v) {
-            int r = lane;
-            for (int w2 = 0; w2 < nw; ++w2) {
-                if (w2 == warp) continue;
-                const unsigned long long* run = s_runs + 32 * w2;
-                int lo = 0, hi = 32;  // count of entries > v (runs are descending)
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (run[mid] > v) lo = mid + 1;
-                    else hi = mid;
-                }
-                r += lo;
+    const int32_t* of = p.offs + (size_t)u * (p.Cmax + 1);
+    const bool small = nc <= SEL_FAST;
+    int* bsz = small ? s_bsz : p.gw + (size_t)u * p.npow_max;
+    if (small) {
+        bool in = false;
+        if (tid < nc) {
+            const unsigned long long k = s_key[tid];
+            const int w = s_w[tid];
+            const int c = key_id(k);
+            const int o0 = of[c], o1 = of[c + 1];
+            int rank = 0, above = 0;
+            for (int j = 0; j < nc; ++j) {
+                const bool gt = s_key[j] > k;
+                rank += gt;
+                above += gt ? s_w[j] : 0;
             }
-            s_key[r] = v;  // every s_key read happened before the barrier
-            s_w[r] = w;
+            in = above + w <= p.budget;
+            s_runs[rank] = k;
+            s_bsz[rank] = o1 - o0;
+            s_ofs[rank] = o0;
         }
-        __syncthreads();
-        const int ws = tid < nc ? s_w[tid] : 0;
-        int tot;
-        const int inc = block_exclusive_scan(ws, s_warp, &tot) + ws;
-        kstar = __syncthreads_count(tid < nc && inc <= p.budget);
-        sorted = s_key;
+        kstar = __syncthreads_count(in);
+        if (kstar == 0 && nc > 0) kstar = 1;  // the top community alone exceeds the budget: take it
+        sorted = s_runs;
     } else {
-        // rare: more candidates than one register sort holds; sort them in
+        // rare: more candidates than shared memory holds; sort them in
         // global scratch (block-wide bitonic, barriers between stages)
         unsigned long long* gk = p.gkey + (size_t)u * p.npow_max;
         int* gw = p.gw + (size_t)u * p.npow_max;
@@ -305,22 +316,21 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         atomicAdd(&s_cnt, mine);
         __syncthreads();
         kstar = s_cnt;
+        if (kstar == 0 && nc > 0) kstar = 1;  // the top community alone exceeds the budget: take it
         sorted = gk;
+        __syncthreads();
+        for (int i = tid; i < kstar; i += nt) {  // gw's weights are no longer needed
+            const int c = key_id(gk[i]);
+            bsz[i] = of[c + 1] - of[c];
+        }
     }
-    if (kstar == 0 && nc > 0) kstar = 1;  // the top community alone exceeds the budget: take it
 
-    // 3. ranked ids, membership mask, build-time run sizes in rank order
+    // 4. ranked ids and membership mask; inclusive prefix of the run sizes
     int32_t* selc = p.sel_comm + (size_t)u * p.Cmax;
-    const int32_t* of = p.offs + (size_t)u * (p.Cmax + 1);
-    const bool small = kstar <= SEL_FAST;
-    int* bsz = small ? s_bsz : p.gw + (size_t)u * p.npow_max;
     for (int i = tid; i < kstar; i += nt) {
         const int c = key_id(sorted[i]);
         selc[i] = c;
         atomicOr(&s_mask[c >> 5], 1u << (c & 31));
-        const int o0 = of[c];
-        bsz[i] = of[c + 1] - o0;
-        if (small) s_ofs[i] = o0;
     }
     __syncthreads();
     const int nb = block_scan_inplace(bsz, kstar, s_warp);  // inclusive
@@ -336,22 +346,27 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         // one token per thread per round: its run is found by binary search in
         // the inclusive run prefix; a round's loads are issued before its stores
         for (int t0 = tid; t0 < nb; t0 += RND * nt) {
-            int val[RND];
+            int src[RND];
 #pragma unroll
             for (int r = 0; r < RND; ++r) {
                 const int t = t0 + r * nt;
-                val[r] = 0;
+                src[r] = 0;
                 if (t < nb) {
-                    int lo = 0, hi = kstar - 1;  // first k with bsz[k] > t
-                    while (lo < hi) {
-                        const int mid = (lo + hi) >> 1;
-                        if (bsz[mid] > t) hi = mid;
-                        else lo = mid + 1;
-                    }
-                    const int start = lo ? bsz[lo - 1] : 0;
-                    val[r] = tk[s_ofs[lo] + (t - start)];
+                    // first k with s_bsz[k] > t, i.e. the number of inclusive
+                    // run ends <= t: branch-free binary lifting over shared
+                    // memory, so the rounds' searches interleave
+                    int lo = 0;
+#pragma unroll
+                    for (int step = SEL_FAST / 2; step > 0; step >>= 1)
+                        if (lo + step <= kstar && s_bsz[lo + step - 1] <= t) lo += step;
+                    const int start = lo ? s_bsz[lo - 1] : 0;
+                    src[r] = s_ofs[lo] + (t - start);
                 }
             }
+            // all of the round's loads in flight together (src 0 is in range)
+            int val[RND];
+#pragma unroll
+            for (int r = 0; r < RND; ++r) val[r] = tk[src[r]];
 #pragma unroll
             for (int r = 0; r < RND; ++r) {
                 const int t = t0 + r * nt;
@@ -407,14 +422,14 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
 
 template <typename T, int D, int GQ>
 __global__ void __launch_bounds__(SEL_THREADS) score_kernel(SelectParams p) {
+    pdl_wait();  // q may come from the kernel before
     const int u = blockIdx.y;
     const int C = min(p.num_comm[u], p.Cmax);
     score_rows<T, D, GQ>(p, u, C);
 }
 
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
-    // wait until every score and histogram update of the scoring kernel is visible
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();  // every score and histogram update of the scoring kernel is visible
     const int u = blockIdx.x;
     const int C = min(p.num_comm[u], p.Cmax);
     select_unit(p, u, C);
@@ -451,16 +466,9 @@ cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
     score_kernel<T, D, GQ><<<grid, SEL_THREADS, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.U);
-    cfg.blockDim = dim3(SEL_THREADS);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, select_kernel, p);
+    // (the scoring kernel follows the histogram memset, so it is launched
+    // plainly; the selection overlaps the scoring kernel's tail)
+    return launch_pdl(select_kernel, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
 }
 }  // namespace
 

@@ -49,8 +49,7 @@ __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParam
     __shared__ int s_cand[CKV_NEIGHBOURS];
     __shared__ float s_score[CKV_NEIGHBOURS];
     __shared__ int s_best, s_n, s_tl;
-    // everything this kernel reads may come from the kernel before it
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();  // everything this kernel reads may come from the kernel before it
     const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = u / p.G, g = u - b * p.G;
     const int gq = p.Hq / p.Hkv;
@@ -191,24 +190,13 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
     p.dev_err = g.dev_err;
     p.assigned = assigned;
     if (p.U <= 0) return cudaSuccess;
-    // programmatic dependent launch: the block launch overlaps the previous
-    // kernel's tail; the kernel waits for it before its first load
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.U);
-    cfg.blockDim = dim3(CKV_NEIGHBOURS * 32);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    const dim3 grid(p.U), block(CKV_NEIGHBOURS * 32);
     if (c.dtype == CKV_DTYPE_BF16) {
-        if (c.d == 128) return cudaLaunchKernelEx(&cfg, assign_kernel<__nv_bfloat16, 128>, p);
-        return cudaLaunchKernelEx(&cfg, assign_kernel<__nv_bfloat16, 64>, p);
+        if (c.d == 128) return launch_pdl(assign_kernel<__nv_bfloat16, 128>, grid, block, 0, st, p);
+        return launch_pdl(assign_kernel<__nv_bfloat16, 64>, grid, block, 0, st, p);
     }
-    if (c.d == 128) return cudaLaunchKernelEx(&cfg, assign_kernel<float, 128>, p);
-    return cudaLaunchKernelEx(&cfg, assign_kernel<float, 64>, p);
+    if (c.d == 128) return launch_pdl(assign_kernel<float, 128>, grid, block, 0, st, p);
+    return launch_pdl(assign_kernel<float, 64>, grid, block, 0, st, p);
 }
 
 }  // namespace ckv

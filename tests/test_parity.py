@@ -224,3 +224,17 @@ def test_append_assign_matches_external_append():
         assert torch.equal(a.st.K, b.st.K) and torch.equal(a.st.V, b.st.V)
         for name in ("comm_of", "cnt", "cent", "tail_tok", "tail_comm", "tail_len", "dev_err"):
             assert torch.equal(getattr(a.st.graph, name), getattr(b.st.graph, name)), name
+
+
+@pytest.mark.parametrize("budget_frac", [1.0, 0.5])
+def test_many_candidates_global_sort(budget_frac):
+    """More than 256 communities at or above the crossing bin: the selection
+    takes its global-memory sort path (every community, or about half)."""
+    T = 60000
+    wl = small(f"many_cand_{budget_frac}", 39, B=1, Hq=4, Hkv=1, T=T, budgets=(int(T * budget_frac),),
+               steps=2, update=True)
+    case = Case(wl)
+    assert case.C > 600
+    for _ in range(wl.steps):
+        case.step(wl.budget)
+    assert int(case.st.sel.n_sel.max().item()) > 256
