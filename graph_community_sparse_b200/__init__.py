@@ -202,8 +202,10 @@ def new_selection(cache: CacheDesc, graph: Graph, tok_cap: int, device="cuda") -
 
 
 def new_workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    # torch's caching allocator hands out 512-byte aligned blocks
-    return torch.empty((max(int(nbytes), 256),), dtype=torch.uint8, device=device)
+    """Zeroed (the library needs its first 256 bytes zero before first use
+    and leaves them zero); torch's caching allocator hands out 512-byte
+    aligned blocks."""
+    return torch.zeros((max(int(nbytes), 256),), dtype=torch.uint8, device=device)
 
 
 # ----------------------------------------------------------------------------

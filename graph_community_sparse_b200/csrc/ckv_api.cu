@@ -194,7 +194,7 @@ ckv_status ckv_workspace_size(const ckv_cache_desc* cache, const ckv_graph_desc*
         need = need > b ? need : b;
         need = need > c ? need : c;
     }
-    *bytes = need;
+    *bytes = ckv::ws_head_bytes(cache->B, cache->Hq) + need;
     return ok();
 }
 
@@ -208,9 +208,11 @@ ckv_status ckv_build_centroids(const ckv_cache_desc* cache, const int32_t* label
     if (T > cache->T_cap) return fail(CKV_ERR_CAPACITY, "T = %d > T_cap = %d", T, cache->T_cap);
     if (labels_stride < T) return fail(CKV_ERR_INVALID_ARG, "labels_stride < T");
     const int U = cache->B * graphs_per_seq(cache, graph);
-    CKV_TRY(check_ws(ws, ws_bytes, ckv::build_ws_bytes(U, graph->Cmax, graph->T_cap)));
+    const size_t head = ckv::ws_head_bytes(cache->B, cache->Hq);
+    CKV_TRY(check_ws(ws, ws_bytes, head + ckv::build_ws_bytes(U, graph->Cmax, graph->T_cap)));
     return cuda_status(ckv::launch_build(cache_view(cache), graph_view(cache, graph), labels, labels_stride, T,
-                                         ws, reinterpret_cast<cudaStream_t>(stream)),
+                                         static_cast<char*>(ws) + head,
+                                         reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_build_centroids");
 }
 
@@ -224,7 +226,8 @@ ckv_status ckv_score_select(const ckv_cache_desc* cache, const ckv_graph_desc* g
     if (!q) return fail(CKV_ERR_INVALID_ARG, "q is NULL");
     if (!aligned16(q)) return fail(CKV_ERR_MISALIGNED, "q must be 16-byte aligned");
     if (budget < 0) return fail(CKV_ERR_INVALID_ARG, "budget < 0");
-    CKV_TRY(check_ws(ws, ws_bytes, ckv::select_ws_bytes((int)U, graph->Cmax)));
+    CKV_TRY(check_ws(ws, ws_bytes,
+                     ckv::ws_head_bytes(cache->B, cache->Hq) + ckv::select_ws_bytes((int)U, graph->Cmax)));
     return cuda_status(ckv::launch_score_select(cache_view(cache), graph_view(cache, graph), q, budget,
                                                 sel_view(sel), ws, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_score_select");
@@ -240,7 +243,8 @@ ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q, const c
     if (!q || !out) return fail(CKV_ERR_INVALID_ARG, "q or out is NULL");
     if (!aligned16(q) || !aligned16(out)) return fail(CKV_ERR_MISALIGNED, "q and out must be 16-byte aligned");
     const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : cache->Hq / cache->Hkv;
-    CKV_TRY(check_ws(ws, ws_bytes, ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap)));
+    CKV_TRY(check_ws(ws, ws_bytes,
+                     ckv::ws_head_bytes(cache->B, cache->Hq) + ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap)));
     return cuda_status(ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q,
                                                  out, nbr8, ws, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_sparse_decode");
@@ -259,7 +263,7 @@ ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const void* q,
     if (!q || !out) return fail(CKV_ERR_INVALID_ARG, "q or out is NULL");
     if (!aligned16(q) || !aligned16(out)) return fail(CKV_ERR_MISALIGNED, "q and out must be 16-byte aligned");
     const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : cache->Hq / cache->Hkv;
-    const size_t need = ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap);
+    const size_t need = ckv::ws_head_bytes(cache->B, cache->Hq) + ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap);
     if (need > CKV_NOALLOC_SCRATCH_BYTES)
         return fail(CKV_ERR_UNSUPPORTED,
                     "ckv_sparse_decode_noalloc: these shapes need %zu bytes of scratch, above the library's "
@@ -308,7 +312,8 @@ ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t 
     if (T < 1 || T > cache->T_cap) return fail(CKV_ERR_CAPACITY, "T = %d outside [1, T_cap]", T);
     const int64_t U = (int64_t)cache->B * cache->Hkv;
     if (U * T > (int64_t)1 << 30) return fail(CKV_ERR_UNSUPPORTED, "B*Hkv*T above 2^30");
-    CKV_TRY(check_ws(ws, ws_bytes, ckv::decode_ws_bytes((int)U, cache->Hq / cache->Hkv, cache->d, 0)));
+    CKV_TRY(check_ws(ws, ws_bytes,
+                     ckv::ws_head_bytes(cache->B, cache->Hq) + ckv::decode_ws_bytes((int)U, cache->Hq / cache->Hkv, cache->d, 0)));
     return cuda_status(ckv::launch_dense_decode(cache_view(cache), q, T, out, ws,
                                                 reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_dense_decode");

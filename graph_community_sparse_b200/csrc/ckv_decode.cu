@@ -38,6 +38,31 @@
 namespace ckv {
 
 constexpr int DEC_WARPS = 4;
+// Work split of the attention kernel: the first 7/8 of the concatenated token
+// lists are cut into one equal slice per warp; the last 1/8 is handed out in
+// chunks of at least DYN_CHUNK_MIN tokens (at most NCH_MAX chunks) from an
+// atomic ticket, so warps on SMs that run faster (the SMs of a GPC share its
+// memory bandwidth unevenly) take more of it and all warps end together.
+constexpr int DYN_DEN = 8;
+constexpr int DYN_CHUNK_MIN = 64;
+constexpr int NCH_MAX = 4096;
+
+struct DynSplit {
+    int R;      // tokens of the static part, [0, R)
+    int per_s;  // static tokens per warp
+    int chk;    // dynamic chunk length
+    int nch;    // dynamic chunks
+};
+
+__host__ __device__ __forceinline__ DynSplit dyn_split(int total, int W) {
+    DynSplit d;
+    const int dyn = total / DYN_DEN;
+    d.chk = max(DYN_CHUNK_MIN, (dyn + NCH_MAX - 1) / NCH_MAX);
+    d.nch = (dyn + d.chk - 1) / d.chk;
+    d.R = total - dyn;
+    d.per_s = max(1, (d.R + W - 1) / W);
+    return d;
+}
 constexpr int TOK_PER_IT = 8;
 constexpr float RESCALE_THRESH = 8.0f;
 
@@ -347,30 +372,44 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(
         total = p.U * p.T;
     }
     if (total <= 0) return;
-    const int per = (total + p.W - 1) / p.W;
-    const int start = w * per;
-    if (start >= total) return;
-    const int end = min(start + per, total);
+    const DynSplit sp = dyn_split(total, p.W);
 
-    int u;
-    if constexpr (DENSE) {
-        u = start / p.T;
-    } else {
-        int a = 0, c = p.U;  // s_pre[a] <= start < s_pre[c]
-        while (c - a > 1) {
-            const int mid = (a + c) >> 1;
-            if (s_pre[mid] <= start) a = mid;
-            else c = mid;
+    // tokens [start, end) of the concatenated lists; partial of unit u in
+    // slot sbase + u
+    auto run_range = [&](int start, int end, int sbase) {
+        int u;
+        if constexpr (DENSE) {
+            u = start / p.T;
+        } else {
+            int a = 0, c = p.U;  // s_pre[a] <= start < s_pre[c]
+            while (c - a > 1) {
+                const int mid = (a + c) >> 1;
+                if (s_pre[mid] <= start) a = mid;
+                else c = mid;
+            }
+            u = a;
         }
-        u = a;
-    }
+        while (true) {
+            const int ubeg = DENSE ? u * p.T : s_pre[u];
+            const int uend = DENSE ? ubeg + p.T : s_pre[u + 1];
+            const int lo = max(start, ubeg), hi = min(end, uend);
+            if (lo < hi) process_segment<T, D, GQ, DENSE>(p, u, lo - ubeg, hi - ubeg, sbase + u, wsm, lane);
+            if (end <= uend || u + 1 >= p.U) break;
+            ++u;
+        }
+    };
+
+    // static slice: slots [0, W + U)
+    const int start = w * sp.per_s;
+    if (start < sp.R) run_range(start, min(start + sp.per_s, sp.R), w);
+    // dynamic chunks: slots [W + U, W + 2U + nch)
     while (true) {
-        const int ubeg = DENSE ? u * p.T : s_pre[u];
-        const int uend = DENSE ? ubeg + p.T : s_pre[u + 1];
-        const int lo = max(start, ubeg), hi = min(end, uend);
-        if (lo < hi) process_segment<T, D, GQ, DENSE>(p, u, lo - ubeg, hi - ubeg, w + u, wsm, lane);
-        if (end <= uend || u + 1 >= p.U) break;
-        ++u;
+        int c = 0;
+        if (lane == 0) c = atomicAdd(p.ws.ticket, 1);
+        c = __shfl_sync(FULL, c, 0);
+        if (c >= sp.nch) break;
+        const int c0 = sp.R + c * sp.chk;
+        run_range(c0, min(c0 + sp.chk, total), p.W + p.U + c);
     }
 }
 
@@ -427,6 +466,8 @@ template <int D, int GQ, bool DENSE>
 __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_merge(DecodeParams p) {
     pdl_wait();  // the attention kernel's partials are complete and visible
     const int u = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    // no kernel of this call takes a ticket any more: return it to zero
+    if (u == 0 && t == 0) *p.ws.ticket = 0;
     int b, kvh, h0;
     unit_heads(p, u, GQ, DENSE, b, kvh, h0);
     int ubeg, uend, total;
@@ -445,9 +486,21 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
         if (!DENSE && p.want_nbr && t < 8) p.nbr8[(size_t)u * 8 + t] = -1;
         return;
     }
-    const int per = (total + p.W - 1) / p.W;
-    const int wf = ubeg / per, nslots = (uend - 1) / per - wf + 1;
-    const size_t s0 = (size_t)wf + u;
+    // the unit's partials: static slices [sA, sA + nA), then dynamic chunks
+    // [sB, sB + nB) (the attention kernel's split, recomputed)
+    const DynSplit sp = dyn_split(total, p.W);
+    int nA = 0, nB = 0;
+    size_t sA = 0, sB = 0;
+    if (ubeg < sp.R) {
+        const int f = ubeg / sp.per_s, l = (min(uend, sp.R) - 1) / sp.per_s;
+        sA = (size_t)f + u;
+        nA = l - f + 1;
+    }
+    if (uend > sp.R) {
+        const int f = (max(ubeg, sp.R) - sp.R) / sp.chk, l = (uend - 1 - sp.R) / sp.chk;
+        sB = (size_t)p.W + p.U + f + u;
+        nB = l - f + 1;
+    }
     const DecodeWs& ws = p.ws;
 
     if (!DENSE && p.want_nbr && warp >= D / 32) {
@@ -548,7 +601,10 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
         Ls[h] = 0.f;
         A[h] = 0.f;
     }
-    for (int c0 = 0; c0 < nslots; c0 += CH) {
+    for (int part = 0; part < 2; ++part) {
+      const size_t s0 = part ? sB : sA;
+      const int nslots = part ? nB : nA;
+      for (int c0 = 0; c0 < nslots; c0 += CH) {
         float xm[CH][GQ], xl[CH][GQ], xa[CH][GQ];
         // unconditional loads at constant offsets from one base (the slot
         // arrays carry MERGE_PAD spare slots, so a chunk never reads past
@@ -597,6 +653,7 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
             A[h] = fmaf(A[h], fo, a);
             M[h] = mn;
         }
+      }
     }
 #pragma unroll
     for (int h = 0; h < GQ; ++h) outu[h * D + t] = A[h] / Ls[h];
@@ -606,15 +663,22 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
 // host side
 // ---------------------------------------------------------------------------
 
+// Partial slots: W + U for the static slices, then NCH_MAX + U for the
+// dynamic chunks, then MERGE_PAD spares.
+static size_t decode_slots(int U) { return (size_t)MAX_DECODE_WARPS + NCH_MAX + 2 * (size_t)U + MERGE_PAD; }
+
 size_t decode_ws_bytes(int U, int gq, int d, int lam_cap) {
-    const size_t slots = (size_t)MAX_DECODE_WARPS + U + MERGE_PAD;
+    const size_t slots = decode_slots(U);
     return align256(slots * gq * 4) * 2 + align256(slots * gq * d * 4) + align256((size_t)U * lam_cap * 4);
 }
 
-DecodeWs carve_decode_ws(void* ws, int U, int gq, int d, int lam_cap) {
-    const size_t slots = (size_t)MAX_DECODE_WARPS + U + MERGE_PAD;
+// ws: the workspace base (its head holds the ticket); the parts follow the head
+DecodeWs carve_decode_ws(void* ws, size_t head, int U, int gq, int d, int lam_cap) {
+    const size_t slots = decode_slots(U);
     char* p = static_cast<char*>(ws);
     DecodeWs w;
+    w.ticket = reinterpret_cast<int*>(p);
+    p += head;
     w.m = reinterpret_cast<float*>(p);
     p += align256(slots * gq * 4);
     w.l = reinterpret_cast<float*>(p);
@@ -686,7 +750,7 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
     p.unit_prefix = s.unit_prefix;
     p.n_tok = s.n_tok;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
-    p.ws = carve_decode_ws(ws, p.U, g.gq, c.d, s.tok_cap);
+    p.ws = carve_decode_ws(ws, ws_head_bytes(c.B, c.Hq), p.U, g.gq, c.d, s.tok_cap);
     p.want_nbr = nbr8 != nullptr;
     p.out = out;
     p.nbr8 = nbr8;
@@ -710,7 +774,7 @@ cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float*
     p.T = T;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
     const int gq = c.Hq / c.Hkv;
-    p.ws = carve_decode_ws(ws, p.U, gq, c.d, 0);
+    p.ws = carve_decode_ws(ws, ws_head_bytes(c.B, c.Hq), p.U, gq, c.d, 0);
     p.out = out;
     return dispatch<true>(c, gq, p, st);
 }

@@ -207,7 +207,18 @@ struct SelView {
 };
 
 // workspace carving
+// Workspace head, shared by every call on a workspace and zero before its
+// first use: the attention kernels' work ticket (WS_RESERVED bytes), then one
+// score histogram of HIST_BINS counters per possible graph unit (B * Hq).
+// Every call leaves the head zero (the attention's merge returns the ticket,
+// the selection clears each histogram after reading it).  The other parts of
+// each call start after the head.
+constexpr size_t WS_RESERVED = 256;
+constexpr int HIST_BITS = 12;
+constexpr int HIST_BINS = 1 << HIST_BITS;
+
 struct DecodeWs {
+    int* ticket;   // dynamic chunk counter (the workspace's first bytes)
     float* m;      // [slots, GQ]
     float* l;      // [slots, GQ]
     float* acc;    // [slots, GQ, D]
@@ -220,7 +231,7 @@ size_t select_ws_bytes(int U, int Cmax);
 // lam_cap: selection entries per unit whose graph logits are kept (the
 // selection's tok_cap; 0 for the dense comparator)
 size_t decode_ws_bytes(int U, int gq, int d, int lam_cap);
-DecodeWs carve_decode_ws(void* ws, int U, int gq, int d, int lam_cap);
+DecodeWs carve_decode_ws(void* ws, size_t head, int U, int gq, int d, int lam_cap);
 
 cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* labels,
                          int64_t labels_stride, int T, void* ws, cudaStream_t st);
@@ -240,6 +251,7 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
                                  const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline size_t ws_head_bytes(int B, int Hq) { return WS_RESERVED + align256((size_t)B * Hq * HIST_BINS * 4); }
 
 // Programmatic dependent launch.  Kernels launched by launch_pdl() start
 // with pdl_wait(), so they read and write nothing before the previous kernel

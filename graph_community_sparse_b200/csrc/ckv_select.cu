@@ -24,7 +24,8 @@
 //    the unit's token list: sinks, build-time members of each selected
 //    community (from the community-contiguous CSR), then the selected tail
 //    members.
-// The histograms are zeroed by a memset issued in the same call.
+// The histograms live in the workspace head: zero on entry, and each
+// selection block clears its unit's histogram after reading it.
 #include <math.h>
 
 #include "ckv_internal.cuh"
@@ -34,8 +35,8 @@ namespace ckv {
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_THREADS = SEL_WARPS * 32;
 constexpr int SCORE_ROWS = SEL_WARPS * 8;  // centres per block
-constexpr int SEL_HBITS = 12;
-constexpr int SEL_HBINS = 1 << SEL_HBITS;
+constexpr int SEL_HBITS = HIST_BITS;
+constexpr int SEL_HBINS = HIST_BINS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates sorted in registers
 
 struct SelectParams {
@@ -183,9 +184,13 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     static_assert(per == 16, "four int4 histogram loads per thread");
     int4 hv[4];
     {
-        const int4* h4 = reinterpret_cast<const int4*>(hist + per * tid);
+        int4* h4 = reinterpret_cast<int4*>(const_cast<int32_t*>(hist) + per * tid);
 #pragma unroll
         for (int i = 0; i < 4; ++i) hv[i] = __ldcg(h4 + i);
+        // leave the histogram zero for the next call (each thread clears the
+        // bins it alone read)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h4[i] = make_int4(0, 0, 0, 0);
     }
     int wv[RND];
     float sv[RND];
@@ -346,22 +351,31 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         // one token per thread per round: its run is found by binary search in
         // the inclusive run prefix; a round's loads are issued before its stores
         for (int t0 = tid; t0 < nb; t0 += RND * nt) {
+            // the run of each of the round's tokens: first k with s_bsz[k] > t
+            // (the number of inclusive run ends <= t), by branch-free binary
+            // lifting done for all of the round's tokens in lockstep, so the
+            // RND searches' shared-memory loads overlap
+            int tt[RND], lo[RND];
+#pragma unroll
+            for (int r = 0; r < RND; ++r) {
+                tt[r] = min(t0 + r * nt, nb - 1);
+                lo[r] = 0;
+            }
+#pragma unroll
+            for (int step = SEL_FAST / 2; step > 0; step >>= 1) {
+#pragma unroll
+                for (int r = 0; r < RND; ++r) {
+                    const int probe = min(lo[r] + step, kstar) - 1;  // in range: kstar >= 1
+                    const bool fits = lo[r] + step <= kstar;
+                    const bool le = s_bsz[probe] <= tt[r];
+                    lo[r] += (fits & le) ? step : 0;
+                }
+            }
             int src[RND];
 #pragma unroll
             for (int r = 0; r < RND; ++r) {
-                const int t = t0 + r * nt;
-                src[r] = 0;
-                if (t < nb) {
-                    // first k with s_bsz[k] > t, i.e. the number of inclusive
-                    // run ends <= t: branch-free binary lifting over shared
-                    // memory, so the rounds' searches interleave
-                    int lo = 0;
-#pragma unroll
-                    for (int step = SEL_FAST / 2; step > 0; step >>= 1)
-                        if (lo + step <= kstar && s_bsz[lo + step - 1] <= t) lo += step;
-                    const int start = lo ? s_bsz[lo - 1] : 0;
-                    src[r] = s_ofs[lo] + (t - start);
-                }
+                const int start = lo[r] ? s_bsz[lo[r] - 1] : 0;
+                src[r] = s_ofs[lo[r]] + (tt[r] - start);
             }
             // all of the round's loads in flight together (src 0 is in range)
             int val[RND];
@@ -447,14 +461,13 @@ static int next_pow2(int x) {
 
 namespace {
 struct SelWs {
-    size_t scores, hist, gkey, gw, total;
+    size_t scores, gkey, gw, total;
 };
 SelWs sel_ws_layout(int U, int Cmax) {
     SelWs l;
     const size_t np = (size_t)next_pow2(Cmax);
     l.scores = 0;
-    l.hist = l.scores + align256((size_t)U * Cmax * 4);
-    l.gkey = l.hist + align256((size_t)U * SEL_HBINS * 4);
+    l.gkey = l.scores + align256((size_t)U * Cmax * 4);
     l.gw = l.gkey + align256((size_t)U * np * 8);
     l.total = l.gw + align256((size_t)U * np * 4);
     return l;
@@ -463,11 +476,8 @@ SelWs sel_ws_layout(int U, int Cmax) {
 template <typename T, int D, int GQ>
 cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
     dim3 grid((p.Cmax + SCORE_ROWS - 1) / SCORE_ROWS, p.U);
-    score_kernel<T, D, GQ><<<grid, SEL_THREADS, 0, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(score_kernel<T, D, GQ>, grid, dim3(SEL_THREADS), 0, st, p);
     if (e != cudaSuccess) return e;
-    // (the scoring kernel follows the histogram memset, so it is launched
-    // plainly; the selection overlaps the scoring kernel's tail)
     return launch_pdl(select_kernel, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
 }
 }  // namespace
@@ -478,12 +488,12 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
                                 const SelView& s, void* ws, cudaStream_t st) {
     const int U = c.B * g.G;
     const SelWs l = sel_ws_layout(U, g.Cmax);
-    char* w = static_cast<char*>(ws);
+    char* w = static_cast<char*>(ws) + ws_head_bytes(c.B, c.Hq);
     SelectParams p{};
     p.q = q;
     p.cent = g.cent;
     p.scores = reinterpret_cast<float*>(w + l.scores);
-    p.hist = reinterpret_cast<int32_t*>(w + l.hist);
+    p.hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + WS_RESERVED);  // zero on entry
     p.gkey = reinterpret_cast<unsigned long long*>(w + l.gkey);
     p.gw = reinterpret_cast<int32_t*>(w + l.gw);
     p.cnt = g.cnt;
@@ -511,9 +521,6 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     p.max_tail = g.max_tail;
     p.tok_cap = s.tok_cap;
     p.budget = budget;
-    // the per-unit histograms start at zero
-    cudaError_t e = cudaMemsetAsync(p.hist, 0, l.gkey - l.hist, st);
-    if (e != cudaSuccess) return e;
 
 #define CKV_SC_CASE(TT, DD, GG) \
     if (c.d == DD && g.gq == GG) return launch_t<TT, DD, GG>(p, st);

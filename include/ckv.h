@@ -30,6 +30,11 @@
  *  - No call allocates device memory.  Scratch comes from the caller's
  *    workspace `ws` of `ws_bytes` bytes (256-byte aligned), sized by
  *    ckv_workspace_size(); a smaller workspace returns CKV_ERR_WORKSPACE.
+ *    Its head (256 + 16384 * B * Hq bytes: the attention kernels' work
+ *    counter and the selection's score histograms) must be zero before the
+ *    workspace's first use, e.g. zero-fill the whole workspace once after
+ *    allocating it; every call leaves the head zero.  The rest needs no
+ *    initialisation.  Calls sharing a workspace must not overlap on the GPU.
  *  - Host-side checks happen before any launch and return a status without
  *    touching the device; ckv_last_error() then names the failed check.
  *    Data-dependent faults detected on the device (a label out of range, a
@@ -215,17 +220,19 @@ CKV_API ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q,
  * until the process exits.
  *   - Calls needing more scratch than CKV_NOALLOC_SCRATCH_BYTES return
  *     CKV_ERR_UNSUPPORTED before touching the device.  The need is the size
- *     ckv_workspace_size's attention part reports for these shapes: about
- *     4 * (8192 + U) * gq * (d + 2) bytes of split-K partials (gq query
- *     heads per graph, U = B * graphs per sequence) plus 4 * U * sel->tok_cap
- *     bytes of neighbour logits.  Per-head graphs with d = 128 need about
- *     4.3 MiB + the logits; Hq/Hkv = 8 with d = 128 in per-group mode needs
- *     over 32 MiB and is refused.
+ *     ckv_workspace_size reports for the attention alone: the head
+ *     (256 + 16384 * B * Hq bytes), about 4 * (12288 + 2U) * gq * (d + 2)
+ *     bytes of split-K partials (gq query heads per graph, U = B * graphs per
+ *     sequence) and 4 * U * sel->tok_cap bytes of neighbour logits.  Per-head
+ *     graphs with d = 128 need about 6.4 MiB + the head + the logits;
+ *     Hq/Hkv = 8 with d = 128 in per-group mode needs over 32 MiB and is
+ *     refused.
  *   - The first call on each device looks up the array's device address
  *     (with that device current); make that first call before any stream
  *     capture.  No call allocates or frees memory.
  *   - All calls share the one array and it keeps the previous call's
- *     contents (nothing in it needs to start at zero).  Calls that overlap
+ *     contents (it starts at zero when the library loads; calls leave its
+ *     work counter at zero).  Calls that overlap
  *     on the GPU, e.g. on two streams at once, race on it and give wrong
  *     results: serialise them.
  */
