@@ -21,6 +21,7 @@ __all__ = [
     "Graph", "Selection", "cache_desc", "new_graph", "new_selection", "new_workspace",
     "ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
     "ckv_sparse_decode_noalloc", "NOALLOC_SCRATCH_BYTES", "ckv_assign_update", "ckv_append_assign",
+    "ckv_sparse_decode_append",
     "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP",
@@ -36,7 +37,8 @@ PER_GROUP, PER_HEAD = 0, 1
 DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
 NEIGHBOURS = 8
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_dense_decode",
+            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
+            "ckv_dense_decode",
             "ckv_status_string", "ckv_last_error", "ckv_abi_version")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -80,9 +82,12 @@ lib.ckv_sparse_decode.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(Selection
 lib.ckv_sparse_decode_noalloc.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p]
 lib.ckv_assign_update.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p]
 lib.ckv_append_assign.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p, _p, _p]
+lib.ckv_sparse_decode_append.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _i32, _p,
+                                         _p, _p, _p, _sz, _p]
 lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
 for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-           "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_dense_decode"):
+           "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
+           "ckv_dense_decode"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.ckv_status_string.argtypes = [ctypes.c_int]
 lib.ckv_status_string.restype = ctypes.c_char_p
@@ -262,14 +267,31 @@ def ckv_assign_update(cache: CacheDesc, graph: Graph, pos: int, nbr8: torch.Tens
            "ckv_assign_update")
 
 
+def _check_rows(cache: CacheDesc, **rows) -> None:
+    shape = (cache.B, cache.Hkv, cache.d)
+    for name, t in rows.items():
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {shape} tensor, got {tuple(t.shape)}")
+
+
+def ckv_sparse_decode_append(cache: CacheDesc, q: torch.Tensor, graph: Graph, sel: Selection, out: torch.Tensor,
+                             nbr8: Optional[torch.Tensor], pos: int, k_new: torch.Tensor, v_new: torch.Tensor,
+                             assigned: Optional[torch.Tensor], ws: torch.Tensor, stream=None) -> None:
+    """ckv_sparse_decode + ckv_append_assign in one call (the update runs in
+    the attention's merge kernel)."""
+    _check_rows(cache, k_new=k_new, v_new=v_new)
+    _check(lib.ckv_sparse_decode_append(ctypes.byref(cache), q.data_ptr(), ctypes.byref(graph.desc),
+                                        ctypes.byref(sel.desc), out.data_ptr(), _ptr(nbr8), pos, k_new.data_ptr(),
+                                        v_new.data_ptr(), _ptr(assigned), ws.data_ptr(), ws.numel(),
+                                        _stream(stream)),
+           "ckv_sparse_decode_append")
+
+
 def ckv_append_assign(cache: CacheDesc, graph: Graph, pos: int, k_new: torch.Tensor, v_new: torch.Tensor,
                       nbr8: torch.Tensor, assigned: Optional[torch.Tensor], stream=None) -> None:
     """k_new, v_new: [B, Hkv, d] contiguous in the cache dtype; written to
     row ``pos`` of K and V by the library, then the update runs."""
-    shape = (cache.B, cache.Hkv, cache.d)
-    for name, t in (("k_new", k_new), ("v_new", v_new)):
-        if tuple(t.shape) != shape or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous {shape} tensor, got {tuple(t.shape)}")
+    _check_rows(cache, k_new=k_new, v_new=v_new)
     _check(lib.ckv_append_assign(ctypes.byref(cache), ctypes.byref(graph.desc), pos, k_new.data_ptr(),
                                  v_new.data_ptr(), nbr8.data_ptr(), _ptr(assigned), _stream(stream)),
            "ckv_append_assign")

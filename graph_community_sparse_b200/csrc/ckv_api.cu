@@ -6,6 +6,7 @@
 
 #include <string>
 
+#include "ckv_assign.cuh"
 #include "ckv_internal.cuh"
 
 namespace {
@@ -246,7 +247,7 @@ ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q, const c
     CKV_TRY(check_ws(ws, ws_bytes,
                      ckv::ws_head_bytes(cache->B, cache->Hq) + ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap)));
     return cuda_status(ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q,
-                                                 out, nbr8, ws, reinterpret_cast<cudaStream_t>(stream)),
+                                                 out, nbr8, ws, nullptr, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_sparse_decode");
 }
 
@@ -274,7 +275,7 @@ ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const void* q,
     cudaError_t e = ckv::static_decode_scratch(&scratch, &have);
     if (e != cudaSuccess) return cuda_status(e, "ckv_sparse_decode_noalloc: scratch address lookup");
     return cuda_status(ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q,
-                                                 out, nbr8, scratch, reinterpret_cast<cudaStream_t>(stream)),
+                                                 out, nbr8, scratch, nullptr, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_sparse_decode_noalloc");
 }
 
@@ -302,6 +303,31 @@ ckv_status ckv_append_assign(const ckv_cache_desc* cache, const ckv_graph_desc* 
     return cuda_status(ckv::launch_assign_update(cache_view(cache), graph_view(cache, graph), pos, k_new, v_new,
                                                  nbr8, assigned, reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_append_assign");
+}
+
+ckv_status ckv_sparse_decode_append(const ckv_cache_desc* cache, const void* q, const ckv_graph_desc* graph,
+                                    const ckv_selection_desc* sel, float* out, int32_t* nbr8, int32_t pos,
+                                    const void* k_new, const void* v_new, int32_t* assigned, void* ws,
+                                    size_t ws_bytes, ckv_stream_t stream) {
+    CKV_TRY(check_cache(cache, true));
+    CKV_TRY(check_graph(cache, graph));
+    const int64_t U = (int64_t)cache->B * graphs_per_seq(cache, graph);
+    CKV_TRY(check_sel(graph, sel, U));
+    if (!q || !out) return fail(CKV_ERR_INVALID_ARG, "q or out is NULL");
+    if (!aligned16(q) || !aligned16(out)) return fail(CKV_ERR_MISALIGNED, "q and out must be 16-byte aligned");
+    if (!k_new || !v_new) return fail(CKV_ERR_INVALID_ARG, "k_new or v_new is NULL");
+    if (!aligned16(k_new) || !aligned16(v_new))
+        return fail(CKV_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
+    if (pos < 0 || pos >= cache->T_cap) return fail(CKV_ERR_CAPACITY, "pos = %d outside [0, T_cap)", pos);
+    const int gq = graph->mode == CKV_GRAPH_PER_HEAD ? 1 : cache->Hq / cache->Hkv;
+    CKV_TRY(check_ws(ws, ws_bytes,
+                     ckv::ws_head_bytes(cache->B, cache->Hq) + ckv::decode_ws_bytes((int)U, gq, cache->d, sel->tok_cap)));
+    const ckv::CacheView cv = cache_view(cache);
+    const ckv::GraphView gv = graph_view(cache, graph);
+    const ckv::AssignParams ap = ckv::make_assign_params(cv, gv, pos, k_new, v_new, nullptr, assigned);
+    return cuda_status(ckv::launch_sparse_decode(cv, gv, sel_view(sel), q, out, nbr8, ws, &ap,
+                                                 reinterpret_cast<cudaStream_t>(stream)),
+                       "ckv_sparse_decode_append");
 }
 
 ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t T, float* out, void* ws,

@@ -33,6 +33,7 @@
 #include <math.h>
 #include <type_traits>
 
+#include "ckv_assign.cuh"
 #include "ckv_internal.cuh"
 
 namespace ckv {
@@ -102,7 +103,10 @@ struct DecodeParams {
     int W;                  // warps in the grid
     int want_nbr;
     float* out;
-    int32_t* nbr8;
+    int32_t* nbr8;          // may be NULL when only the fused update needs them
+    int append;             // fused community update (and K/V append) in the merge
+    int key_bf16;           // dtype of the new key rows
+    AssignParams ap;
 };
 
 __device__ __forceinline__ void unit_heads(const DecodeParams& p, int u, int gq, bool dense,
@@ -457,6 +461,15 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x)
     return x;
 }
 
+// The fused community update of unit u by the merge block's NBR_WARPS
+// neighbour warps (thread xt of 32 NBR_WARPS), given its neighbour positions.
+template <int D>
+__device__ __forceinline__ void merge_assign(const DecodeParams& p, int u, const int* nbpos, int xt) {
+    auto sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory"); };
+    if (p.key_bf16) assign_unit<__nv_bfloat16, D, NBR_WARPS>(p.ap, u, nbpos, xt, sync);
+    else assign_unit<float, D, NBR_WARPS>(p.ap, u, nbpos, xt, sync);
+}
+
 // One block per unit: threads 0..D-1 own one output dimension each (all the
 // unit's heads); the NBR_WARPS extra warps search the top-8 neighbours.  Slots are
 // combined in slot order, a chunk of slots at a time, by a per-thread online
@@ -483,7 +496,12 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
     float* outu = p.out + ((size_t)b * p.Hq + h0) * D;
     if (uend <= ubeg) {
         for (int i = t; i < GQ * D; i += blockDim.x) outu[i] = 0.f;
-        if (!DENSE && p.want_nbr && t < 8) p.nbr8[(size_t)u * 8 + t] = -1;
+        if (!DENSE && p.want_nbr && p.nbr8 && t < 8) p.nbr8[(size_t)u * 8 + t] = -1;
+        if (!DENSE && p.append && warp >= D / 32) {
+            __shared__ int s_none[CKV_NEIGHBOURS];
+            if (t - D < CKV_NEIGHBOURS) s_none[t - D] = -1;
+            merge_assign<D>(p, u, s_none, t - D);  // no neighbour: the token joins nothing
+        }
         return;
     }
     // the unit's partials: static slices [sA, sA + nA), then dynamic chunks
@@ -556,12 +574,17 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
         for (int k = 0; k < NBR_KEEP; ++k) offer(kk[k]);
         for (int i = p.S + xt + NBR_KEEP * NBR_THREADS; i < n; i += NBR_THREADS) offer(key_at(i));
         asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory");
+        __shared__ int s_nbpos[CKV_NEIGHBOURS];
         if (xw == 0) {
             const int cnt = s_cnt;
-            int32_t* outn = p.nbr8 + (size_t)u * 8;
+            int32_t* outn = p.nbr8 ? p.nbr8 + (size_t)u * 8 : nullptr;
             if (cnt <= 32) {
                 const unsigned long long x = warp_sort_desc(lane < cnt ? s_cand[lane] : 0ull, lane);
-                if (lane < 8) outn[lane] = x ? nbr_pos(x) : -1;
+                if (lane < 8) {
+                    const int np = x ? nbr_pos(x) : -1;
+                    s_nbpos[lane] = np;
+                    if (outn) outn[lane] = np;
+                }
             } else {
                 // many candidates (ties in the logits): 8 rounds, each taking
                 // the best key below the previous winner, from the shared
@@ -581,10 +604,18 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
                         }
                     }
                     best = warp_max_u64(best);
-                    if (lane == 0) outn[r] = best ? nbr_pos(best) : -1;
+                    if (lane == 0) {
+                        const int np = best ? nbr_pos(best) : -1;
+                        s_nbpos[r] = np;
+                        if (outn) outn[r] = np;
+                    }
                     prev = best;  // 0 once the entries run out: every later round finds none
                 }
             }
+        }
+        if (p.append) {
+            asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory");  // s_nbpos complete
+            merge_assign<D>(p, u, s_nbpos, xt);
         }
         return;
     }
@@ -731,7 +762,8 @@ cudaError_t dispatch(const CacheView& c, int gq, DecodeParams p, cudaStream_t st
 }  // namespace
 
 cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const SelView& s,
-                                 const void* q, float* out, int32_t* nbr8, void* ws, cudaStream_t st) {
+                                 const void* q, float* out, int32_t* nbr8, void* ws, const AssignParams* ap,
+                                 cudaStream_t st) {
     DecodeParams p{};
     p.k = c.k;
     p.v = c.v;
@@ -751,9 +783,14 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
     p.n_tok = s.n_tok;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);
     p.ws = carve_decode_ws(ws, ws_head_bytes(c.B, c.Hq), p.U, g.gq, c.d, s.tok_cap);
-    p.want_nbr = nbr8 != nullptr;
+    p.want_nbr = nbr8 != nullptr || ap != nullptr;
     p.out = out;
     p.nbr8 = nbr8;
+    if (ap) {
+        p.append = 1;
+        p.key_bf16 = c.dtype == CKV_DTYPE_BF16;
+        p.ap = *ap;
+    }
     return dispatch<false>(c, g.gq, p, st);
 }
 

@@ -237,8 +237,13 @@ cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* 
                          int64_t labels_stride, int T, void* ws, cudaStream_t st);
 cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const void* q, int budget,
                                 const SelView& s, void* ws, cudaStream_t st);
+struct AssignParams;
+// ap non-NULL: the merge kernel also runs the community update (and the
+// K/V append when ap carries the new rows) for every unit, after finding
+// its neighbours.
 cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const SelView& s,
-                                 const void* q, float* out, int32_t* nbr8, void* ws, cudaStream_t st);
+                                 const void* q, float* out, int32_t* nbr8, void* ws, const AssignParams* ap,
+                                 cudaStream_t st);
 cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float* out, void* ws,
                                 cudaStream_t st);
 // Device address and size of the library's own decode scratch (looked up once

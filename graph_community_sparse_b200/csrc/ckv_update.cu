@@ -1,194 +1,27 @@
-// Local community update for a newly generated token, sm_100a.
-//
-// A new token never triggers a global re-partition: it is attached to one of
-// the neighbouring communities and only that community's centre changes, at a
-// cost set by the head dimension rather than the context length (CommunityKV,
-// rit.work summary, section "A graph of tokens replaces re-clustering",
-// paragraph 6; the abstract describes the rule as constant-time).
-//
-// The candidate communities are those of the 8 neighbour positions found by
-// the attention kernel; each distinct candidate costs one d-long dot product
-// with the new key; the winner's centre moves by (k - c)/(n + 1) and its
-// count grows by one.  O(8 d) work per graph.
+// Local community update for a newly generated token, sm_100a: the
+// stand-alone kernel (ckv_assign_update, ckv_append_assign).  The update of
+// one graph unit, and where it comes from in the pages, is in ckv_assign.cuh;
+// the attention's merge kernel runs the same code when the step is fused.
 #include <math.h>
 
-#include "ckv_internal.cuh"
+#include "ckv_assign.cuh"
 
 namespace ckv {
 
-struct AssignParams {
-    const void* k;      // new key rows: the cache at pos, or the caller's k_new
-    int64_t sb, sh;     // element strides of k between sequences / KV heads
-    // fused append (ckv_append_assign): copy the caller's rows into the cache
-    const void* k_new;
-    const void* v_new;
-    void* k_dst;        // K row (b = 0, kv head 0) at pos; NULL: no append
-    void* v_dst;
-    int64_t csb, csh;   // cache element strides between sequences / KV heads
-    int row_vec;        // 16-byte vectors per row
-    int U, G, Hq, Hkv, d, per_head, Cmax, T_cap, max_tail, pos;
-    float inv_sqrt_d;
-    const int32_t* nbr8;
-    int32_t* comm_of;
-    int32_t* cnt;
-    float* cent;
-    int32_t* tail_tok;
-    int32_t* tail_comm;
-    int32_t* tail_len;
-    int32_t* dev_err;
-    int32_t* assigned;
-};
-
-// One block per graph unit; warp i scores candidate i (the community of
-// neighbour i, skipped when empty or already seen), so all candidate centres
-// are fetched at once.  Thread 0 picks the winner; the block updates its
-// centre row.
+// One block per graph unit, one warp per candidate (see assign_unit).
 template <typename T, int D>
 __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParams p) {
-    constexpr int E = D / 32;
-    __shared__ int s_cand[CKV_NEIGHBOURS];
-    __shared__ float s_score[CKV_NEIGHBOURS];
-    __shared__ int s_best, s_n, s_tl;
+    __shared__ int s_nbr[CKV_NEIGHBOURS];
     pdl_wait();  // everything this kernel reads may come from the kernel before it
-    const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = u / p.G, g = u - b * p.G;
-    const int gq = p.Hq / p.Hkv;
-    const int kvh = p.per_head ? g / gq : g;
-    if (p.k_dst && (!p.per_head || g % gq == 0) && warp == CKV_NEIGHBOURS - 1) {
-        // the first graph of each (sequence, KV head) appends its K and V rows
-        const uint4* ks = static_cast<const uint4*>(p.k_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
-        const uint4* vs = static_cast<const uint4*>(p.v_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
-        const size_t eoff = (size_t)(b * p.csb + kvh * p.csh);  // elements
-        const size_t esz = p.row_vec * 16 / (size_t)p.d;
-        uint4* kd = reinterpret_cast<uint4*>(static_cast<char*>(p.k_dst) + eoff * esz);
-        uint4* vd = reinterpret_cast<uint4*>(static_cast<char*>(p.v_dst) + eoff * esz);
-        for (int i = lane; i < p.row_vec; i += 32) {
-            kd[i] = ks[i];
-            vd[i] = vs[i];
-        }
-    }
-    if (tid < CKV_NEIGHBOURS) {
-        int c = -1;
-        const int np = p.nbr8[(size_t)u * CKV_NEIGHBOURS + tid];
-        if (np >= 0 && np < p.T_cap) {
-            const int cc = p.comm_of[(size_t)u * p.T_cap + np];
-            if (cc >= 0 && cc < p.Cmax) c = cc;
-        }
-        s_cand[tid] = c;
-    }
-    if (tid == 0) {
-        s_tl = p.tail_len[u];
-    }
-    const T* krow = static_cast<const T*>(p.k) + b * p.sb + kvh * p.sh + lane * E;
-    float kx[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) kx[e] = to_f32(krow[e]);
+    const int u = blockIdx.x;
+    if (threadIdx.x < CKV_NEIGHBOURS) s_nbr[threadIdx.x] = p.nbr8[(size_t)u * CKV_NEIGHBOURS + threadIdx.x];
     __syncthreads();
-
-    // warp i: score of candidate i (-inf when absent or a repeat)
-    {
-        const int ci = s_cand[warp];
-        bool use = ci >= 0;
-        for (int j = 0; j < warp; ++j) use = use && s_cand[j] != ci;
-        float s = -INFINITY;
-        if (use) {
-            const float* cr = p.cent + ((size_t)u * p.Cmax + ci) * D + lane * E;
-            float a = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) a = fmaf(kx[e], cr[e], a);
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
-            s = a * p.inv_sqrt_d;
-        }
-        if (lane == 0) s_score[warp] = use ? s : -INFINITY;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int best = -1;
-        float bs = -INFINITY;
-        for (int i = 0; i < CKV_NEIGHBOURS; ++i) {
-            const int ci = s_cand[i];
-            if (ci < 0 || s_score[i] == -INFINITY) continue;
-            if (best < 0 || s_score[i] > bs || (s_score[i] == bs && ci < best)) {
-                best = ci;
-                bs = s_score[i];
-            }
-        }
-        int32_t* cpos = p.comm_of + (size_t)u * p.T_cap + p.pos;
-        if (best >= 0 && s_tl >= p.max_tail) {
-            atomicOr(p.dev_err, CKV_DEVERR_TAIL_FULL);
-            best = -1;
-        }
-        s_best = best;
-        if (best < 0) {
-            *cpos = -1;
-            if (p.assigned) p.assigned[u] = -1;
-        } else {
-            const int n = p.cnt[(size_t)u * p.Cmax + best];
-            s_n = n;
-            p.cnt[(size_t)u * p.Cmax + best] = n + 1;
-            *cpos = best;
-            p.tail_tok[(size_t)u * p.max_tail + s_tl] = p.pos;
-            p.tail_comm[(size_t)u * p.max_tail + s_tl] = best;
-            p.tail_len[u] = s_tl + 1;
-            if (p.assigned) p.assigned[u] = best;
-        }
-    }
-    __syncthreads();
-    const int best = s_best;
-    if (best < 0 || warp != 0) return;
-    // running mean: c <- c + (k - c) / (n + 1)
-    float* cr = p.cent + ((size_t)u * p.Cmax + best) * D + lane * E;
-    const float denom = (float)(s_n + 1);
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const float c0 = cr[e];
-        cr[e] = c0 + (kx[e] - c0) / denom;
-    }
+    assign_unit<T, D, CKV_NEIGHBOURS>(p, u, s_nbr, threadIdx.x, [] { __syncthreads(); });
 }
 
 cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const void* k_new,
                                  const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st) {
-    AssignParams p{};
-    const size_t esz = c.dtype == CKV_DTYPE_BF16 ? 2 : 4;
-    if (k_new) {
-        // new key from the caller's contiguous [B, Hkv, d] rows; append them
-        p.k = k_new;
-        p.sb = (int64_t)c.Hkv * c.d;
-        p.sh = c.d;
-        p.k_new = k_new;
-        p.v_new = v_new;
-        p.k_dst = const_cast<char*>(static_cast<const char*>(c.k)) + (size_t)pos * c.st * esz;
-        p.v_dst = const_cast<char*>(static_cast<const char*>(c.v)) + (size_t)pos * c.st * esz;
-    } else {
-        // new key already in the cache at pos
-        p.k = static_cast<const char*>(c.k) + (size_t)pos * c.st * esz;
-        p.sb = c.sb;
-        p.sh = c.sh;
-    }
-    p.csb = c.sb;
-    p.csh = c.sh;
-    p.row_vec = (int)(c.d * esz / 16);
-    p.U = c.B * g.G;
-    p.G = g.G;
-    p.Hq = c.Hq;
-    p.Hkv = c.Hkv;
-    p.d = c.d;
-    p.per_head = g.mode == CKV_GRAPH_PER_HEAD;
-    p.Cmax = g.Cmax;
-    p.T_cap = g.T_cap;
-    p.max_tail = g.max_tail;
-    p.pos = pos;
-    p.inv_sqrt_d = 1.0f / sqrtf((float)c.d);
-    p.nbr8 = nbr8;
-    p.comm_of = g.comm_of;
-    p.cnt = g.cnt;
-    p.cent = g.cent;
-    p.tail_tok = g.tail_tok;
-    p.tail_comm = g.tail_comm;
-    p.tail_len = g.tail_len;
-    p.dev_err = g.dev_err;
-    p.assigned = assigned;
+    const AssignParams p = make_assign_params(c, g, pos, k_new, v_new, nbr8, assigned);
     if (p.U <= 0) return cudaSuccess;
     const dim3 grid(p.U), block(CKV_NEIGHBOURS * 32);
     if (c.dtype == CKV_DTYPE_BF16) {

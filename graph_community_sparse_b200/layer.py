@@ -11,6 +11,7 @@ from typing import Optional
 import torch
 
 from . import (PER_GROUP, PER_HEAD, Graph, Selection, cache_desc, ckv_append_assign, ckv_assign_update,
+               ckv_sparse_decode_append,
                ckv_build_centroids, ckv_dense_decode, ckv_score_select, ckv_sparse_decode,
                ckv_workspace_size, new_graph, new_selection, new_workspace, NEIGHBOURS)
 
@@ -57,6 +58,15 @@ class LayerState:
     def decode(self, q: torch.Tensor, budget: int, want_nbr: bool = True, stream=None) -> torch.Tensor:
         self.select(q, budget, stream)
         return self.attend(q, want_nbr, stream)
+
+    def attend_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> torch.Tensor:
+        """attend (neighbours into nbr8) and append in one call: the update
+        runs inside the attention's merge kernel."""
+        pos = self.T
+        ckv_sparse_decode_append(self.cache, q, self.graph, self.sel, self.out, self.nbr8, pos, k_new.contiguous(),
+                                 v_new.contiguous(), self.assigned, self.ws, stream)
+        self.T += 1
+        return self.out
 
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> torch.Tensor:
         """Write the new token's K/V rows ([B, Hkv, d]) at position T and let

@@ -270,6 +270,20 @@ CKV_API ckv_status ckv_append_assign(const ckv_cache_desc* cache, const ckv_grap
                                      const int32_t* nbr8, int32_t* assigned, ckv_stream_t stream);
 
 /*
+ * One call for the decode step after the selection: ckv_sparse_decode
+ * followed by ckv_append_assign (pos, k_new, v_new, assigned as there),
+ * with the update run by the attention's merge kernel as soon as each unit's
+ * neighbours are known, so no separate update launch follows.  nbr8 may be
+ * NULL (the neighbours are then not written out).  Same results, bit for
+ * bit, as the two calls in sequence.
+ */
+CKV_API ckv_status ckv_sparse_decode_append(const ckv_cache_desc* cache, const void* q,
+                                            const ckv_graph_desc* graph, const ckv_selection_desc* sel,
+                                            float* out, int32_t* nbr8, int32_t pos, const void* k_new,
+                                            const void* v_new, int32_t* assigned, void* ws,
+                                            size_t ws_bytes, ckv_stream_t stream);
+
+/*
  * Dense comparator: exact GQA decode attention over positions [0, T) of every
  * (b, kv head), out fp32 [B, Hq, d].  The pages measure their speed-ups against
  * dense attention ([R-B], [ABS]).  Workspace: ckv_workspace_size().

@@ -156,6 +156,15 @@ CASES = [
                                                                   5, FAKE, FAKE + 8, FAKE, FAKE, None), INVALID),
     ("append null nbr", lambda: ckv.lib.ckv_append_assign(ctypes.byref(_cache()), ctypes.byref(_graph()), 5,
                                                           FAKE, FAKE, None, FAKE, None), INVALID),
+    ("fused pos", lambda: ckv.lib.ckv_sparse_decode_append(ctypes.byref(_cache()), FAKE, ctypes.byref(_graph()),
+                                                           ctypes.byref(_sel()), FAKE, None, 4096, FAKE, FAKE,
+                                                           None, FAKE, 1 << 40, None), CAPACITY),
+    ("fused null v_new", lambda: ckv.lib.ckv_sparse_decode_append(ctypes.byref(_cache()), FAKE, ctypes.byref(_graph()),
+                                                                  ctypes.byref(_sel()), FAKE, None, 5, FAKE, None,
+                                                                  None, FAKE, 1 << 40, None), INVALID),
+    ("fused ws small", lambda: ckv.lib.ckv_sparse_decode_append(ctypes.byref(_cache()), FAKE, ctypes.byref(_graph()),
+                                                                ctypes.byref(_sel()), FAKE, None, 5, FAKE, FAKE,
+                                                                None, FAKE, 1000, None), WORKSPACE),
     ("dense T", lambda: ckv.lib.ckv_dense_decode(ctypes.byref(_cache()), FAKE, 0, FAKE, FAKE, 1 << 40, None),
      CAPACITY),
     ("dense ws", lambda: ckv.lib.ckv_dense_decode(ctypes.byref(_cache()), FAKE, 100, FAKE, FAKE, 8, None),

@@ -238,3 +238,27 @@ def test_many_candidates_global_sort(budget_frac):
     for _ in range(wl.steps):
         case.step(wl.budget)
     assert int(case.st.sel.n_sel.max().item()) > 256
+
+
+def test_fused_decode_append_matches_separate_calls():
+    """ckv_sparse_decode_append (update run by the merge kernel) gives the
+    same outputs, neighbours, cache and graph state, bit for bit, as
+    ckv_sparse_decode followed by ckv_append_assign."""
+    for wl in (small("fused_head", 40, mode="head", T=2500, budgets=(200,), steps=3),
+               small("fused_group", 41, steps=3), synth.WORKLOADS["tiny"].replace(steps=3)):
+        a, b = Case(wl), Case(wl)
+        for i in range(wl.steps):
+            q = synth.draw_queries(wl, a.draw, i)
+            kn, vn = synth.draw_new_tokens(wl, a.draw, i)
+            kn, vn = kn.to(a.st.K.dtype), vn.to(a.st.V.dtype)
+            a.st.select(q, wl.budget)
+            b.st.select(q, wl.budget)
+            oa = a.st.attend_append(q, kn, vn).clone()
+            ob = b.st.attend(q).clone()
+            b.st.append(kn, vn)
+            torch.cuda.synchronize()
+            assert torch.equal(oa, ob), wl.key
+            assert torch.equal(a.st.nbr8, b.st.nbr8) and torch.equal(a.st.assigned, b.st.assigned)
+            assert torch.equal(a.st.K, b.st.K) and torch.equal(a.st.V, b.st.V)
+            for name in ("comm_of", "cnt", "cent", "tail_tok", "tail_comm", "tail_len", "dev_err"):
+                assert torch.equal(getattr(a.st.graph, name), getattr(b.st.graph, name)), (wl.key, name)
