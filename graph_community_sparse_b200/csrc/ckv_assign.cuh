@@ -97,7 +97,9 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     constexpr int E = D / 32;
     __shared__ int s_cand[CKV_NEIGHBOURS];
     __shared__ float s_score[CKV_NEIGHBOURS];
-    __shared__ int s_best, s_n, s_tl;
+    __shared__ int s_cnt[CKV_NEIGHBOURS];
+    __shared__ float s_row[CKV_NEIGHBOURS][D];  // candidate centres, reused by the update
+    __shared__ int s_best, s_bi, s_n, s_tl;
     const int lane = tid & 31, warp = tid >> 5;
     const int b = u / p.G, g = u - b * p.G;
     const int gq = p.Hq / p.Hkv;
@@ -140,9 +142,14 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
         float s = -INFINITY;
         if (use) {
             const float* cr = p.cent + ((size_t)u * p.Cmax + ci) * D + lane * E;
+            if (lane == 0) s_cnt[i] = p.cnt[(size_t)u * p.Cmax + ci];
             float a = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) a = fmaf(kx[e], cr[e], a);
+            for (int e = 0; e < E; ++e) {
+                const float c = cr[e];
+                s_row[i][lane * E + e] = c;
+                a = fmaf(kx[e], c, a);
+            }
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
             s = a * p.inv_sqrt_d;
@@ -151,13 +158,14 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     }
     sync();
     if (tid == 0) {
-        int best = -1;
+        int best = -1, bi = -1;
         float bs = -INFINITY;
         for (int i = 0; i < CKV_NEIGHBOURS; ++i) {
             const int ci = s_cand[i];
             if (ci < 0 || s_score[i] == -INFINITY) continue;
             if (best < 0 || s_score[i] > bs || (s_score[i] == bs && ci < best)) {
                 best = ci;
+                bi = i;
                 bs = s_score[i];
             }
         }
@@ -167,11 +175,12 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
             best = -1;
         }
         s_best = best;
+        s_bi = bi;
         if (best < 0) {
             *cpos = -1;
             if (p.assigned) p.assigned[u] = -1;
         } else {
-            const int n = p.cnt[(size_t)u * p.Cmax + best];
+            const int n = s_cnt[bi];  // read by the candidate's warp above
             s_n = n;
             p.cnt[(size_t)u * p.Cmax + best] = n + 1;
             *cpos = best;
@@ -184,12 +193,14 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     sync();
     const int best = s_best;
     if (best < 0 || warp != 0) return;
-    // running mean: c <- c + (k - c) / (n + 1)
+    // running mean: c <- c + (k - c) / (n + 1), from the copy of the centre
+    // taken while scoring
     float* cr = p.cent + ((size_t)u * p.Cmax + best) * D + lane * E;
+    const float* c0r = s_row[s_bi] + lane * E;
     const float denom = (float)(s_n + 1);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        const float c0 = cr[e];
+        const float c0 = c0r[e];
         cr[e] = c0 + (kx[e] - c0) / denom;
     }
 }

@@ -55,9 +55,11 @@ struct DynSplit {
     int nch;    // dynamic chunks
 };
 
-__host__ __device__ __forceinline__ DynSplit dyn_split(int total, int W) {
+// dense: static slices only (its units are long, so a dynamic tail would
+// multiply the partials each merge block combines)
+__host__ __device__ __forceinline__ DynSplit dyn_split(int total, int W, bool dense) {
     DynSplit d;
-    const int dyn = total / DYN_DEN;
+    const int dyn = dense ? 0 : total / DYN_DEN;
     d.chk = max(DYN_CHUNK_MIN, (dyn + NCH_MAX - 1) / NCH_MAX);
     d.nch = (dyn + d.chk - 1) / d.chk;
     d.R = total - dyn;
@@ -105,7 +107,6 @@ struct DecodeParams {
     float* out;
     int32_t* nbr8;          // may be NULL when only the fused update needs them
     int append;             // fused community update (and K/V append) in the merge
-    int key_bf16;           // dtype of the new key rows
     AssignParams ap;
 };
 
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(
         total = p.U * p.T;
     }
     if (total <= 0) return;
-    const DynSplit sp = dyn_split(total, p.W);
+    const DynSplit sp = dyn_split(total, p.W, DENSE);
 
     // tokens [start, end) of the concatenated lists; partial of unit u in
     // slot sbase + u
@@ -463,11 +464,10 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x)
 
 // The fused community update of unit u by the merge block's NBR_WARPS
 // neighbour warps (thread xt of 32 NBR_WARPS), given its neighbour positions.
-template <int D>
+template <typename T, int D>
 __device__ __forceinline__ void merge_assign(const DecodeParams& p, int u, const int* nbpos, int xt) {
     auto sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory"); };
-    if (p.key_bf16) assign_unit<__nv_bfloat16, D, NBR_WARPS>(p.ap, u, nbpos, xt, sync);
-    else assign_unit<float, D, NBR_WARPS>(p.ap, u, nbpos, xt, sync);
+    assign_unit<T, D, NBR_WARPS>(p.ap, u, nbpos, xt, sync);
 }
 
 // One block per unit: threads 0..D-1 own one output dimension each (all the
@@ -475,7 +475,7 @@ __device__ __forceinline__ void merge_assign(const DecodeParams& p, int u, const
 // combined in slot order, a chunk of slots at a time, by a per-thread online
 // merge: no shared memory and no barriers, so the merge costs about two
 // dependent rounds of loads.
-template <int D, int GQ, bool DENSE>
+template <typename T, int D, int GQ, bool DENSE>
 __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_merge(DecodeParams p) {
     pdl_wait();  // the attention kernel's partials are complete and visible
     const int u = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -500,13 +500,13 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
         if (!DENSE && p.append && warp >= D / 32) {
             __shared__ int s_none[CKV_NEIGHBOURS];
             if (t - D < CKV_NEIGHBOURS) s_none[t - D] = -1;
-            merge_assign<D>(p, u, s_none, t - D);  // no neighbour: the token joins nothing
+            merge_assign<T, D>(p, u, s_none, t - D);  // no neighbour: the token joins nothing
         }
         return;
     }
     // the unit's partials: static slices [sA, sA + nA), then dynamic chunks
     // [sB, sB + nB) (the attention kernel's split, recomputed)
-    const DynSplit sp = dyn_split(total, p.W);
+    const DynSplit sp = dyn_split(total, p.W, DENSE);
     int nA = 0, nB = 0;
     size_t sA = 0, sB = 0;
     if (ubeg < sp.R) {
@@ -615,7 +615,7 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
         }
         if (p.append) {
             asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory");  // s_nbpos complete
-            merge_assign<D>(p, u, s_nbpos, xt);
+            merge_assign<T, D>(p, u, s_nbpos, xt);
         }
         return;
     }
@@ -737,7 +737,7 @@ cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
     p.W = blocks * DEC_WARPS;
     e = launch_pdl(kern, dim3(blocks), dim3(DEC_WARPS * 32), smem, st, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_merge<D, GQ, DENSE>, dim3(p.U), dim3(D + (DENSE ? 0 : 32 * NBR_WARPS)), 0, st, p);
+    return launch_pdl(decode_merge<T, D, GQ, DENSE>, dim3(p.U), dim3(D + (DENSE ? 0 : 32 * NBR_WARPS)), 0, st, p);
 }
 
 template <bool DENSE>
@@ -788,7 +788,6 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
     p.nbr8 = nbr8;
     if (ap) {
         p.append = 1;
-        p.key_bf16 = c.dtype == CKV_DTYPE_BF16;
         p.ap = *ap;
     }
     return dispatch<false>(c, g.gq, p, st);

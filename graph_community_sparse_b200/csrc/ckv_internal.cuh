@@ -264,7 +264,8 @@ inline size_t ws_head_bytes(int B, int Hq) { return WS_RESERVED + align256((size
 // the launch itself (block scheduling) with that kernel's tail.  No kernel
 // signals its dependents early: measured on the step, letting the next
 // kernel's blocks take SM slots before the previous kernel ends slowed the
-// scoring and selection and did not speed up the attention.
+// scoring and selection, and the attention followed by its merge (about
+// 63 -> 71 us per call on a 128K-context batch of 8).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 template <typename... Params, typename... Args>
