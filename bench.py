@@ -303,13 +303,14 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     # per-call breakdown (for the roofline), in its own pass of steps right
     # after the timed ones, with an event between the two calls
     bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(B_steps)]
-    rows_hist, ntok_hist, ncomm_hist = [], [], []
+    rows_hist, ntok_hist, nsel_hist, ncomm_hist = [], [], [], []
     for j in range(B_steps):
         new_episode_if_due()
         flush()
         one_step(W_steps + K_steps + j, bevs[j], per_call=True)
         rows_hist.append(count_rows(st.sel))
         ntok_hist.append(st.sel.n_tok.long().sum())
+        nsel_hist.append(st.sel.n_sel.long().sum())
         ncomm_hist.append(num_comm.sum())
     torch.cuda.synchronize()
     if int(st.graph.dev_err.item()) != 0:
@@ -319,6 +320,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
 
     rows = np.array([int(r.item()) for r in rows_hist], dtype=np.float64)
     ntok = np.array([int(r.item()) for r in ntok_hist], dtype=np.float64)
+    nsel = np.array([int(r.item()) for r in nsel_hist], dtype=np.float64)
     ncomm = float(ncomm_hist[0].item())
     q_bytes = wl.B * wl.Hq * wl.d * esz
     out_bytes = wl.B * wl.Hq * wl.d * 4
@@ -328,7 +330,10 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         # up to 8 candidate centres read per unit, one centre row updated,
         # and the new K/V rows copied into the cache
         dec_bytes = dec_bytes + ntok * 8 + U * (8 * 4 + 8 * wl.d * 4 + 2 * wl.d * 4) + 4 * wl.B * wl.Hkv * wl.d * esz
-    sel_bytes = ncomm * wl.d * 4 + q_bytes + ncomm * 4 * 3 + ntok * 4
+    # the scoring pass reads every centre in bf16; the selected communities
+    # (at least) are re-scored from the fp32 centres; per community a size is
+    # read and a score bound written and read back; the token list is written
+    sel_bytes = ncomm * wl.d * 2 + nsel * wl.d * 4 + q_bytes + ncomm * 4 * 3 + ntok * 4
     peak, peak_src = measured_peaks()
 
     def gbs(bytes_, ms):

@@ -34,6 +34,7 @@ struct AssignParams {
     int32_t* comm_of;
     int32_t* cnt;
     float* cent;
+    __nv_bfloat16* cent_lp;
     int32_t* tail_tok;
     int32_t* tail_comm;
     int32_t* tail_len;
@@ -79,6 +80,7 @@ inline AssignParams make_assign_params(const CacheView& c, const GraphView& g, i
     p.comm_of = g.comm_of;
     p.cnt = g.cnt;
     p.cent = g.cent;
+    p.cent_lp = g.cent_lp;
     p.tail_tok = g.tail_tok;
     p.tail_comm = g.tail_comm;
     p.tail_len = g.tail_len;
@@ -196,12 +198,15 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     // running mean: c <- c + (k - c) / (n + 1), from the copy of the centre
     // taken while scoring
     float* cr = p.cent + ((size_t)u * p.Cmax + best) * D + lane * E;
+    __nv_bfloat16* clp = p.cent_lp + ((size_t)u * p.Cmax + best) * D + lane * E;
     const float* c0r = s_row[s_bi] + lane * E;
     const float denom = (float)(s_n + 1);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const float c0 = c0r[e];
-        cr[e] = c0 + (kx[e] - c0) / denom;
+        const float c1 = c0 + (kx[e] - c0) / denom;
+        cr[e] = c1;
+        clp[e] = __float2bfloat16_rn(c1);  // the scoring copy follows the centre
     }
 }
 

@@ -32,6 +32,7 @@ struct BuildParams {
     int32_t* tok;
     int32_t* cnt;
     float* cent;
+    __nv_bfloat16* cent_lp;
     int32_t* num_comm;
     int32_t* tail_len;
     int32_t* dev_err;
@@ -166,7 +167,9 @@ __global__ void __launch_bounds__(256) build_mean(BuildParams p) {
         double s = 0.0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
-        p.cent[((size_t)u * p.Cmax + c) * D + threadIdx.x] = n > 0 ? (float)(s / (double)n) : 0.f;
+        const float m = n > 0 ? (float)(s / (double)n) : 0.f;
+        p.cent[((size_t)u * p.Cmax + c) * D + threadIdx.x] = m;
+        p.cent_lp[((size_t)u * p.Cmax + c) * D + threadIdx.x] = __float2bfloat16_rn(m);
     }
 }
 
@@ -199,6 +202,7 @@ cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* 
     p.tok = g.tok;
     p.cnt = g.cnt;
     p.cent = g.cent;
+    p.cent_lp = g.cent_lp;
     p.num_comm = g.num_comm;
     p.tail_len = g.tail_len;
     p.dev_err = g.dev_err;

@@ -190,6 +190,7 @@ struct GraphView {
     int32_t* tok;
     int32_t* cnt;
     float* cent;
+    __nv_bfloat16* cent_lp;
     int32_t* num_comm;
     int32_t* tail_tok;
     int32_t* tail_comm;

@@ -6,24 +6,31 @@
 // re-clustering", paragraph 4); the active token budget is small (section
 // "The speed-up depends on how many graphs the model stores").
 //
-// Two kernels, 8 warps per block:
-//  * score_kernel, grid (centre blocks of 64, units): s_c = max over the
-//    graph's query heads of q_h . cent_c / sqrt(d), a streaming
-//    matrix-vector product over the fp32 centres (one half-warp per row,
+// The score is s_c = max over the graph's query heads of q_h . cent_c /
+// sqrt(d) in fp32, and the selection is exactly the one those scores give;
+// but the centres are streamed only once, in bf16 (cent_lp), which halves
+// the bytes of the pass over every community:
+//  * score_kernel, grid (centre blocks of 128, units): a streaming
+//    matrix-vector product over the bf16 centres (one half-warp per row,
 //    16-byte loads, the value-exchanging butterfly of the attention kernel
-//    for the head sums).  Each score is stored and its community size is
-//    added, with a global atomic, to a per-unit histogram over the top 12
-//    bits of its key, key = (orderable score << 32) | ~id (unique; orders
-//    communities by score desc, id asc);
+//    for the head sums) gives s~_c and a rigorous bound e_c >= |s_c - s~_c|
+//    from sum |q| |cent_lp| (LP_REL_BOUND).  The upper bound s~ + e is
+//    stored; the community's size is added, with a global atomic, to a
+//    per-unit histogram over the top 12 bits of the key of the lower bound
+//    s~ - e, key = (orderable score << 32) | ~id (unique; orders communities
+//    by score desc, id asc);
 //  * select_kernel, one block per unit, launched as a programmatic
-//    dependent (its launch overlaps the scoring; it waits in hardware for the
-//    scores): the histogram gives the bin the budget cut falls in; only the
-//    keys from that bin up (typically a few dozen) are ranked, each against
-//    all the others in shared memory, which also gives the size above it and
-//    so the cut (at least the top community), with no sort.  Then
-//    the unit's token list: sinks, build-time members of each selected
-//    community (from the community-contiguous CSR), then the selected tail
-//    members.
+//    dependent: the lower-bound histogram gives a bin edge t with more than
+//    the budget's weight of communities certainly scoring >= t, so every
+//    selected community scores >= t; the candidates are the communities
+//    whose upper bound reaches t (typically a few dozen), and only they are
+//    re-scored exactly in fp32 from cent.  A non-candidate scores below t
+//    and so below every selected one, so ranking the candidates alone, each
+//    against the others in shared memory (which also gives the size above
+//    it and so the cut, at least the top community, with no sort), gives
+//    the exact selection.  Then the unit's token list: sinks, build-time
+//    members of each selected community (from the community-contiguous CSR),
+//    then the selected tail members.
 // The histograms live in the workspace head: zero on entry, and each
 // selection block clears its unit's histogram after reading it.
 #include <math.h>
@@ -34,15 +41,23 @@ namespace ckv {
 
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_THREADS = SEL_WARPS * 32;
-constexpr int SCORE_ROWS = SEL_WARPS * 8;  // centres per block
+constexpr int SCORE_ROWS = SEL_WARPS * 16;  // centres per block
 constexpr int SEL_HBITS = HIST_BITS;
 constexpr int SEL_HBINS = HIST_BINS;
-constexpr int SEL_FAST = SEL_THREADS;       // candidates sorted in registers
+constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
+// Bound on |fp32 score from cent - fp32 score from cent_lp| per unit of
+// sum_i |q_i| |cent_lp_i| / sqrt(d): bf16 rounding contributes at most 2^-9
+// (1 + 2^-9), the two fp32 dot products' rounding (depth <= 13 for d <= 128)
+// about 2^-19 each; 2^-8 leaves a factor 1.9 of margin.  The absolute term
+// covers bf16 subnormals.
+constexpr float LP_REL_BOUND = 1.0f / 256.0f;
+constexpr float LP_ABS_BOUND = 1e-30f;
 
 struct SelectParams {
     const void* q;
     const float* cent;
-    float* scores;              // [U, Cmax]
+    const __nv_bfloat16* cent_lp;
+    float* scores;              // [U, Cmax] upper bound of each score (first pass)
     int32_t* hist;              // [U, SEL_HBINS]
     unsigned long long* gkey;   // [U, npow_max] scratch for large candidate sets
     int32_t* gw;                // [U, npow_max]
@@ -92,14 +107,47 @@ __device__ int block_scan_inplace(int* a, int n, int* s_warp) {
     return total;
 }
 
-// Scores of this block's (up to) SCORE_ROWS centres of unit u.
+// Raw bf16 row part of a lane (E elements, 2E bytes), kept packed until used.
+template <int E> struct RawPart;
+template <> struct RawPart<8> {
+    uint4 w;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void zero() { w = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[8]) const {
+        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+        x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+    }
+};
+template <> struct RawPart<4> {
+    uint2 w;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint2*>(p); }
+    __device__ __forceinline__ void zero() { w = make_uint2(0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[4]) const {
+        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    }
+};
+
+// First-pass scores of this block's (up to) SCORE_ROWS centres of unit u:
+// a warp owns SCORE_ROWS / SEL_WARPS consecutive rows, a half-warp every
+// other one; all of a lane's row parts are loaded (packed) before any is
+// used, so each warp keeps SCORE_ROWS / SEL_WARPS bf16 rows in flight.
 template <typename T, int D, int GQ>
 __device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) {
     constexpr int E = D / 16;
+    constexpr int RW = SCORE_ROWS / SEL_WARPS;  // rows per warp
+    constexpr int RH = RW / 2;                  // rows per half-warp
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int half = lane >> 4, l16 = lane & 15;
-    const int row0 = blockIdx.x * SCORE_ROWS + warp * 8;
+    const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
     if (row0 >= C) return;
+    RawPart<E> raw[RH];
+#pragma unroll
+    for (int j = 0; j < RH; ++j) {
+        const int c = row0 + 2 * j + half;
+        if (c < C) raw[j].load(p.cent_lp + ((size_t)u * p.Cmax + c) * D + l16 * E);
+        else raw[j].zero();
+    }
+    const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
     const int b = u / p.G, g = u - b * p.G;
     const int h0 = p.per_head ? g : g * GQ;
     float qr[GQ][E];
@@ -107,42 +155,41 @@ __device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) 
     for (int h = 0; h < GQ; ++h)
         load_row_part<T, E>(static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h0 + h) * D + l16 * E, qr[h]);
 
-    float x[4][E];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int c = row0 + 2 * j + half;
-        if (c < C) {
-            load_row_part<float, E>(p.cent + ((size_t)u * p.Cmax + c) * D + l16 * E, x[j]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < E; ++e) x[j][e] = 0.f;
-        }
-    }
-    const int wc = (lane < 8 && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
     int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float part[GQ];
+    for (int j = 0; j < RH; ++j) {
+        float x[E];
+        raw[j].unpack(x);
+        float part[GQ], mag[GQ];
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
-            float a = 0.f;
+            float a = 0.f, m = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) a = fmaf(qr[h][e], x[j][e], a);
+            for (int e = 0; e < E; ++e) {
+                a = fmaf(qr[h][e], x[e], a);
+                m = fmaf(fabsf(qr[h][e]), fabsf(x[e]), m);
+            }
             part[h] = a;
+            mag[h] = m;
         }
         float s = halfwarp_reduce_heads<GQ>(part, lane);
         s = halfwarp_max_over_heads<GQ>(s) * p.inv_sqrt_d;
+        float m = halfwarp_reduce_heads<GQ>(mag, lane);
+        m = halfwarp_max_over_heads<GQ>(m) * p.inv_sqrt_d;
+        // |exact score - s| <= 2^-8 m (see LP_REL_BOUND)
+        const float err = fmaf(LP_REL_BOUND, m, LP_ABS_BOUND);
         const int c = row0 + 2 * j + half;
         const int w = __shfl_sync(FULL, wc, 2 * j + half);
         if (l16 == 0 && c < C) {
-            p.scores[(size_t)u * p.Cmax + c] = s;
-            if (w > 0) atomicAdd(hist + (int)(score_key(s, c) >> (64 - SEL_HBITS)), w);
+            p.scores[(size_t)u * p.Cmax + c] = s + err;
+            if (w > 0) atomicAdd(hist + (int)(score_key(s - err, c) >> (64 - SEL_HBITS)), w);
         }
     }
 }
 
 // Selection for unit u after all its scores are in (see the file comment).
-// Scores and the histogram were written by other blocks: read through L2.
+// Score bounds and the histogram were written by other blocks: read through L2.
+template <typename T, int D, int GQ>
 __device__ void select_unit(const SelectParams& p, int u, int C) {
     __shared__ unsigned long long s_key[SEL_FAST];
     __shared__ int s_w[SEL_FAST];
@@ -200,6 +247,55 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         wv[r] = cn[c];
         sv[r] = __ldcg(sc + c);
     }
+    // this lane's part of the graph's queries, for the exact re-scoring
+    constexpr int EW = D / 32;
+    float qw[GQ][EW];
+    {
+        const int b = u / p.G, g = u - b * p.G;
+        const int h0 = p.per_head ? g : g * GQ;
+#pragma unroll
+        for (int h = 0; h < GQ; ++h)
+#pragma unroll
+            for (int e = 0; e < EW; ++e)
+                qw[h][e] = to_f32(static_cast<const T*>(p.q)[((size_t)b * p.Hq + h0 + h) * D + lane * EW + e]);
+    }
+    // exact fp32 scores, from cent, of the n candidates whose keys (built
+    // from the upper bounds) are in keys[]: one warp per candidate, four
+    // candidates' rows in flight per warp; the keys are replaced in place
+    auto rescore = [&](unsigned long long* keys, int n) {
+        for (int i0 = warp; i0 < n; i0 += 4 * nw) {
+            float row[4][EW];
+            int cid[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                cid[r] = key_id(keys[min(i0 + r * nw, n - 1)]);
+                const float* cr = p.cent + ((size_t)u * p.Cmax + cid[r]) * D + lane * EW;
+#pragma unroll
+                for (int e = 0; e < EW; ++e) row[r][e] = cr[e];
+            }
+            unsigned long long nk[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                float best = -INFINITY;
+#pragma unroll
+                for (int h = 0; h < GQ; ++h) {
+                    float a = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EW; ++e) a = fmaf(qw[h][e], row[r][e], a);
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+                    best = fmaxf(best, a);
+                }
+                nk[r] = score_key(best * p.inv_sqrt_d, cid[r]);
+            }
+            __syncwarp();  // every lane has read its keys before lane 0 rewrites them
+            if (lane == 0) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    if (i0 + r * nw < n) keys[i0 + r * nw] = nk[r];
+            }
+        }
+    };
 
     // 1. crossing bin: thread t owns bins [per*t, per*t + per)
     {
@@ -249,6 +345,10 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     }
     __syncthreads();
     const int nc = s_nc;
+    if (nc <= SEL_FAST) {
+        rescore(s_key, nc);
+        __syncthreads();
+    }
 
     // 3. the cut.  Few candidates (the usual case): no sort; candidate i's
     //    rank is the number of larger keys and the weight above it their size
@@ -294,6 +394,8 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
             const unsigned long long k = score_key(__ldcg(sc + c), c);
             if ((int)(k >> (64 - SEL_HBITS)) >= bstar) gk[atomicAdd(&s_nc, 1)] = k;
         }
+        __syncthreads();
+        rescore(gk, nc);
         __syncthreads();
         int np2 = 1;
         while (np2 < nc) np2 <<= 1;
@@ -442,11 +544,12 @@ __global__ void __launch_bounds__(SEL_THREADS) score_kernel(SelectParams p) {
     score_rows<T, D, GQ>(p, u, C);
 }
 
+template <typename T, int D, int GQ>
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
     pdl_wait();  // every score and histogram update of the scoring kernel is visible
     const int u = blockIdx.x;
     const int C = min(p.num_comm[u], p.Cmax);
-    select_unit(p, u, C);
+    select_unit<T, D, GQ>(p, u, C);
 }
 
 // ---------------------------------------------------------------------------
@@ -478,7 +581,7 @@ cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
     dim3 grid((p.Cmax + SCORE_ROWS - 1) / SCORE_ROWS, p.U);
     cudaError_t e = launch_pdl(score_kernel<T, D, GQ>, grid, dim3(SEL_THREADS), 0, st, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(select_kernel, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
+    return launch_pdl(select_kernel<T, D, GQ>, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
 }
 }  // namespace
 
@@ -492,6 +595,7 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     SelectParams p{};
     p.q = q;
     p.cent = g.cent;
+    p.cent_lp = g.cent_lp;
     p.scores = reinterpret_cast<float*>(w + l.scores);
     p.hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + WS_RESERVED);  // zero on entry
     p.gkey = reinterpret_cast<unsigned long long*>(w + l.gkey);

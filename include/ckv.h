@@ -64,7 +64,7 @@ extern "C" {
 #define CKV_API
 #endif
 
-#define CKV_ABI_VERSION 1
+#define CKV_ABI_VERSION 2
 #define CKV_NEIGHBOURS 8
 
 typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
@@ -112,6 +112,10 @@ typedef struct {
  *   tok      int32 [U, T_cap]   members sorted by (community, position)
  *   cnt      int32 [U, Cmax]    member count, including tail members
  *   cent     fp32  [U, Cmax, d] running-mean centre of each community
+ *   cent_lp  bf16  [U, Cmax, d] cent rounded to nearest, kept in step by the
+ *                  build and the update: the scoring streams it (half the
+ *                  bytes) and re-scores only the communities whose bounds
+ *                  reach the budget cut from cent (see ckv_score_select)
  *   num_comm int32 [U]          1 + largest community id present
  *   tail_tok, tail_comm int32 [U, max_tail]  tokens joined after the build
  *   tail_len int32 [U]
@@ -130,6 +134,7 @@ typedef struct {
     int32_t* tok;
     int32_t* cnt;
     float* cent;
+    uint16_t* cent_lp;  /* bf16 bits [U, Cmax, d]: cent rounded, for the first scoring pass */
     int32_t* num_comm;
     int32_t* tail_tok;
     int32_t* tail_comm;
@@ -187,7 +192,10 @@ CKV_API ckv_status ckv_build_centroids(const ckv_cache_desc* cache, const int32_
  *   select  rank non-empty communities by (s_c desc, id asc); take the
  *           longest ranked prefix whose cnt sum is <= budget, and at least the
  *           top community; the sinks come on top of the budget.
- * Writes every field of `sel`.  budget >= 0.
+ * Writes every field of `sel`.  budget >= 0.  The pass over all communities
+ * reads the bf16 copy cent_lp with a rigorous error bound per score; only
+ * the communities whose bound reaches the budget cut are re-scored from the
+ * fp32 cent, so the selection is the one the fp32 scores give.
  */
 CKV_API ckv_status ckv_score_select(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
                             const void* q, int32_t budget, const ckv_selection_desc* sel,

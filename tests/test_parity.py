@@ -262,3 +262,38 @@ def test_fused_decode_append_matches_separate_calls():
             assert torch.equal(a.st.K, b.st.K) and torch.equal(a.st.V, b.st.V)
             for name in ("comm_of", "cnt", "cent", "tail_tok", "tail_comm", "tail_len", "dev_err"):
                 assert torch.equal(getattr(a.st.graph, name), getattr(b.st.graph, name)), (wl.key, name)
+
+
+def test_scoring_copy_tracks_centres():
+    """cent_lp is cent rounded to bf16 (round to nearest even), after the
+    build and after every update."""
+    wl = small("cent_lp", 42, steps=3)
+    case = Case(wl)
+    assert torch.equal(case.st.graph.cent_lp, case.st.graph.cent.to(torch.bfloat16))
+    for _ in range(wl.steps):
+        case.step(wl.budget)
+        assert torch.equal(case.st.graph.cent_lp, case.st.graph.cent.to(torch.bfloat16))
+
+
+def test_cut_among_scores_closer_than_bf16():
+    """Every community's keys are one vector scaled by 1 + 1e-4 * id, so
+    neighbouring communities' scores differ by ~1e-3, far below what the bf16
+    scoring pass resolves (~2e-2) and far above the 1e-5 tie band: the exact
+    re-scoring alone decides the ranking and the cut, which must equal the
+    oracle's."""
+    wl = small("near_ties", 43, dtype="f32", B=1, T=3000, budgets=(1000,), steps=1, update=False)
+    case = Case(wl)
+    q = synth.draw_queries(wl, case.draw, 0)
+    labels = case.draw.labels
+    gq = wl.Hq // wl.Hkv
+    for g in range(wl.G):
+        lab = torch.from_numpy(labels[0, g].astype(np.int64)).cuda()
+        v = q[0, g * gq].float()
+        rows = v[None, :] * (1.0 + 1e-4 * lab.clamp(min=0).float())[:, None]
+        keep = lab < 0  # sinks keep their keys
+        case.st.K[0, g, : wl.T] = torch.where(keep[:, None], case.st.K[0, g, : wl.T], rows)
+    case.st.build(torch.from_numpy(labels.reshape(case.U, wl.T).astype(np.int32)).cuda(), wl.T)
+    rep = case.step(wl.budget, update=False)
+    assert rep.band_selections == 0
+    n_sel = case.st.sel.n_sel.cpu().numpy()
+    assert np.all(n_sel > 3)
