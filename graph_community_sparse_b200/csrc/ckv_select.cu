@@ -260,22 +260,23 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
                 qw[h][e] = to_f32(static_cast<const T*>(p.q)[((size_t)b * p.Hq + h0 + h) * D + lane * EW + e]);
     }
     // exact fp32 scores, from cent, of the n candidates whose keys (built
-    // from the upper bounds) are in keys[]: one warp per candidate, four
+    // from the upper bounds) are in keys[]: one warp per candidate, RSC
     // candidates' rows in flight per warp; the keys are replaced in place
+    constexpr int RSC = 8;
     auto rescore = [&](unsigned long long* keys, int n) {
-        for (int i0 = warp; i0 < n; i0 += 4 * nw) {
-            float row[4][EW];
-            int cid[4];
+        for (int i0 = warp; i0 < n; i0 += RSC * nw) {
+            float row[RSC][EW];
+            int cid[RSC];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < RSC; ++r) {
                 cid[r] = key_id(keys[min(i0 + r * nw, n - 1)]);
                 const float* cr = p.cent + ((size_t)u * p.Cmax + cid[r]) * D + lane * EW;
 #pragma unroll
                 for (int e = 0; e < EW; ++e) row[r][e] = cr[e];
             }
-            unsigned long long nk[4];
+            unsigned long long nk[RSC];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < RSC; ++r) {
                 float best = -INFINITY;
 #pragma unroll
                 for (int h = 0; h < GQ; ++h) {
@@ -291,7 +292,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
             __syncwarp();  // every lane has read its keys before lane 0 rewrites them
             if (lane == 0) {
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
+                for (int r = 0; r < RSC; ++r)
                     if (i0 + r * nw < n) keys[i0 + r * nw] = nk[r];
             }
         }
@@ -328,6 +329,10 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
             if (i < SEL_FAST) {
                 s_key[i] = k;
                 s_w[i] = w;
+                // its fp32 centre is re-scored next: start fetching it into L2
+                const char* row = reinterpret_cast<const char*>(p.cent + ((size_t)u * p.Cmax + c) * D);
+#pragma unroll
+                for (int l = 0; l < D * 4 / 128; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 128 * l));
             }
         }
     };
