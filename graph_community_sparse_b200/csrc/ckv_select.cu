@@ -350,6 +350,15 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     }
     __syncthreads();
     const int nc = s_nc;
+    const int32_t* of = p.offs + (size_t)u * (p.Cmax + 1);
+    // each candidate's CSR run, loaded now so the loads overlap the re-scoring
+    // (the id bits of a key do not change when it is re-scored)
+    int o0 = 0, o1 = 0;
+    if (tid < min(nc, SEL_FAST)) {
+        const int c = key_id(s_key[tid]);
+        o0 = of[c];
+        o1 = of[c + 1];
+    }
     if (nc <= SEL_FAST) {
         rescore(s_key, nc);
         __syncthreads();
@@ -362,7 +371,6 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     //    Each candidate's CSR run is looked up meanwhile and stored at its rank.
     int kstar;
     const unsigned long long* sorted;
-    const int32_t* of = p.offs + (size_t)u * (p.Cmax + 1);
     const bool small = nc <= SEL_FAST;
     int* bsz = small ? s_bsz : p.gw + (size_t)u * p.npow_max;
     if (small) {
@@ -370,8 +378,6 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         if (tid < nc) {
             const unsigned long long k = s_key[tid];
             const int w = s_w[tid];
-            const int c = key_id(k);
-            const int o0 = of[c], o1 = of[c + 1];
             int rank = 0, above = 0;
             for (int j = 0; j < nc; ++j) {
                 const bool gt = s_key[j] > k;
@@ -382,6 +388,12 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
             s_runs[rank] = k;
             s_bsz[rank] = o1 - o0;
             s_ofs[rank] = o0;
+            if (in || rank == 0) {
+                // the token copy reads this run next: start fetching it into L2
+                const int32_t* run = p.tok + (size_t)u * p.T_cap + o0;
+                const int lines = min((o1 - o0 + 31) >> 5, 8);
+                for (int l = 0; l < lines; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(run + 32 * l));
+            }
         }
         kstar = __syncthreads_count(in);
         if (kstar == 0 && nc > 0) kstar = 1;  // the top community alone exceeds the budget: take it
