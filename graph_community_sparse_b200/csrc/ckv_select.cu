@@ -118,6 +118,22 @@ template <> struct RawPart<8> {
         x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
     }
 };
+template <> struct RawPart<16> {
+    uint4 w0, w1;
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+        w0 = reinterpret_cast<const uint4*>(p)[0];
+        w1 = reinterpret_cast<const uint4*>(p)[1];
+    }
+    __device__ __forceinline__ void zero() { w0 = w1 = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[16]) const {
+        const uint32_t v[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            x[2 * i] = bf16_lo(v[i]);
+            x[2 * i + 1] = bf16_hi(v[i]);
+        }
+    }
+};
 template <> struct RawPart<4> {
     uint2 w;
     __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint2*>(p); }
@@ -131,8 +147,66 @@ template <> struct RawPart<4> {
 // a warp owns SCORE_ROWS / SEL_WARPS consecutive rows, a half-warp every
 // other one; all of a lane's row parts are loaded (packed) before any is
 // used, so each warp keeps SCORE_ROWS / SEL_WARPS bf16 rows in flight.
+// One query head per graph: 8 lanes per row (D/8 elements each), so a warp
+// instruction covers 4 rows and a row's sums take 3 shuffle levels.
+template <typename T, int D>
+__device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int C) {
+    constexpr int E = D / 8;
+    constexpr int RW = SCORE_ROWS / SEL_WARPS;  // rows per warp
+    constexpr int RQ = RW / 4;                  // rows per 8-lane group
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int oct = lane >> 3, l8 = lane & 7;
+    const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
+    if (row0 >= C) return;
+    RawPart<E> raw[RQ];
+#pragma unroll
+    for (int j = 0; j < RQ; ++j) {
+        const int c = row0 + 4 * j + oct;
+        if (c < C) raw[j].load(p.cent_lp + ((size_t)u * p.Cmax + c) * D + l8 * E);
+        else raw[j].zero();
+    }
+    const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
+    const int b = u / p.G, g = u - b * p.G;
+    float qr[E];
+    {
+        const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + g) * D + l8 * E;  // head g
+#pragma unroll
+        for (int e = 0; e < E; ++e) qr[e] = to_f32(qp[e]);
+    }
+    int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
+#pragma unroll
+    for (int j = 0; j < RQ; ++j) {
+        float x[E];
+        raw[j].unpack(x);
+        float a = 0.f, m = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            a = fmaf(qr[e], x[e], a);
+            m = fmaf(fabsf(qr[e]), fabsf(x[e]), m);
+        }
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) {
+            a += __shfl_xor_sync(FULL, a, o);
+            m += __shfl_xor_sync(FULL, m, o);
+        }
+        const float sc = a * p.inv_sqrt_d;
+        // |exact score - sc| <= 2^-8 m / sqrt(d) (see LP_REL_BOUND)
+        const float err = fmaf(LP_REL_BOUND, m * p.inv_sqrt_d, LP_ABS_BOUND);
+        const int c = row0 + 4 * j + oct;
+        const int w = __shfl_sync(FULL, wc, 4 * j + oct);
+        if (l8 == 0 && c < C) {
+            p.scores[(size_t)u * p.Cmax + c] = sc + err;
+            if (w > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), w);
+        }
+    }
+}
+
 template <typename T, int D, int GQ>
 __device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) {
+    if constexpr (GQ == 1) {
+        score_rows_gq1<T, D>(p, u, C);
+        return;
+    }
     constexpr int E = D / 16;
     constexpr int RW = SCORE_ROWS / SEL_WARPS;  // rows per warp
     constexpr int RH = RW / 2;                  // rows per half-warp
