@@ -134,6 +134,28 @@ template <> struct RawPart<16> {
         }
     }
 };
+template <> struct RawPart<32> {
+    uint4 w[4];
+    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = reinterpret_cast<const uint4*>(p)[i];
+    }
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __device__ __forceinline__ void unpack(float (&x)[32]) const {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t v[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                x[8 * i + 2 * k] = bf16_lo(v[k]);
+                x[8 * i + 2 * k + 1] = bf16_hi(v[k]);
+            }
+        }
+    }
+};
 template <> struct RawPart<4> {
     uint2 w;
     __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint2*>(p); }
@@ -147,21 +169,24 @@ template <> struct RawPart<4> {
 // a warp owns SCORE_ROWS / SEL_WARPS consecutive rows, a half-warp every
 // other one; all of a lane's row parts are loaded (packed) before any is
 // used, so each warp keeps SCORE_ROWS / SEL_WARPS bf16 rows in flight.
-// One query head per graph: 8 lanes per row (D/8 elements each), so a warp
-// instruction covers 4 rows and a row's sums take 3 shuffle levels.
+// One query head per graph: SC_LPR lanes per row (D/SC_LPR elements each),
+// so a warp instruction covers 32/SC_LPR rows and a row's sums take
+// log2(SC_LPR) shuffle levels.
+constexpr int SC_LPR = 8;
 template <typename T, int D>
 __device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int C) {
-    constexpr int E = D / 8;
+    constexpr int E = D / SC_LPR;
+    constexpr int GR = 32 / SC_LPR;             // rows per warp instruction
     constexpr int RW = SCORE_ROWS / SEL_WARPS;  // rows per warp
-    constexpr int RQ = RW / 4;                  // rows per 8-lane group
+    constexpr int RQ = RW / GR;                 // rows per lane group
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int oct = lane >> 3, l8 = lane & 7;
+    const int oct = lane / SC_LPR, l8 = lane % SC_LPR;
     const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
     if (row0 >= C) return;
     RawPart<E> raw[RQ];
 #pragma unroll
     for (int j = 0; j < RQ; ++j) {
-        const int c = row0 + 4 * j + oct;
+        const int c = row0 + GR * j + oct;
         if (c < C) raw[j].load(p.cent_lp + ((size_t)u * p.Cmax + c) * D + l8 * E);
         else raw[j].zero();
     }
@@ -185,15 +210,15 @@ __device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int
             m = fmaf(fabsf(qr[e]), fabsf(x[e]), m);
         }
 #pragma unroll
-        for (int o = 4; o >= 1; o >>= 1) {
+        for (int o = SC_LPR / 2; o >= 1; o >>= 1) {
             a += __shfl_xor_sync(FULL, a, o);
             m += __shfl_xor_sync(FULL, m, o);
         }
         const float sc = a * p.inv_sqrt_d;
         // |exact score - sc| <= 2^-8 m / sqrt(d) (see LP_REL_BOUND)
         const float err = fmaf(LP_REL_BOUND, m * p.inv_sqrt_d, LP_ABS_BOUND);
-        const int c = row0 + 4 * j + oct;
-        const int w = __shfl_sync(FULL, wc, 4 * j + oct);
+        const int c = row0 + GR * j + oct;
+        const int w = __shfl_sync(FULL, wc, GR * j + oct);
         if (l8 == 0 && c < C) {
             p.scores[(size_t)u * p.Cmax + c] = sc + err;
             if (w > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), w);
