@@ -192,11 +192,29 @@ class RowCounter:
         return self.map[: self.dummy].sum(dtype=torch.long)
 
 
-def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
-    from graph_community_sparse_b200.layer import LayerState
+class BenchLayer:
+    """One layer of the step: its cache, graph state, labels and the per-step
+    queries and new tokens (seeded by the layer index)."""
 
+    def __init__(self, wl: synth.Workload, seed_layer: int, device, T_cap: int, max_tail: int, n_total: int):
+        from graph_community_sparse_b200.layer import LayerState
+
+        draw = synth.draw_cache(wl, layer=seed_layer, device=device, T_cap=T_cap)
+        C = int(draw.labels.max()) + 1
+        self.st = LayerState(draw.K, draw.V, wl.Hq, wl.mode, wl.S, C, max_tail)
+        self.labels = torch.from_numpy(draw.labels.reshape(self.st.U, wl.T).astype(np.int32)).to(device)
+        self.qs = [synth.draw_queries(wl, draw, i, seed_layer) for i in range(n_total)]
+        self.news = ([synth.draw_new_tokens(wl, draw, i, seed_layer) for i in range(n_total)]
+                     if wl.update else [])
+
+    def build(self, T: int) -> None:
+        self.st.build(self.labels, T)
+
+
+def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     K_steps, W_steps = args.steps, args.warmup
     budget = args.budget if args.budget is not None else wl.budget
+    n_layers = args.layers if args.layers is not None else wl.layers
     B_steps = min(K_steps, 100)
     n_total = W_steps + K_steps + B_steps + args.e2e_steps
     # Update workloads run in episodes of the workload's own length (e.g. 64
@@ -205,28 +223,29 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     episode = wl.steps if wl.update else 0
     extra = episode + 8 if wl.update else 0
     T_cap = wl.T + extra
-    layer = rank  # per-rank seeds: each rank owns a different batch of sequences
-    draw = synth.draw_cache(wl, layer=layer, device=device, T_cap=T_cap)
-    C = int(draw.labels.max()) + 1
-    st = LayerState(draw.K, draw.V, wl.Hq, wl.mode, wl.S, C, max(extra, 1))
-    U = st.U
-    labels = torch.from_numpy(draw.labels.reshape(U, wl.T).astype(np.int32)).to(device)
+    # per-rank seeds: each rank owns a different batch of sequences
+    layers = [BenchLayer(wl, rank * n_layers + l, device, T_cap, max(extra, 1), n_total) for l in range(n_layers)]
+    st0 = layers[0].st
+    U = st0.U
     torch.cuda.synchronize()
     b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     b0.record()
-    st.build(labels, wl.T)
+    for L in layers:
+        L.build(wl.T)
     b1.record()
     torch.cuda.synchronize()
     build_ms = b0.elapsed_time(b1)
-    if int(st.graph.dev_err.item()) != 0:
-        raise RuntimeError(f"build reported device error {int(st.graph.dev_err.item())}")
 
-    qs = [synth.draw_queries(wl, draw, i, layer) for i in range(n_total)]
-    news = [synth.draw_new_tokens(wl, draw, i, layer) for i in range(n_total)] if wl.update else []
+    def check_dev_err(what: str):
+        for li, L in enumerate(layers):
+            err = int(L.st.graph.dev_err.item())
+            if err != 0:
+                raise RuntimeError(f"{what}: layer {li} reported device error {err}")
+
+    check_dev_err("build")
     # 1 GiB > L2; its ~0.3 ms on the GPU also lets the host enqueue a whole step
     # before the GPU reaches it, so the events time device work, not launch gaps
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.float32, device=device)
-
     # then reading another 512 MiB leaves L2 clean: the dirty lines of the
     # write are written back here, not charged to the step's first kernel
     clean_buf = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device=device)
@@ -239,36 +258,39 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     esz = 2 if wl.dtype == "bf16" else 4
     row_bytes = 2 * wl.d * esz
     per_head = wl.mode == "head"
-    num_comm = st.graph.num_comm.long()
     episodes = [0]
 
     def new_episode_if_due():
-        if wl.update and st.T - wl.T >= episode:
-            st.build(labels, wl.T)
+        if wl.update and st0.T - wl.T >= episode:
+            for L in layers:
+                L.build(wl.T)
             episodes[0] += 1
 
     def one_step(i, ev=None, per_call=False):
-        """ev: [start, end] events, or [start, after selection, end] with
-        per_call (events between the calls break the programmatic-launch
-        chain from the selection into the attention, so the timed steps do
-        not use them)."""
-        q = qs[i]
+        """ev: [start, end] events, or with per_call [start, then after each
+        layer's selection and after its attention]: events between the calls
+        break the programmatic-launch chain from the selection into the
+        attention, so the timed steps do not use them."""
         if ev:
             ev[0].record()
-        st.select(q, budget)
-        if ev and per_call:
-            ev[1].record()
-        if wl.update:
-            k, v = news[i]
-            st.attend_append(q, k, v)
-        else:
-            st.attend(q, want_nbr=False)
-        if ev:
+        for li, L in enumerate(layers):
+            q = L.qs[i]
+            L.st.select(q, budget)
+            if ev and per_call:
+                ev[1 + 2 * li].record()
+            if wl.update:
+                k, v = L.news[i]
+                L.st.attend_append(q, k, v)
+            else:
+                L.st.attend(q, want_nbr=False)
+            if ev and per_call:
+                ev[2 + 2 * li].record()
+        if ev and not per_call:
             ev[-1].record()
 
     # a selection never holds more than S + max(budget, largest community) tokens
-    max_cnt = int(st.graph.cnt.max().item()) + extra
-    cap = min(st.sel.sel_tok.shape[1], wl.S + max(budget, max_cnt))
+    max_cnt = max(int(L.st.graph.cnt.max().item()) for L in layers) + extra
+    cap = min(st0.sel.sel_tok.shape[1], wl.S + max(budget, max_cnt))
     count_rows = RowCounter(wl, U, T_cap, cap, device)
     clock_sampler = ClockSampler(device.index).__enter__()
     time.sleep(0.5)  # let the sampler start before the warm-up
@@ -301,35 +323,38 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     max_total_s = reduce_max(total_s, device)
 
     # per-call breakdown (for the roofline), in its own pass of steps right
-    # after the timed ones, with an event between the two calls
-    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(B_steps)]
-    rows_hist, ntok_hist, nsel_hist, ncomm_hist = [], [], [], []
+    # after the timed ones, with an event between the calls
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(1 + 2 * n_layers)] for _ in range(B_steps)]
+    rows_hist, ntok_hist, nsel_hist = [], [], []
     for j in range(B_steps):
         new_episode_if_due()
         flush()
         one_step(W_steps + K_steps + j, bevs[j], per_call=True)
-        rows_hist.append(count_rows(st.sel))
-        ntok_hist.append(st.sel.n_tok.long().sum())
-        nsel_hist.append(st.sel.n_sel.long().sum())
-        ncomm_hist.append(num_comm.sum())
+        rows_hist.append(sum(count_rows(L.st.sel) for L in layers))
+        ntok_hist.append(sum(L.st.sel.n_tok.long().sum() for L in layers))
+        nsel_hist.append(sum(L.st.sel.n_sel.long().sum() for L in layers))
     torch.cuda.synchronize()
-    if int(st.graph.dev_err.item()) != 0:
-        raise RuntimeError(f"device error word {int(st.graph.dev_err.item())}")
-    sel_ms = [e[0].elapsed_time(e[1]) for e in bevs]
-    dec_ms = [e[1].elapsed_time(e[2]) for e in bevs]
+    check_dev_err("timed steps")
+    # per step, summed over the layers: each selection from the previous
+    # layer's attention end (or the step start), each attention from its
+    # selection end
+    sel_ms = [sum((e[0] if li == 0 else e[2 * li]).elapsed_time(e[1 + 2 * li]) for li in range(n_layers))
+              for e in bevs]
+    dec_ms = [sum(e[1 + 2 * li].elapsed_time(e[2 + 2 * li]) for li in range(n_layers)) for e in bevs]
 
     rows = np.array([int(r.item()) for r in rows_hist], dtype=np.float64)
     ntok = np.array([int(r.item()) for r in ntok_hist], dtype=np.float64)
     nsel = np.array([int(r.item()) for r in nsel_hist], dtype=np.float64)
-    ncomm = float(ncomm_hist[0].item())
-    q_bytes = wl.B * wl.Hq * wl.d * esz
-    out_bytes = wl.B * wl.Hq * wl.d * 4
+    ncomm = float(sum(int(L.st.graph.num_comm.long().sum().item()) for L in layers))
+    q_bytes = n_layers * wl.B * wl.Hq * wl.d * esz
+    out_bytes = n_layers * wl.B * wl.Hq * wl.d * 4
     dec_bytes = rows * row_bytes + ntok * 4 + q_bytes + out_bytes
     if wl.update:
         # neighbours, the logit of every list entry (written and read back),
         # up to 8 candidate centres read per unit, one centre row updated,
         # and the new K/V rows copied into the cache
-        dec_bytes = dec_bytes + ntok * 8 + U * (8 * 4 + 8 * wl.d * 4 + 2 * wl.d * 4) + 4 * wl.B * wl.Hkv * wl.d * esz
+        dec_bytes = dec_bytes + ntok * 8 + n_layers * (U * (8 * 4 + 8 * wl.d * 4 + 2 * wl.d * 4)
+                                                       + 4 * wl.B * wl.Hkv * wl.d * esz)
     # the scoring pass reads every centre in bf16; the selected communities
     # (at least) are re-scored from the fp32 centres; per community a size is
     # read and a score bound written and read back; the token list is written
@@ -341,6 +366,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
 
     dec_gbs = gbs(dec_bytes, dec_ms)
     sel_gbs = gbs(sel_bytes, sel_ms)
+    per = f" (sum over {n_layers} layers)" if n_layers > 1 else ""
     kernels = {
         "ckv_score_select": {"ms": float(np.mean(sel_ms)), "bytes": float(np.mean(sel_bytes)), "GB/s": sel_gbs,
                              "frac": sel_gbs / peak},
@@ -352,65 +378,73 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     dom = max((dec_name, "ckv_score_select"), key=lambda k: kernels[k]["ms"])
     roofline = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": peak, "unit": "GB/s",
                 "frac": kernels[dom]["GB/s"] / peak, "peak_source": peak_src,
-                "traffic": profile_traffic(dom, wl.key), "bytes_per_launch": kernels[dom]["bytes"],
+                "traffic": profile_traffic(dom, wl.key) if n_layers == 1 else None,
+                "bytes_per_launch": kernels[dom]["bytes"] / n_layers,
                 "timing": "CUDA events around the library call on its stream, mean over a pass of "
-                          f"{B_steps} steps right after the timed ones (the timed steps carry no events "
-                          "between calls, which would break the programmatic-launch chain)"}
+                          f"{B_steps} steps right after the timed ones{per} (the timed steps carry no "
+                          "events between calls, which would break the programmatic-launch chain)"}
 
-    # dense comparator on the same cache and queries
-    dense_out = torch.empty_like(st.out)
+    # dense comparator on the same caches and queries
+    dense_out = torch.empty_like(st0.out)
     dms = []
     for j in range(max(3, min(K_steps, 10)) + 2):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        st.dense(qs[j % len(qs)], dense_out)
+        for L in layers:
+            L.st.dense(L.qs[j % len(L.qs)], dense_out)
         e1.record()
         dms.append((e0, e1))
     torch.cuda.synchronize()
     dms = [a.elapsed_time(b) for a, b in dms[2:]]
-    dense_bytes = wl.B * wl.Hkv * st.T * row_bytes + q_bytes + out_bytes
+    dense_bytes = n_layers * wl.B * wl.Hkv * st0.T * row_bytes + q_bytes + out_bytes
     dense_gbs = dense_bytes / (np.mean(dms) * 1e-3) / 1e9
     dense = {"ms": float(np.mean(dms)), "bytes": float(dense_bytes), "GB/s": float(dense_gbs),
-             "frac": float(dense_gbs / peak), "T": st.T,
+             "frac": float(dense_gbs / peak), "T": st0.T,
              "sparse_step_speedup": float(np.mean(dms) / np.mean(step_ms))}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: every layer's q
+    # (and new K/V rows) in from pinned memory, its outputs back
     e2e = None
     if args.e2e_steps > 0:
         pin = dict(pin_memory=True)
-        q_host = [qs[i].cpu().pin_memory() for i in range(n_total)]
-        kv_host = [(k.cpu().pin_memory(), v.cpu().pin_memory()) for k, v in news] if wl.update else []
-        q_dev = torch.empty_like(qs[0])
-        k_dev = torch.empty_like(news[0][0]) if wl.update else None
-        v_dev = torch.empty_like(news[0][1]) if wl.update else None
-        out_h = torch.empty(st.out.shape, dtype=torch.float32, **pin)
-        nbr_h = torch.empty(st.nbr8.shape, dtype=torch.int32, **pin)
-        asg_h = torch.empty(st.assigned.shape, dtype=torch.int32, **pin)
-        e_ms = []
-        h2d = q_host[0].numel() * q_host[0].element_size()
+        io = []
+        for L in layers:
+            io.append(dict(
+                q_host=[L.qs[i].cpu().pin_memory() for i in range(n_total)],
+                kv_host=[(k.cpu().pin_memory(), v.cpu().pin_memory()) for k, v in L.news] if wl.update else [],
+                q_dev=torch.empty_like(L.qs[0]),
+                k_dev=torch.empty_like(L.news[0][0]) if wl.update else None,
+                v_dev=torch.empty_like(L.news[0][1]) if wl.update else None,
+                out_h=torch.empty(L.st.out.shape, dtype=torch.float32, **pin),
+                nbr_h=torch.empty(L.st.nbr8.shape, dtype=torch.int32, **pin),
+                asg_h=torch.empty(L.st.assigned.shape, dtype=torch.int32, **pin)))
+        h2d = n_layers * io[0]["q_dev"].numel() * io[0]["q_dev"].element_size()
         if wl.update:
-            h2d += 2 * kv_host[0][0].numel() * kv_host[0][0].element_size()
-        d2h = out_h.numel() * 4 + (nbr_h.numel() * 4 + asg_h.numel() * 4 if wl.update else 0)
+            h2d += n_layers * 2 * io[0]["k_dev"].numel() * io[0]["k_dev"].element_size()
+        d2h = n_layers * (io[0]["out_h"].numel() * 4
+                          + ((io[0]["nbr_h"].numel() + io[0]["asg_h"].numel()) * 4 if wl.update else 0))
+        e_ms = []
         for j in range(args.e2e_steps):
             i = W_steps + K_steps + B_steps + j
             new_episode_if_due()
             flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            q_dev.copy_(q_host[i], non_blocking=True)
-            if wl.update:
-                k_dev.copy_(kv_host[i][0], non_blocking=True)
-                v_dev.copy_(kv_host[i][1], non_blocking=True)
-            st.select(q_dev, budget)
-            if wl.update:
-                st.attend_append(q_dev, k_dev, v_dev)
-            else:
-                st.attend(q_dev, want_nbr=False)
-            out_h.copy_(st.out, non_blocking=True)
-            if wl.update:
-                nbr_h.copy_(st.nbr8, non_blocking=True)
-                asg_h.copy_(st.assigned, non_blocking=True)
+            for L, b in zip(layers, io):
+                b["q_dev"].copy_(b["q_host"][i], non_blocking=True)
+                if wl.update:
+                    b["k_dev"].copy_(b["kv_host"][i][0], non_blocking=True)
+                    b["v_dev"].copy_(b["kv_host"][i][1], non_blocking=True)
+                L.st.select(b["q_dev"], budget)
+                if wl.update:
+                    L.st.attend_append(b["q_dev"], b["k_dev"], b["v_dev"])
+                else:
+                    L.st.attend(b["q_dev"], want_nbr=False)
+                b["out_h"].copy_(L.st.out, non_blocking=True)
+                if wl.update:
+                    b["nbr_h"].copy_(L.st.nbr8, non_blocking=True)
+                    b["asg_h"].copy_(L.st.assigned, non_blocking=True)
             e1.record()
             e_ms.append((e0, e1))
         torch.cuda.synchronize()
@@ -425,9 +459,9 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": n_ranks, "steps": K_steps,
         "warmup": W_steps, "ms_per_step": max_total_s * 1e3 / K_steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.key, "title": wl.title, "B_per_gpu": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv,
-                   "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
-                   "communities_per_graph": float(ncomm / U), "budget": budget, "sinks": wl.S,
+        "config": {"workload": wl.key, "title": wl.title, "B_per_gpu": wl.B, "layers": n_layers, "Hq": wl.Hq,
+                   "Hkv": wl.Hkv, "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
+                   "communities_per_graph": float(ncomm / (U * n_layers)), "budget": budget, "sinks": wl.S,
                    "update": wl.update, "layout": wl.layout,
                    "l2": "flushed by a 1 GiB write then a 512 MiB read before every timed step, outside the CUDA events",
                    "parallelism": f"dp{n_ranks} (independent batches, no collective)"},
@@ -436,7 +470,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "kernels": kernels,
         "dense": dense,
         "e2e": e2e,
-        "gpu_launches": K_steps * (KERNELS_PER_STEP_UPDATE if wl.update else KERNELS_PER_STEP_STATIC),
+        "gpu_launches": K_steps * n_layers * (KERNELS_PER_STEP_UPDATE if wl.update else KERNELS_PER_STEP_STATIC),
         "clocks": clocks,
         "build_ms": build_ms,
         "wall_s_timed_region": wall,
@@ -496,14 +530,15 @@ def sample_units(wl: synth.Workload, n: int, seed: int):
     return [allu[i] for i in sorted(idx)]
 
 
-def cpu_baseline(wl: synth.Workload, budget: int, device, n_units: int) -> dict:
+def cpu_baseline(wl: synth.Workload, budget: int, device, n_units: int, n_layers: int = 1) -> dict:
     draw = synth.draw_cache(wl, device=device)
     units = sample_units(wl, n_units, 1)
     t = oracle_unit_seconds(wl, draw, units, budget, 0)
-    per_step = t / len(units) * (wl.B * wl.G)
+    per_step = t / len(units) * (wl.B * wl.G) * n_layers
     del draw
+    lay = f" x {n_layers} layers" if n_layers > 1 else ""
     return {"value": 1.0 / per_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
-            "sample": f"{len(units)} of {wl.B * wl.G} graph units of one decode step "
+            "sample": f"{len(units)} of {wl.B * wl.G} graph units of one decode step{lay} "
                       f"({t:.1f} s single-threaded float64 numpy), scaled to the whole step"}
 
 
@@ -538,6 +573,8 @@ def parse(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--batch", type=int, default=None, help="override the batch (small profiling captures)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layers per step (default: the workload's; each has its own cache and graphs)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-units", type=int, default=48, help="graph units the CPU baseline times")
@@ -574,7 +611,8 @@ def main(argv=None):
         res = run_cuda(args, wl, rank, ws, device)
         if rank == 0 and ws == 1 and not args.no_cpu_baseline:
             torch.cuda.empty_cache()
-            res["cpu_baseline"] = cpu_baseline(wl, res["config"]["budget"], device, args.cpu_units)
+            res["cpu_baseline"] = cpu_baseline(wl, res["config"]["budget"], device, args.cpu_units,
+                                               res["config"]["layers"])
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
