@@ -80,10 +80,25 @@ struct RowGeom {
     static constexpr int TILE = TOK_PER_IT * ROW;
 };
 
+// bf16 caches whose graphs serve several query heads use the tensor-core
+// segment loop (ckv_decode_mma.cuh); the others the scalar one below.
+template <typename T, int GQ>
+struct UseMma {
+    static constexpr bool v = std::is_same<T, __nv_bfloat16>::value && GQ >= 2;
+};
+template <typename T, int GQ>
+struct DecMinBlocks {
+    static constexpr int v = UseMma<T, GQ>::v ? 2 : MinBlocks<GQ>::v;
+};
+template <int D>
+struct MmaGeom;
+
 template <typename T, int D, int GQ>
 struct DecSmem {
     static constexpr int PBUF = TOK_PER_IT * GQ * 4;
-    static constexpr int WARP = Stages<GQ>::v * 2 * RowGeom<T, D>::TILE + ((PBUF + 127) / 128) * 128;
+    static constexpr int SCALAR = Stages<GQ>::v * 2 * RowGeom<T, D>::TILE + ((PBUF + 127) / 128) * 128;
+    static constexpr int MMA = 3 * 2 * 16 * D * 2;  // MMA_STAGES x (K, V) x MMA_TOK rows of bf16
+    static constexpr int WARP = UseMma<T, GQ>::v ? MMA : SCALAR;
     static constexpr int CTA_FIXED = DEC_WARPS * WARP;
 };
 
@@ -131,6 +146,8 @@ __device__ __forceinline__ float exp2_approx(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+
+#include "ckv_decode_mma.cuh"
 
 // One warp, one unit, list positions [lo, hi) of the unit's selection (or
 // cache positions, dense).  Full iterations (all 8 tokens valid, past the
@@ -340,7 +357,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 }
 
 template <typename T, int D, int GQ, bool DENSE>
-__global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(DecodeParams p) {
+__global__ void __launch_bounds__(DEC_WARPS * 32, DecMinBlocks<T, GQ>::v) decode_main(DecodeParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     pdl_wait();  // the selection comes from the kernel before
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -398,7 +415,12 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, MinBlocks<GQ>::v) decode_main(
             const int ubeg = DENSE ? u * p.T : s_pre[u];
             const int uend = DENSE ? ubeg + p.T : s_pre[u + 1];
             const int lo = max(start, ubeg), hi = min(end, uend);
-            if (lo < hi) process_segment<T, D, GQ, DENSE>(p, u, lo - ubeg, hi - ubeg, sbase + u, wsm, lane);
+            if (lo < hi) {
+                if constexpr (UseMma<T, GQ>::v)
+                    process_segment_mma<D, GQ, DENSE>(p, u, lo - ubeg, hi - ubeg, sbase + u, wsm, lane);
+                else
+                    process_segment<T, D, GQ, DENSE>(p, u, lo - ubeg, hi - ubeg, sbase + u, wsm, lane);
+            }
             if (end <= uend || u + 1 >= p.U) break;
             ++u;
         }

@@ -36,6 +36,8 @@ SHAPES = [
     small("f32_d64_head", 25, dtype="f32", d=64, mode="head", Hq=8, Hkv=4),
     small("bf16_zipf", 26, sizes="zipf", T=6000, budgets=(700,), update=False),
     small("bf16_spans", 27, layout="spans"),
+    small("bf16_d128_gq8", 28, Hq=32, Hkv=4),
+    small("bf16_d64_gq4_head", 29, d=64, mode="head", Hq=16, Hkv=4, budgets=(150,)),
 ]
 
 
