@@ -45,6 +45,7 @@ constexpr int DEC_WARPS = 4;
 // atomic ticket, so warps on SMs that run faster (the SMs of a GPC share its
 // memory bandwidth unevenly) take more of it and all warps end together.
 constexpr int DYN_DEN = 8;
+constexpr int MIN_WARP_TOKENS = 64;
 constexpr int DYN_CHUNK_MIN = 64;
 constexpr int NCH_MAX = 4096;
 
@@ -63,7 +64,9 @@ __host__ __device__ __forceinline__ DynSplit dyn_split(int total, int W, bool de
     d.chk = max(DYN_CHUNK_MIN, (dyn + NCH_MAX - 1) / NCH_MAX);
     d.nch = (dyn + d.chk - 1) / d.chk;
     d.R = total - dyn;
-    d.per_s = max(1, (d.R + W - 1) / W);
+    // at least MIN_WARP_TOKENS per warp: small problems use fewer warps, so
+    // each unit has fewer partials to merge
+    d.per_s = max(MIN_WARP_TOKENS, (d.R + W - 1) / W);
     return d;
 }
 constexpr int TOK_PER_IT = 8;
