@@ -34,6 +34,7 @@
 // The histograms live in the workspace head: zero on entry, and each
 // selection block clears its unit's histogram after reading it.
 #include <math.h>
+#include <type_traits>
 
 #include "ckv_internal.cuh"
 
@@ -226,10 +227,98 @@ __device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int
     }
 }
 
+// Several query heads per graph with a bf16 q: both products on the tensor
+// cores (mma.sync m16n8k16), heads as the A rows (padded with zeros), eight
+// communities per n-tile as the B columns, loaded straight from global
+// memory in fragment order: S = Q C~^T and the bound's M = |Q| |C~|^T, whose
+// operands are the same registers with the sign bits cleared.  A warp takes
+// two n-tiles (16 communities); the 4 lanes of quad 0 then hold, per
+// community, the max over the group's heads of both.
+__device__ __forceinline__ void mma_sc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(0u), "r"(a1), "r"(0u), "r"(b0), "r"(b1));
+}
+
+template <int D, int GQ>
+__device__ __forceinline__ void score_rows_mma(const SelectParams& p, int u, int C) {
+    constexpr int KS = D / 16;
+    constexpr int RW = SCORE_ROWS / SEL_WARPS;  // 16 communities per warp
+    static_assert(RW == 16, "two n-tiles of 8 per warp");
+    constexpr uint32_t ABS = 0x7fff7fffu;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, tq = lane & 3;
+    const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
+    if (row0 >= C) return;
+    // B fragments of both n-tiles: community row0 + 8t + g, dims kk*16 + 2tq (+8)
+    uint32_t bf[2][KS][2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int c = row0 + 8 * t + g;
+        const __nv_bfloat16* row = p.cent_lp + ((size_t)u * p.Cmax + min(c, C - 1)) * D + 2 * tq;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const uint32_t x0 = *reinterpret_cast<const uint32_t*>(row + kk * 16);
+            const uint32_t x1 = *reinterpret_cast<const uint32_t*>(row + kk * 16 + 8);
+            bf[t][kk][0] = c < C ? x0 : 0u;
+            bf[t][kk][1] = c < C ? x1 : 0u;
+        }
+    }
+    const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
+    const int b = u / p.G, gg = u - b * p.G;
+    const int h0 = gg * GQ;  // per-group graphs (several heads)
+    uint32_t qa[KS][2];
+    {
+        const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + h0 + min(g, GQ - 1)) * D + 2 * tq;
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            const uint32_t x0 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16);
+            const uint32_t x1 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8);
+            qa[kk][0] = g < GQ ? x0 : 0u;
+            qa[kk][1] = g < GQ ? x1 : 0u;
+        }
+    }
+    int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, macc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            mma_sc(sacc, qa[kk][0], qa[kk][1], bf[t][kk][0], bf[t][kk][1]);
+            mma_sc(macc, qa[kk][0] & ABS, qa[kk][1] & ABS, bf[t][kk][0] & ABS, bf[t][kk][1] & ABS);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            // max over the group's heads (rows g < GQ)
+            float sv = g < GQ ? sacc[e] : -INFINITY, mv = g < GQ ? macc[e] : 0.f;
+#pragma unroll
+            for (int o = 4; o <= 16; o <<= 1) {
+                sv = fmaxf(sv, __shfl_xor_sync(FULL, sv, o));
+                mv = fmaxf(mv, __shfl_xor_sync(FULL, mv, o));
+            }
+            const int r = 8 * t + 2 * tq + e;  // community row within the warp's 16
+            const int w = __shfl_sync(FULL, wc, r);
+            const float sc = sv * p.inv_sqrt_d;
+            const float err = fmaf(LP_REL_BOUND, mv * p.inv_sqrt_d, LP_ABS_BOUND);
+            const int c = row0 + r;
+            if (g == 0 && c < C) {
+                p.scores[(size_t)u * p.Cmax + c] = sc + err;
+                if (w > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), w);
+            }
+        }
+    }
+}
+
 template <typename T, int D, int GQ>
 __device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) {
     if constexpr (GQ == 1) {
         score_rows_gq1<T, D>(p, u, C);
+        return;
+    }
+    if constexpr (GQ > 1 && std::is_same<T, __nv_bfloat16>::value) {
+        score_rows_mma<D, GQ>(p, u, C);
         return;
     }
     constexpr int E = D / 16;
