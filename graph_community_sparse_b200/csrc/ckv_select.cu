@@ -384,6 +384,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     __shared__ unsigned long long s_runs[SEL_FAST];
     __shared__ int s_bsz[SEL_FAST];
     __shared__ int s_ofs[SEL_FAST];
+    __shared__ int s_len[SEL_FAST];  // candidate i's build-time run length
     __shared__ unsigned s_mask[MAX_CMAX / 32];
     __shared__ int s_warp[33];
     __shared__ int s_bstar, s_nc, s_nt, s_cnt;
@@ -549,6 +550,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     }
     if (nc <= SEL_FAST) {
         rescore(s_key, nc);
+        if (tid < nc) s_len[tid] = o1 - o0;
         __syncthreads();
     }
 
@@ -566,15 +568,18 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         if (tid < nc) {
             const unsigned long long k = s_key[tid];
             const int w = s_w[tid];
-            int rank = 0, above = 0;
+            // rank, the size ranked above (for the cut) and the run length
+            // ranked above (the run's place in the token list)
+            int rank = 0, above = 0, above_len = 0;
             for (int j = 0; j < nc; ++j) {
                 const bool gt = s_key[j] > k;
                 rank += gt;
                 above += gt ? s_w[j] : 0;
+                above_len += gt ? s_len[j] : 0;
             }
             in = above + w <= p.budget;
             s_runs[rank] = k;
-            s_bsz[rank] = o1 - o0;
+            s_bsz[rank] = above_len + (o1 - o0);  // inclusive prefix in rank order
             s_ofs[rank] = o0;
             if (in || rank == 0) {
                 // the token copy reads this run next: start fetching it into L2
@@ -637,7 +642,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         }
     }
 
-    // 4. ranked ids and membership mask; inclusive prefix of the run sizes
+    // 4. ranked ids and membership mask
     int32_t* selc = p.sel_comm + (size_t)u * p.Cmax;
     for (int i = tid; i < kstar; i += nt) {
         const int c = key_id(sorted[i]);
@@ -645,7 +650,9 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         atomicOr(&s_mask[c >> 5], 1u << (c & 31));
     }
     __syncthreads();
-    const int nb = block_scan_inplace(bsz, kstar, s_warp);  // inclusive
+    // tokens of the selected runs; their inclusive prefix (the small path
+    // ranked it already)
+    const int nb = small ? (kstar > 0 ? s_bsz[kstar - 1] : 0) : block_scan_inplace(bsz, kstar, s_warp);
 
     int32_t* out = p.sel_tok + (size_t)u * p.tok_cap;
     const int32_t* tk = p.tok + (size_t)u * p.T_cap;
