@@ -42,7 +42,9 @@ namespace ckv {
 
 constexpr int SEL_WARPS = 8;
 constexpr int SEL_THREADS = SEL_WARPS * 32;
-constexpr int SCORE_ROWS = SEL_WARPS * 16;  // centres per block
+constexpr int SCORE_ROWS = SEL_WARPS * 16;      // centres per block (several heads per graph)
+constexpr int SCORE_ROWS_GQ1 = SEL_WARPS * 16;  // centres per block (one head per graph)
+template <int GQ> struct ScoreBlockRows { static constexpr int v = GQ == 1 ? SCORE_ROWS_GQ1 : SCORE_ROWS; };
 constexpr int SEL_HBITS = HIST_BITS;
 constexpr int SEL_HBINS = HIST_BINS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
@@ -178,11 +180,11 @@ template <typename T, int D>
 __device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int C) {
     constexpr int E = D / SC_LPR;
     constexpr int GR = 32 / SC_LPR;             // rows per warp instruction
-    constexpr int RW = SCORE_ROWS / SEL_WARPS;  // rows per warp
+    constexpr int RW = SCORE_ROWS_GQ1 / SEL_WARPS;  // rows per warp
     constexpr int RQ = RW / GR;                 // rows per lane group
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int oct = lane / SC_LPR, l8 = lane % SC_LPR;
-    const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
+    const int row0 = blockIdx.x * SCORE_ROWS_GQ1 + warp * RW;
     if (row0 >= C) return;
     RawPart<E> raw[RQ];
 #pragma unroll
@@ -790,7 +792,8 @@ SelWs sel_ws_layout(int U, int Cmax) {
 
 template <typename T, int D, int GQ>
 cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
-    dim3 grid((p.Cmax + SCORE_ROWS - 1) / SCORE_ROWS, p.U);
+    constexpr int rows = ScoreBlockRows<GQ>::v;
+    dim3 grid((p.Cmax + rows - 1) / rows, p.U);
     cudaError_t e = launch_pdl(score_kernel<T, D, GQ>, grid, dim3(SEL_THREADS), 0, st, p);
     if (e != cudaSuccess) return e;
     return launch_pdl(select_kernel<T, D, GQ>, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
