@@ -192,6 +192,28 @@ def assign(k_new: np.ndarray, cent: np.ndarray, candidates: Sequence[int]) -> in
     return best
 
 
+def assign_vote(k_new: np.ndarray, cent: np.ndarray, neighbour_comms: Sequence[int]) -> int:
+    """Step 6, second half, the alternative "graph-like" rule (the pages say
+    only that the token joins a suitable neighbouring community): the
+    community holding the most of the 8 neighbours wins; among equally
+    frequent ones the larger k_new . cent_c / sqrt(d), then the lower id;
+    -1 without candidates.  neighbour_comms lists each neighbour's community
+    (repeats count)."""
+    k_new = np.asarray(k_new, dtype=np.float64)
+    votes = {}
+    for c in neighbour_comms:
+        c = int(c)
+        if c >= 0:
+            votes[c] = votes.get(c, 0) + 1
+    best, best_key = -1, None
+    for c in sorted(votes):
+        s = float(np.dot(k_new, cent[c])) / math.sqrt(k_new.shape[0])
+        key = (votes[c], s)
+        if best < 0 or key > best_key:
+            best, best_key = c, key
+    return best
+
+
 # ----------------------------------------------------------------------------
 # a whole decode step over a batch
 # ----------------------------------------------------------------------------

@@ -230,6 +230,36 @@ def test_assign_bruteforce_ties_and_one_update():
     assert O.assign(np.ones(d), np.ones((C, d)), []) == -1
 
 
+def test_assign_vote_worked_examples_and_bruteforce():
+    """The majority-vote rule: most frequent neighbour community, then the
+    larger score, then the lower id."""
+    d = 4
+    cent = np.array([[1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0], [2, 0, 0, 0]], dtype=np.float64)
+    k = np.array([1.0, 0.5, 0.0, 0.0])
+    # worked by hand: votes {2: 3, 0: 2, 1: 2} -> 2 wins although its score (0) is the lowest
+    assert O.assign_vote(k, cent, [2, 0, 2, 1, 0, 2, 1, -1]) == 2
+    # equal votes {0: 2, 3: 2}: scores 1/2 and 2/2 -> 3; the score rule would also pick 3
+    assert O.assign_vote(k, cent, [0, 3, 0, 3]) == 3
+    # equal votes and equal scores (cent[1] = cent[2] seen from k2) -> the lower id
+    k2 = np.array([0.0, 1.0, 1.0, 0.0])
+    assert O.assign_vote(k2, cent, [2, 1]) == 1
+    assert O.assign_vote(k, cent, [-1, -1]) == -1 and O.assign_vote(k, cent, []) == -1
+    rng = np.random.default_rng(23)
+    C = 6
+    for _ in range(200):
+        cent = rng.integers(-2, 3, (C, d)).astype(np.float64)
+        k = rng.integers(-2, 3, d).astype(np.float64)
+        nb = list(rng.integers(-1, C, size=8))
+        got = O.assign_vote(k, cent, nb)
+        valid = [c for c in nb if c >= 0]
+        if not valid:
+            assert got == -1
+            continue
+        # brute force: enumerate the communities, compare (votes, score, -id)
+        best = max(set(valid), key=lambda c: (valid.count(c), float(np.dot(k, cent[c])), -c))
+        assert got == best
+
+
 def test_multi_step_invariants_on_tiny_workload():
     """Tiny workload, all steps: sinks present, no duplicate positions, the
     top community always selected, exactly one count changes per graph and
