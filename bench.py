@@ -93,17 +93,28 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def csrc_digest() -> str:
+    """sha256 over every CUDA source and header of the library (names and
+    contents, in name order): any kernel change alters it."""
+    d = os.path.join(ROOT, "graph_community_sparse_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode() + b"\0" + open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()
+
+
 def profile_traffic(kernel: str, workload: str):
     """DRAM bytes per launch recorded by the committed ncu summary for this
-    kernel and workload, valid only while the kernel source is unchanged."""
+    kernel and workload, valid only while no kernel source has changed since
+    the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     try:
         d = json.load(open(path))
         ent = d[kernel][workload]
-        src = os.path.join(ROOT, "graph_community_sparse_b200", "csrc", ent["source"])
-        if hashlib.sha256(open(src, "rb").read()).hexdigest() != ent["sha256"]:
+        if ent["csrc_sha256"] != csrc_digest():
             return None
         return float(ent["bytes_per_launch"])
     except Exception:
@@ -201,7 +212,7 @@ class BenchLayer:
 
         draw = synth.draw_cache(wl, layer=seed_layer, device=device, T_cap=T_cap)
         C = int(draw.labels.max()) + 1
-        self.st = LayerState(draw.K, draw.V, wl.Hq, wl.mode, wl.S, C, max_tail)
+        self.st = LayerState(draw.K, draw.V, wl.Hq, wl.mode, wl.S, C, max_tail, rule=wl.assign_rule)
         self.labels = torch.from_numpy(draw.labels.reshape(self.st.U, wl.T).astype(np.int32)).to(device)
         self.qs = [synth.draw_queries(wl, draw, i, seed_layer) for i in range(n_total)]
         self.news = ([synth.draw_new_tokens(wl, draw, i, seed_layer) for i in range(n_total)]
@@ -209,6 +220,39 @@ class BenchLayer:
 
     def build(self, T: int) -> None:
         self.st.build(self.labels, T)
+
+
+@torch.no_grad()
+def assignment_drift(layers, wl: synth.Workload, T0: int, n_members: int = 1024) -> dict:
+    """How well the running-mean centres still describe their members: the
+    mean of |k - c| / |k| over the tokens joined since the last build (k the
+    token's key, c its community's current centre), beside the same quantity
+    over a sample of build-time members.  A diagnostic read after the timed
+    steps, not part of the step."""
+    tail, mem = [], []
+    for L in layers:
+        st, gr = L.st, L.st.graph
+        dev = st.K.device
+        u = torch.arange(st.U, device=dev)
+        b, g = u // wl.G, u % wl.G
+        kvh = g // (wl.Hq // wl.Hkv) if wl.mode == "head" else g
+        rng = torch.Generator(device="cpu").manual_seed(7)
+        sample = wl.S + torch.randperm(T0 - wl.S, generator=rng)[:n_members].to(dev)
+        for pos, acc in ((torch.arange(T0, st.T, device=dev), tail), (sample, mem)):
+            if pos.numel() == 0:
+                continue
+            comm = gr.comm_of[:, pos].long()                           # [U, P]
+            k = st.K[b[:, None], kvh[:, None], pos[None, :]].float()   # [U, P, d]
+            c = gr.cent[u[:, None], comm.clamp(min=0)]                  # [U, P, d]
+            r = (k - c).norm(dim=-1) / k.norm(dim=-1).clamp_min(1e-30)
+            acc.append(r[comm >= 0])
+    tail = torch.cat(tail) if tail else torch.zeros(0)
+    mem = torch.cat(mem) if mem else torch.zeros(0)
+    return {"rule": wl.assign_rule, "tail_tokens": int(tail.numel()),
+            "tail_rel_dist": float(tail.mean()) if tail.numel() else None,
+            "member_rel_dist": float(mem.mean()) if mem.numel() else None,
+            "metric": "mean |k - c(k)| / |k| over tokens joined since the build (tail) and over "
+                      f"{n_members} sampled build-time members per graph"}
 
 
 def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
@@ -335,6 +379,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         nsel_hist.append(sum(L.st.sel.n_sel.long().sum() for L in layers))
     torch.cuda.synchronize()
     check_dev_err("timed steps")
+    drift = assignment_drift(layers, wl, wl.T) if wl.update else None
     # per step, summed over the layers: each selection from the previous
     # layer's attention end (or the step start), each attention from its
     # selection end
@@ -462,13 +507,15 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "config": {"workload": wl.key, "title": wl.title, "B_per_gpu": wl.B, "layers": n_layers, "Hq": wl.Hq,
                    "Hkv": wl.Hkv, "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
                    "communities_per_graph": float(ncomm / (U * n_layers)), "budget": budget, "sinks": wl.S,
-                   "update": wl.update, "layout": wl.layout,
+                   "update": wl.update, "assign_rule": wl.assign_rule if wl.update else None,
+                   "layout": wl.layout,
                    "l2": "flushed by a 1 GiB write then a 512 MiB read before every timed step, outside the CUDA events",
                    "parallelism": f"dp{n_ranks} (independent batches, no collective)"},
         "tokens_per_s": value * wl.B,
         "roofline": roofline,
         "kernels": kernels,
         "dense": dense,
+        "drift": drift,
         "e2e": e2e,
         "gpu_launches": K_steps * n_layers * (KERNELS_PER_STEP_UPDATE if wl.update else KERNELS_PER_STEP_STATIC),
         "clocks": clocks,
@@ -518,7 +565,8 @@ def oracle_unit_seconds(wl: synth.Workload, draw: synth.CacheDraw, units, budget
                 O.attention(q[b, h], K, V, toks)
             nbr = O.neighbours(q[b, heads], K, toks, wl.S)
             if wl.update:
-                O.assign(kn[b, kvh], cent, [int(st.comm_of[p]) for p in nbr])
+                pick = O.assign_vote if wl.assign_rule == "vote" else O.assign
+                pick(kn[b, kvh], cent, [int(st.comm_of[p]) for p in nbr])
             t += time.perf_counter() - t0
     return t
 
@@ -573,6 +621,8 @@ def parse(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--budget", type=int, default=None)
     ap.add_argument("--batch", type=int, default=None, help="override the batch (small profiling captures)")
+    ap.add_argument("--assign-rule", default=None, choices=["score", "vote"],
+                    help="how a new token picks a neighbouring community (update workloads)")
     ap.add_argument("--layers", type=int, default=None,
                     help="layers per step (default: the workload's; each has its own cache and graphs)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
@@ -592,6 +642,8 @@ def main(argv=None):
     wl = synth.WORKLOADS[args.workload]
     if args.batch is not None:
         wl = wl.replace(B=args.batch)
+    if args.assign_rule is not None:
+        wl = wl.replace(assign_rule=args.assign_rule)
     if args.impl == "reference":
         if rank != 0:
             return 0

@@ -24,6 +24,7 @@ __all__ = [
     "ckv_sparse_decode_append",
     "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
+    "ASSIGN_SCORE", "ASSIGN_VOTE",
     "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP",
     "NEIGHBOURS",
 ]
@@ -34,6 +35,7 @@ LIB_PATH = os.environ.get("CKV_LIB") or os.path.join(os.path.dirname(os.path.abs
 
 DTYPE_F32, DTYPE_BF16 = 0, 1
 PER_GROUP, PER_HEAD = 0, 1
+ASSIGN_SCORE, ASSIGN_VOTE = 0, 1
 DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
 NEIGHBOURS = 8
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
@@ -64,7 +66,7 @@ class CacheDesc(ctypes.Structure):
 
 class GraphDesc(ctypes.Structure):
     _fields_ = [("mode", _i32), ("S", _i32), ("Cmax", _i32), ("max_tail", _i32), ("T_cap", _i32),
-                ("comm_of", _p), ("offs", _p), ("tok", _p), ("cnt", _p), ("cent", _p), ("cent_lp", _p),
+                ("assign_rule", _i32), ("comm_of", _p), ("offs", _p), ("tok", _p), ("cnt", _p), ("cent", _p), ("cent_lp", _p),
                 ("num_comm", _p), ("tail_tok", _p), ("tail_comm", _p), ("tail_len", _p),
                 ("dev_err", _p)]
 
@@ -174,7 +176,8 @@ class Selection:
     unit_prefix: torch.Tensor
 
 
-def new_graph(cache: CacheDesc, mode: int, S: int, Cmax: int, max_tail: int, device="cuda") -> Graph:
+def new_graph(cache: CacheDesc, mode: int, S: int, Cmax: int, max_tail: int, device="cuda",
+              rule: int = ASSIGN_SCORE) -> Graph:
     G = cache.Hq if mode == PER_HEAD else cache.Hkv
     U = cache.B * G
     i32 = dict(dtype=torch.int32, device=device)
@@ -191,7 +194,7 @@ def new_graph(cache: CacheDesc, mode: int, S: int, Cmax: int, max_tail: int, dev
         tail_len=torch.zeros((U,), **i32),
         dev_err=torch.zeros((1,), **i32),
     )
-    desc = GraphDesc(mode, S, Cmax, max_tail, cache.T_cap, *(t[k].data_ptr() for k in (
+    desc = GraphDesc(mode, S, Cmax, max_tail, cache.T_cap, rule, *(t[k].data_ptr() for k in (
         "comm_of", "offs", "tok", "cnt", "cent", "cent_lp", "num_comm", "tail_tok", "tail_comm", "tail_len",
         "dev_err")))
     return Graph(desc, **t)

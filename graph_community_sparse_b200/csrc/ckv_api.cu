@@ -69,6 +69,8 @@ ckv_status check_graph(const ckv_cache_desc* c, const ckv_graph_desc* g) {
     if (g->mode != CKV_GRAPH_PER_GROUP && g->mode != CKV_GRAPH_PER_HEAD)
         return fail(CKV_ERR_INVALID_ARG, "graph mode %d unknown", g->mode);
     if (g->S < 0) return fail(CKV_ERR_INVALID_ARG, "S < 0");
+    if (g->assign_rule != CKV_ASSIGN_SCORE && g->assign_rule != CKV_ASSIGN_VOTE)
+        return fail(CKV_ERR_INVALID_ARG, "assign rule %d unknown", g->assign_rule);
     if (g->Cmax < 1 || g->Cmax > ckv::MAX_CMAX)
         return fail(CKV_ERR_UNSUPPORTED, "Cmax = %d outside [1, %d]", g->Cmax, ckv::MAX_CMAX);
     if (g->max_tail < 0) return fail(CKV_ERR_INVALID_ARG, "max_tail < 0");
@@ -127,6 +129,7 @@ ckv::GraphView graph_view(const ckv_cache_desc* c, const ckv_graph_desc* g) {
     v.Cmax = g->Cmax;
     v.max_tail = g->max_tail;
     v.T_cap = g->T_cap;
+    v.rule = g->assign_rule;
     v.G = graphs_per_seq(c, g);
     v.gq = g->mode == CKV_GRAPH_PER_HEAD ? 1 : c->Hq / c->Hkv;
     v.comm_of = g->comm_of;

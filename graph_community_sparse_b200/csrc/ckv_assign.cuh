@@ -9,8 +9,9 @@
 //
 // The candidate communities are those of the 8 neighbour positions found by
 // the attention; each distinct candidate costs one d-long dot product with
-// the new key; the winner (largest k . c / sqrt(d), ties to the lower id)
-// moves its centre by (k - c)/(n + 1), its count grows by one and (pos, c)
+// the new key; the winner (largest k . c / sqrt(d), ties to the lower id; or,
+// under the vote rule, the candidate named by the most neighbours, the score
+// and then the id breaking ties) moves its centre by (k - c)/(n + 1), its count grows by one and (pos, c)
 // joins the unit's tail.  O(8 d) work per graph.
 #pragma once
 
@@ -29,6 +30,7 @@ struct AssignParams {
     int64_t csb, csh;   // cache element strides between sequences / KV heads
     int row_vec;        // 16-byte vectors per row
     int U, G, Hq, Hkv, d, per_head, Cmax, T_cap, max_tail, pos;
+    int vote;           // CKV_ASSIGN_VOTE: most neighbours first, the score breaks ties
     float inv_sqrt_d;
     const int32_t* nbr8;
     int32_t* comm_of;
@@ -75,6 +77,7 @@ inline AssignParams make_assign_params(const CacheView& c, const GraphView& g, i
     p.T_cap = g.T_cap;
     p.max_tail = g.max_tail;
     p.pos = pos;
+    p.vote = g.rule == CKV_ASSIGN_VOTE;
     p.inv_sqrt_d = 1.0f / sqrtf((float)c.d);
     p.nbr8 = nbr8;
     p.comm_of = g.comm_of;
@@ -160,14 +163,21 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     }
     sync();
     if (tid == 0) {
-        int best = -1, bi = -1;
+        // each distinct candidate carries its score at its first slot; under
+        // the vote rule the number of slots naming it comes first
+        int best = -1, bi = -1, bv = 0;
         float bs = -INFINITY;
         for (int i = 0; i < CKV_NEIGHBOURS; ++i) {
             const int ci = s_cand[i];
             if (ci < 0 || s_score[i] == -INFINITY) continue;
-            if (best < 0 || s_score[i] > bs || (s_score[i] == bs && ci < best)) {
+            int v = 0;
+            if (p.vote) {
+                for (int j = i; j < CKV_NEIGHBOURS; ++j) v += s_cand[j] == ci;
+            }
+            if (best < 0 || v > bv || (v == bv && (s_score[i] > bs || (s_score[i] == bs && ci < best)))) {
                 best = ci;
                 bi = i;
+                bv = v;
                 bs = s_score[i];
             }
         }

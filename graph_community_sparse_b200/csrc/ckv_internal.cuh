@@ -185,6 +185,7 @@ struct CacheView {
 
 struct GraphView {
     int mode, S, Cmax, max_tail, T_cap, G, gq;
+    int rule;  // ckv_assign_rule
     int32_t* comm_of;
     int32_t* offs;
     int32_t* tok;

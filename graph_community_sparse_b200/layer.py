@@ -10,7 +10,7 @@ from typing import Optional
 
 import torch
 
-from . import (PER_GROUP, PER_HEAD, Graph, Selection, cache_desc, ckv_append_assign, ckv_assign_update,
+from . import (ASSIGN_SCORE, ASSIGN_VOTE, PER_GROUP, PER_HEAD, Graph, Selection, cache_desc, ckv_append_assign, ckv_assign_update,
                ckv_sparse_decode_append,
                ckv_build_centroids, ckv_dense_decode, ckv_score_select, ckv_sparse_decode,
                ckv_workspace_size, new_graph, new_selection, new_workspace, NEIGHBOURS)
@@ -21,14 +21,19 @@ class LayerState:
 
     mode: "group" (one graph per KV group) or "head" (one graph per query head).
     tok_cap defaults to T_cap, which can never overflow.
+    rule: how a new token picks among its neighbours' communities, "score"
+    (best k . c) or "vote" (most neighbours, then the score).
     """
 
     def __init__(self, K: torch.Tensor, V: torch.Tensor, Hq: int, mode: str, S: int, Cmax: int,
-                 max_tail: int, tok_cap: Optional[int] = None):
+                 max_tail: int, tok_cap: Optional[int] = None, rule: str = "score"):
+        if rule not in ("score", "vote"):
+            raise ValueError(f"unknown assignment rule {rule!r}")
         self.K, self.V = K, V
         self.cache = cache_desc(K, V, Hq)
         self.mode = PER_HEAD if mode == "head" else PER_GROUP
-        self.graph: Graph = new_graph(self.cache, self.mode, S, Cmax, max_tail, device=K.device)
+        self.graph: Graph = new_graph(self.cache, self.mode, S, Cmax, max_tail, device=K.device,
+                                      rule=ASSIGN_VOTE if rule == "vote" else ASSIGN_SCORE)
         self.sel: Selection = new_selection(self.cache, self.graph, tok_cap or self.cache.T_cap,
                                             device=K.device)
         self.ws = new_workspace(ckv_workspace_size(self.cache, self.graph, self.sel), device=K.device)

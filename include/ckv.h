@@ -64,7 +64,7 @@ extern "C" {
 #define CKV_API
 #endif
 
-#define CKV_ABI_VERSION 2
+#define CKV_ABI_VERSION 3
 #define CKV_NEIGHBOURS 8
 
 typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
@@ -81,6 +81,19 @@ typedef enum {
 
 typedef enum { CKV_DTYPE_F32 = 0, CKV_DTYPE_BF16 = 1 } ckv_dtype;
 typedef enum { CKV_GRAPH_PER_GROUP = 0, CKV_GRAPH_PER_HEAD = 1 } ckv_graph_mode;
+
+/*
+ * How a new token picks its community among those of its 8 neighbours
+ * (ckv_assign_update and the calls fused with it).  [R-A] paragraph 6 only
+ * says the token joins a fitting neighbouring community; two readings:
+ *   CKV_ASSIGN_SCORE  the candidate maximising k_new . cent_c / sqrt(d),
+ *                     ties to the lower id (the default)
+ *   CKV_ASSIGN_VOTE   the community that holds the most of the neighbours
+ *                     (a majority vote over graph edges); among equally
+ *                     frequent ones the larger k_new . cent_c / sqrt(d), then
+ *                     the lower id
+ */
+typedef enum { CKV_ASSIGN_SCORE = 0, CKV_ASSIGN_VOTE = 1 } ckv_assign_rule;
 
 /* Bits of the device error word (ckv_graph_desc.dev_err). */
 #define CKV_DEVERR_SINK_LABEL 1   /* a position < S did not carry label -1            */
@@ -120,6 +133,7 @@ typedef struct {
  *   tail_tok, tail_comm int32 [U, max_tail]  tokens joined after the build
  *   tail_len int32 [U]
  *   dev_err  int32 [1]          OR of CKV_DEVERR_* bits; the caller zeroes it
+ * assign_rule is a ckv_assign_rule; any other value is CKV_ERR_INVALID_ARG.
  * S sink positions 0..S-1 belong to no community and are always attended
  * ([R-A] paragraph 3).  T_cap here must equal the cache's T_cap.
  */
@@ -129,6 +143,7 @@ typedef struct {
     int32_t Cmax;
     int32_t max_tail;
     int32_t T_cap;
+    int32_t assign_rule; /* ckv_assign_rule */
     int32_t* comm_of;
     int32_t* offs;
     int32_t* tok;
@@ -252,9 +267,9 @@ CKV_API ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const 
 
 /*
  * Local update for the token just written at position `pos` (its K/V rows are
- * already in the cache): in every graph unit it joins the candidate
- * community (the communities of nbr8) maximising k_new . cent_c / sqrt(d),
- * ties to the lower id; that centre moves by (k_new - cent)/(cnt + 1), cnt
+ * already in the cache): in every graph unit it joins one of the candidate
+ * communities (those of nbr8), chosen by graph->assign_rule (by default the
+ * one maximising k_new . cent_c / sqrt(d), ties to the lower id); that centre moves by (k_new - cent)/(cnt + 1), cnt
  * grows by one, and (pos, c) is appended to the tail.  O(8 d) per graph,
  * independent of the context length ([R-A] paragraph 6; [ABS]: the
  * update takes constant time).  assigned int32 [U] or NULL receives the community (-1: no

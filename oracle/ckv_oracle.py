@@ -280,9 +280,10 @@ def decode_step(mode: str, Hq: int, Hkv: int, states: Dict[tuple, GraphState],
 
 def assign_step(mode: str, Hq: int, Hkv: int, states: Dict[tuple, GraphState],
                 K: np.ndarray, res: StepResult, pos: int,
-                units: Optional[Sequence[tuple]] = None) -> Dict[tuple, int]:
+                units: Optional[Sequence[tuple]] = None, rule: str = "score") -> Dict[tuple, int]:
     """Step 6 for the token written at ``pos`` (the cache row is already
-    there): each graph's new token joins the best neighbouring community."""
+    there): each graph's new token joins the best neighbouring community,
+    by score (``assign``) or by majority vote (``assign_vote``)."""
     out = {}
     for (b, g) in (units if units is not None else sorted(res.graphs)):
         st = states[(b, g)]
@@ -290,7 +291,8 @@ def assign_step(mode: str, Hq: int, Hkv: int, states: Dict[tuple, GraphState],
         kvh = graph_kv_head(mode, g, Hq, Hkv)
         cand = [int(st.comm_of[p]) for p in gs.nbr]
         cand = [c for c in cand if c >= 0]
-        c_star = assign(K[b, kvh, pos], gs.cent, cand)
+        pick = assign_vote if rule == "vote" else assign
+        c_star = pick(K[b, kvh, pos], gs.cent, cand)
         st.join(pos, c_star)
         gs.assigned = c_star
         out[(b, g)] = c_star

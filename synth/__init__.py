@@ -67,6 +67,7 @@ class Workload:
     min_size: int = 1
     update: bool = False    # assign each new token and append it to the cache
     layout: str = "scatter"
+    assign_rule: str = "score"  # "score" | "vote": how a new token picks a neighbouring community
 
     @property
     def G(self) -> int:

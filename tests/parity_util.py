@@ -12,7 +12,8 @@ Comparison rules:
   * neighbours: equal to the oracle's on the same token set, except for
     positions whose logit lies within BAND of the 8th;
   * assignment: equal, or the two candidates' oracle scores within BAND (then
-    the oracle adopts the GPU's choice and the resync is counted);
+    the oracle adopts the GPU's choice and the resync is counted); under the
+    vote rule the two must also hold the same number of neighbours;
   * counts bit-exact and centres within 1e-5 of the oracle's recomputed means.
 """
 from __future__ import annotations
@@ -40,6 +41,7 @@ class Report:
     band_selections: int = 0
     band_neighbours: int = 0
     resyncs: int = 0
+    rule_decisive: int = 0   # vote rule: units where the score rule would have chosen otherwise
     max_out_err: float = 0.0
     max_cent_err: float = 0.0
     notes: List[str] = field(default_factory=list)
@@ -104,7 +106,8 @@ class Case:
         self.Cmax = Cmax or max(self.C, 1)
         self.U = wl.B * wl.G
         mt = wl.steps if max_tail is None else max_tail
-        self.st = LayerState(self.draw.K, self.draw.V, wl.Hq, wl.mode, wl.S, self.Cmax, mt, tok_cap)
+        self.st = LayerState(self.draw.K, self.draw.V, wl.Hq, wl.mode, wl.S, self.Cmax, mt, tok_cap,
+                             rule=wl.assign_rule)
         lab_t = torch.from_numpy(labs.reshape(self.U, wl.T).astype(np.int32)).to(device)
         self.st.build(lab_t, wl.T)
         self.states: Dict[tuple, O.GraphState] = {}
@@ -209,11 +212,17 @@ class Case:
                 cent = cand_cache[(b, g)]
                 kvh = self.kv_head(g)
                 k_new = kn[b, kvh].double().cpu().numpy()
-                cands = sorted({int(st.comm_of[p]) for p in nbr[u] if p >= 0 and st.comm_of[p] >= 0})
-                ref = O.assign(k_new, cent, cands)
+                named = [int(st.comm_of[p]) for p in nbr[u] if p >= 0 and st.comm_of[p] >= 0]
+                cands = sorted(set(named))
+                vote = wl.assign_rule == "vote"
+                ref = O.assign_vote(k_new, cent, named) if vote else O.assign(k_new, cent, cands)
+                if vote and ref != O.assign(k_new, cent, cands):
+                    rep.rule_decisive += 1
                 got = int(assigned[u])
                 if got != ref:
                     assert got in cands, f"unit {u}: assigned {got} not a candidate {cands}"
+                    if vote:
+                        assert named.count(got) == named.count(ref), f"unit {u}: {got} has fewer votes than {ref}"
                     sr = float(np.dot(k_new, cent[ref])) / math.sqrt(wl.d)
                     sg = float(np.dot(k_new, cent[got])) / math.sqrt(wl.d)
                     assert abs(sr - sg) <= BAND, f"unit {u}: assignment {got} vs {ref}"

@@ -126,6 +126,10 @@ CASES = [
     ("Cmax 0", lambda: _call_build(_cache(), _graph(Cmax=0)), UNSUPPORTED),
     ("Cmax too big", lambda: _call_build(_cache(), _graph(Cmax=100000)), UNSUPPORTED),
     ("graph mode", lambda: _call_build(_cache(), _graph(mode=5)), INVALID),
+    ("assign rule", lambda: _call_build(_cache(), _graph(assign_rule=2)), INVALID),
+    ("negative assign rule", lambda: ckv.lib.ckv_assign_update(ctypes.byref(_cache()),
+                                                              ctypes.byref(_graph(assign_rule=-1)), 5, FAKE, FAKE,
+                                                              None), INVALID),
     ("null graph array", lambda: _call_build(_cache(), _graph(cent=None)), INVALID),
     ("null cent_lp", lambda: _call_build(_cache(), _graph(cent_lp=None)), INVALID),
     ("misaligned cent_lp", lambda: _call_build(_cache(), _graph(cent_lp=FAKE + 8)), MISALIGNED),

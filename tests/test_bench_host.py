@@ -69,3 +69,24 @@ def test_single_process_helpers():
     bench.barrier(cpu)  # no process group: a no-op
     assert bench.job_value(4, 100, 2.0) == 200.0
     assert np.isnan(bench.job_value(1, 10, 0.0))
+
+
+def test_assignment_drift_on_a_hand_built_layer():
+    """One sequence, one KV head, one graph: two communities with centres
+    e0 and e1; positions 0-1 are sinks, 2-5 build-time members, 6-7 joined
+    later.  Every relative distance is worked out by hand."""
+    from types import SimpleNamespace
+
+    wl = synth.WORKLOADS["tiny"].replace(B=1, Hq=1, Hkv=1, d=2, S=2, T=6, mode="group")
+    K = torch.zeros(1, 1, 8, 2)
+    K[0, 0, 2:] = torch.tensor([[1.0, 0], [2, 0], [0, 1], [0, 2], [3, 4], [0, 1]])
+    comm_of = torch.tensor([[-1, -1, 0, 0, 1, 1, 0, -1]], dtype=torch.int32)
+    cent = torch.tensor([[[1.0, 0.0], [0.0, 1.0]]])
+    st = SimpleNamespace(K=K, U=1, T=8, graph=SimpleNamespace(comm_of=comm_of, cent=cent))
+    d = bench.assignment_drift([SimpleNamespace(st=st)], wl, T0=6, n_members=4)
+    # tail: position 6 -> |(3,4)-(1,0)|/5 = sqrt(20)/5; position 7 unassigned (skipped)
+    assert d["tail_tokens"] == 1
+    assert d["tail_rel_dist"] == pytest.approx(np.sqrt(20) / 5)
+    # members 2..5: 0, 1/2, 0, 1/2 -> 1/4
+    assert d["member_rel_dist"] == pytest.approx(0.25)
+    assert d["rule"] == "score"

@@ -230,40 +230,48 @@ def test_assign_bruteforce_ties_and_one_update():
     assert O.assign(np.ones(d), np.ones((C, d)), []) == -1
 
 
-def test_assign_vote_worked_examples_and_bruteforce():
+def check_assign_vote(fn) -> bool:
     """The majority-vote rule: most frequent neighbour community, then the
-    larger score, then the lower id."""
+    larger score, then the lower id; worked cases, then brute force."""
     d = 4
     cent = np.array([[1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0], [2, 0, 0, 0]], dtype=np.float64)
     k = np.array([1.0, 0.5, 0.0, 0.0])
+    ok = True
     # worked by hand: votes {2: 3, 0: 2, 1: 2} -> 2 wins although its score (0) is the lowest
-    assert O.assign_vote(k, cent, [2, 0, 2, 1, 0, 2, 1, -1]) == 2
-    # equal votes {0: 2, 3: 2}: scores 1/2 and 2/2 -> 3; the score rule would also pick 3
-    assert O.assign_vote(k, cent, [0, 3, 0, 3]) == 3
-    # equal votes and equal scores (cent[1] = cent[2] seen from k2) -> the lower id
+    ok &= fn(k, cent, [2, 0, 2, 1, 0, 2, 1, -1]) == 2
+    # equal votes {0: 2, 3: 2}: scores 1/2 and 2/2 -> 3
+    ok &= fn(k, cent, [0, 3, 0, 3]) == 3
+    # equal votes and equal scores (cent[1] and cent[2] seen from k2) -> the lower id
     k2 = np.array([0.0, 1.0, 1.0, 0.0])
-    assert O.assign_vote(k2, cent, [2, 1]) == 1
-    assert O.assign_vote(k, cent, [-1, -1]) == -1 and O.assign_vote(k, cent, []) == -1
+    ok &= fn(k2, cent, [2, 1]) == 1
+    ok &= fn(k, cent, [-1, -1]) == -1 and fn(k, cent, []) == -1
     rng = np.random.default_rng(23)
     C = 6
     for _ in range(200):
         cent = rng.integers(-2, 3, (C, d)).astype(np.float64)
         k = rng.integers(-2, 3, d).astype(np.float64)
-        nb = list(rng.integers(-1, C, size=8))
-        got = O.assign_vote(k, cent, nb)
+        nb = [int(x) for x in rng.integers(-1, C, size=8)]
+        got = fn(k, cent, nb)
         valid = [c for c in nb if c >= 0]
         if not valid:
-            assert got == -1
+            ok &= got == -1
             continue
-        # brute force: enumerate the communities, compare (votes, score, -id)
+        # brute force: every named community, compared on (votes, score, -id)
         best = max(set(valid), key=lambda c: (valid.count(c), float(np.dot(k, cent[c])), -c))
-        assert got == best
+        ok &= got == best
+    return bool(ok)
 
 
-def test_multi_step_invariants_on_tiny_workload():
+def test_assign_vote_worked_examples_and_bruteforce():
+    assert check_assign_vote(O.assign_vote)
+
+
+@pytest.mark.parametrize("rule", ["score", "vote"])
+def test_multi_step_invariants_on_tiny_workload(rule):
     """Tiny workload, all steps: sinks present, no duplicate positions, the
     top community always selected, exactly one count changes per graph and
-    step, and it changes by one."""
+    step, and it changes by one; under the vote rule the chosen community
+    holds the most neighbours."""
     wl = synth.WORKLOADS["tiny"]
     draw = synth.draw_cache(wl, device="cpu")
     K = draw.K.double().numpy()
@@ -282,10 +290,13 @@ def test_multi_step_invariants_on_tiny_workload():
         K[:, :, pos] = kn.double().numpy()
         V[:, :, pos] = vn.double().numpy()
         before = O.centroids(K[0, 0, :states[(0, 0)].T], states[(0, 0)].members())[1]
-        a = O.assign_step(wl.mode, wl.Hq, wl.Hkv, states, K, res, pos)
+        named = [int(states[(0, 0)].comm_of[p]) for p in gs.nbr]
+        a = O.assign_step(wl.mode, wl.Hq, wl.Hkv, states, K, res, pos, rule=rule)
         after = O.centroids(K[0, 0, :states[(0, 0)].T], states[(0, 0)].members())[1]
         diff = after - before
-        assert a[(0, 0)] in {int(states[(0, 0)].comm_of[p]) for p in gs.nbr}
+        assert a[(0, 0)] in named
+        if rule == "vote":
+            assert named.count(a[(0, 0)]) == max(named.count(c) for c in named if c >= 0)
         assert diff.sum() == 1 and diff[a[(0, 0)]] == 1
 
 
@@ -374,6 +385,22 @@ def _mut_neighbours_first_head(q, K, positions, S, k=8):
     return O.neighbours(np.atleast_2d(q)[:1], K, positions, S, k)
 
 
+def _mut_vote_distinct(k_new, cent, neighbour_comms):
+    # repeats dropped: degenerates to the score rule
+    return O.assign(k_new, cent, [c for c in neighbour_comms if c >= 0])
+
+
+def _mut_vote_no_score(k_new, cent, neighbour_comms):
+    # equal votes go to the lower id, ignoring the score
+    valid = [int(c) for c in neighbour_comms if c >= 0]
+    return min(set(valid), key=lambda c: (-valid.count(c), c)) if valid else -1
+
+
+def _mut_vote_high_id(k_new, cent, neighbour_comms):
+    valid = [int(c) for c in neighbour_comms if c >= 0]
+    return max(set(valid), key=lambda c: (valid.count(c), float(np.dot(k_new, cent[c])), c)) if valid else -1
+
+
 _REAL_TOKEN_SET = O.token_set
 
 
@@ -401,6 +428,11 @@ def test_pins_catch_attention_mutants(mutant):
                                     _mut_neighbours_first_head])
 def test_pins_catch_neighbour_mutants(mutant):
     assert not check_neighbours(mutant)
+
+
+@pytest.mark.parametrize("mutant", [_mut_vote_distinct, _mut_vote_no_score, _mut_vote_high_id])
+def test_pins_catch_vote_mutants(mutant):
+    assert not check_assign_vote(mutant)
 
 
 def test_pins_catch_dropped_sinks(monkeypatch):

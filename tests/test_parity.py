@@ -38,6 +38,8 @@ SHAPES = [
     small("bf16_spans", 27, layout="spans"),
     small("bf16_d128_gq8", 28, Hq=32, Hkv=4),
     small("bf16_d64_gq4_head", 29, d=64, mode="head", Hq=16, Hkv=4, budgets=(150,)),
+    small("bf16_group_vote", 44, assign_rule="vote", steps=4),
+    small("f32_d64_head_vote", 45, dtype="f32", d=64, mode="head", Hq=8, Hkv=4, assign_rule="vote"),
 ]
 
 
@@ -247,7 +249,8 @@ def test_fused_decode_append_matches_separate_calls():
     same outputs, neighbours, cache and graph state, bit for bit, as
     ckv_sparse_decode followed by ckv_append_assign."""
     for wl in (small("fused_head", 40, mode="head", T=2500, budgets=(200,), steps=3),
-               small("fused_group", 41, steps=3), synth.WORKLOADS["tiny"].replace(steps=3)):
+               small("fused_group", 41, steps=3), synth.WORKLOADS["tiny"].replace(steps=3),
+               small("fused_vote", 46, mode="head", Hq=16, Hkv=4, d=64, steps=3, assign_rule="vote")):
         a, b = Case(wl), Case(wl)
         for i in range(wl.steps):
             q = synth.draw_queries(wl, a.draw, i)
@@ -299,3 +302,23 @@ def test_cut_among_scores_closer_than_bf16():
     assert rep.band_selections == 0
     n_sel = case.st.sel.n_sel.cpu().numpy()
     assert np.all(n_sel > 3)
+
+
+def test_vote_rule_is_decisive_and_matches_oracle():
+    """Under the vote rule the assignments follow the oracle's majority vote
+    (checked inside Case.step), and on these inputs the vote picks another
+    community than the score rule would in some units, so the check has
+    teeth; the same layer under the score rule makes different choices."""
+    wl = small("vote_decisive", 47, Hq=16, Hkv=4, mode="head", steps=4, assign_rule="vote")
+    vote, score = Case(wl), Case(wl.replace(assign_rule="score"))
+    rep = Report()
+    picks_v, picks_s = [], []
+    for _ in range(wl.steps):
+        vote.step(wl.budget, rep=rep)
+        score.step(wl.budget)
+        picks_v.append(vote.st.assigned.cpu().clone())
+        picks_s.append(score.st.assigned.cpu().clone())
+    assert rep.rule_decisive > 0, rep
+    assert any(not torch.equal(a, b) for a, b in zip(picks_v, picks_s))
+    assert int(vote.st.graph.dev_err.item()) == 0
+    print(rep)
