@@ -396,16 +396,6 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     const float* sc = p.scores + (size_t)u * p.Cmax;
     const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
     const int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
-    // The pages this block writes or reads late (token list, members, CSR
-    // offsets, ranked ids) are touched now by prefetches, so their address
-    // translations overlap the first loads instead of stalling the copy.
-    if (tid < 4) {
-        const void* pg = tid == 0 ? (const void*)(p.sel_tok + (size_t)u * p.tok_cap)
-                       : tid == 1 ? (const void*)(p.tok + (size_t)u * p.T_cap)
-                       : tid == 2 ? (const void*)(p.offs + (size_t)u * (p.Cmax + 1))
-                                  : (const void*)(p.sel_comm + (size_t)u * p.Cmax);
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(pg));
-    }
     for (int i = tid; i < (p.Cmax + 31) / 32; i += nt) s_mask[i] = 0u;
     if (tid == 0) {
         s_bstar = -1;
@@ -758,10 +748,37 @@ __global__ void __launch_bounds__(SEL_THREADS) score_kernel(SelectParams p) {
     score_rows<T, D, GQ>(p, u, C);
 }
 
+// Thread i < SEL_PREFETCH warms one page the selection of unit u reads or
+// writes after its first loads (token list, members, CSR offsets, ranked
+// ids, sizes, fp32 centres, tail), so the address translations are done
+// before they are needed.  None is written by the scoring kernel: issued
+// before waiting for it, they overlap its last blocks.
+constexpr int SEL_PREFETCH = 11;
+__device__ __forceinline__ void select_prefetch(const SelectParams& p, int u, int i, int D) {
+    const size_t crow = (size_t)u * p.Cmax * D;
+    const void* a = nullptr;
+    switch (i) {
+        case 0: a = p.sel_tok + (size_t)u * p.tok_cap; break;
+        case 1: a = p.tok + (size_t)u * p.T_cap; break;
+        case 2: a = p.tok + (size_t)u * p.T_cap + p.T_cap - 1; break;
+        case 3: a = p.offs + (size_t)u * (p.Cmax + 1); break;
+        case 4: a = p.sel_comm + (size_t)u * p.Cmax; break;
+        case 5: a = p.cnt + (size_t)u * p.Cmax; break;
+        case 6: a = p.cent + crow; break;
+        case 7: a = p.cent + crow + (size_t)(p.Cmax - 1) * D; break;
+        case 8: a = p.max_tail > 0 ? p.tail_tok + (size_t)u * p.max_tail : nullptr; break;
+        case 9: a = p.max_tail > 0 ? p.tail_comm + (size_t)u * p.max_tail : nullptr; break;
+        case 10: a = p.tail_len + u; break;
+        default: break;
+    }
+    if (a) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+}
+
 template <typename T, int D, int GQ>
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
-    pdl_wait();  // every score and histogram update of the scoring kernel is visible
     const int u = blockIdx.x;
+    if (threadIdx.x < SEL_PREFETCH) select_prefetch(p, u, threadIdx.x, D);
+    pdl_wait();  // every score and histogram update of the scoring kernel is visible
     const int C = min(p.num_comm[u], p.Cmax);
     select_unit<T, D, GQ>(p, u, C);
 }
