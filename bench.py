@@ -420,6 +420,19 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     kernels[dec_name] = {"ms": float(np.mean(dec_ms)), "bytes": float(np.mean(dec_bytes)), "GB/s": dec_gbs,
                          "frac": dec_gbs / peak, "rows_per_step": float(rows.mean()),
                          "tokens_per_step": float(ntok.mean())}
+    # the whole step against the same peak: both calls' bytes over the timed
+    # steps' mean duration
+    step_bytes = float(np.mean(sel_bytes) + np.mean(dec_bytes))
+    step_gbs = step_bytes / (float(np.mean(step_ms)) * 1e-3) / 1e9
+    step_roofline = {"ms": float(np.mean(step_ms)), "bytes": step_bytes, "GB/s": step_gbs, "frac": step_gbs / peak}
+    # per-layer breakdown of the multi-layer step (means over the per-call pass)
+    per_layer = None
+    if n_layers > 1:
+        per_layer = {
+            "sel_us": [round(float(np.mean([(e[0] if li == 0 else e[2 * li]).elapsed_time(e[1 + 2 * li])
+                                            for e in bevs])) * 1e3, 2) for li in range(n_layers)],
+            "attn_us": [round(float(np.mean([e[1 + 2 * li].elapsed_time(e[2 + 2 * li]) for e in bevs])) * 1e3, 2)
+                        for li in range(n_layers)]}
     dom = max((dec_name, "ckv_score_select"), key=lambda k: kernels[k]["ms"])
     roofline = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": peak, "unit": "GB/s",
                 "frac": kernels[dom]["GB/s"] / peak, "peak_source": peak_src,
@@ -514,6 +527,8 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "tokens_per_s": value * wl.B,
         "roofline": roofline,
         "kernels": kernels,
+        "step_roofline": step_roofline,
+        "per_layer": per_layer,
         "dense": dense,
         "drift": drift,
         "e2e": e2e,
@@ -531,9 +546,10 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
 # ----------------------------------------------------------------------------
 
 def oracle_unit_seconds(wl: synth.Workload, draw: synth.CacheDraw, units, budget: int, step: int,
-                        layer: int = 0) -> float:
+                        layer: int = 0, threads: int = 1) -> float:
     """Wall time of the oracle's steps for the given (b, g) units of one step,
-    single-threaded, inputs already converted to float64."""
+    with the numerical library limited to ``threads`` threads, inputs already
+    converted to float64."""
     import oracle.ckv_oracle as O
     from threadpoolctl import threadpool_limits
 
@@ -549,7 +565,7 @@ def oracle_unit_seconds(wl: synth.Workload, draw: synth.CacheDraw, units, budget
         kn, _ = synth.draw_new_tokens(wl, draw, step, layer)
         kn = kn.double().cpu().numpy()
     t = 0.0
-    with threadpool_limits(1):
+    with threadpool_limits(threads):
         for (b, g) in units:
             st = O.GraphState(draw.labels[b, g], wl.T_cap, wl.S, C)
             kvh = O.graph_kv_head(wl.mode, g, wl.Hq, wl.Hkv)
@@ -583,11 +599,19 @@ def cpu_baseline(wl: synth.Workload, budget: int, device, n_units: int, n_layers
     units = sample_units(wl, n_units, 1)
     t = oracle_unit_seconds(wl, draw, units, budget, 0)
     per_step = t / len(units) * (wl.B * wl.G) * n_layers
+    # the same oracle with the numerical library free to use every host core
+    # (its Python loops stay on one), on half the sample
+    ncpu = os.cpu_count() or 1
+    half = units[: max(1, len(units) // 2)]
+    t_all = oracle_unit_seconds(wl, draw, half, budget, 0, threads=ncpu)
     del draw
     lay = f" x {n_layers} layers" if n_layers > 1 else ""
     return {"value": 1.0 / per_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
             "sample": f"{len(units)} of {wl.B * wl.G} graph units of one decode step{lay} "
-                      f"({t:.1f} s single-threaded float64 numpy), scaled to the whole step"}
+                      f"({t:.1f} s single-threaded float64 numpy), scaled to the whole step",
+            "all_cores": {"value": 1.0 / (t_all / len(half) * (wl.B * wl.G) * n_layers), "unit": "steps/s",
+                          "cores": ncpu, "sample": f"{len(half)} of the same units, numpy free to use {ncpu} "
+                                                   f"threads ({t_all:.1f} s)"}}
 
 
 def run_reference(args, wl: synth.Workload, device) -> dict:

@@ -21,7 +21,7 @@ __all__ = [
     "Graph", "Selection", "cache_desc", "new_graph", "new_selection", "new_workspace",
     "ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
     "ckv_sparse_decode_noalloc", "NOALLOC_SCRATCH_BYTES", "ckv_assign_update", "ckv_append_assign",
-    "ckv_sparse_decode_append",
+    "ckv_sparse_decode_append", "ckv_get_device_error",
     "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "ASSIGN_SCORE", "ASSIGN_VOTE",
@@ -40,6 +40,7 @@ DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2
 NEIGHBOURS = 8
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
             "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
+            "ckv_get_device_error",
             "ckv_dense_decode",
             "ckv_status_string", "ckv_last_error", "ckv_abi_version")
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -87,9 +88,10 @@ lib.ckv_append_assign.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p
 lib.ckv_sparse_decode_append.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _i32, _p,
                                          _p, _p, _p, _sz, _p]
 lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
+lib.ckv_get_device_error.argtypes = [_P(GraphDesc), _p, _P(ctypes.c_int32), _i32]
 for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
-           "ckv_dense_decode"):
+           "ckv_dense_decode", "ckv_get_device_error"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.ckv_status_string.argtypes = [ctypes.c_int]
 lib.ckv_status_string.restype = ctypes.c_char_p
@@ -290,6 +292,15 @@ def ckv_sparse_decode_append(cache: CacheDesc, q: torch.Tensor, graph: Graph, se
                                         v_new.data_ptr(), _ptr(assigned), ws.data_ptr(), ws.numel(),
                                         _stream(stream)),
            "ckv_sparse_decode_append")
+
+
+def ckv_get_device_error(graph: Graph, reset: bool = False, stream=None) -> int:
+    """The graph's device error word (OR of DEVERR_* bits) once the stream's
+    queued work is done; reset=True zeroes it afterwards."""
+    code = ctypes.c_int32(0)
+    _check(lib.ckv_get_device_error(ctypes.byref(graph.desc), _stream(stream), ctypes.byref(code), int(reset)),
+           "ckv_get_device_error")
+    return int(code.value)
 
 
 def ckv_append_assign(cache: CacheDesc, graph: Graph, pos: int, k_new: torch.Tensor, v_new: torch.Tensor,

@@ -169,6 +169,19 @@ extern "C" {
 
 int32_t ckv_abi_version(void) { return CKV_ABI_VERSION; }
 
+ckv_status ckv_get_device_error(const ckv_graph_desc* graph, ckv_stream_t stream, int32_t* code, int32_t reset) {
+    if (!graph || !graph->dev_err) return fail(CKV_ERR_INVALID_ARG, "graph descriptor or its dev_err is NULL");
+    if (!code) return fail(CKV_ERR_INVALID_ARG, "code is NULL");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, graph->dev_err, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e == cudaSuccess && reset && word != 0) e = cudaMemsetAsync(graph->dev_err, 0, sizeof(int32_t), st);
+    if (e != cudaSuccess) return cuda_status(e, "ckv_get_device_error");
+    *code = word;
+    return ok();
+}
+
 const char* ckv_status_string(ckv_status s) {
     switch (s) {
         case CKV_OK: return "CKV_OK";

@@ -314,6 +314,17 @@ CKV_API ckv_status ckv_sparse_decode_append(const ckv_cache_desc* cache, const v
 CKV_API ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t T, float* out,
                             void* ws, size_t ws_bytes, ckv_stream_t stream);
 
+/*
+ * Reads the graph's device error word (ckv_graph_desc.dev_err, an OR of
+ * CKV_DEVERR_* bits) after everything queued on `stream` so far: the one
+ * call that synchronises (it waits for the stream).  *code receives the
+ * word; with reset != 0 the word is then set back to zero on the device.
+ * NULL graph or code: CKV_ERR_INVALID_ARG; a failed copy or wait:
+ * CKV_ERR_CUDA.
+ */
+CKV_API ckv_status ckv_get_device_error(const ckv_graph_desc* graph, ckv_stream_t stream, int32_t* code,
+                                        int32_t reset);
+
 CKV_API const char* ckv_status_string(ckv_status status);
 /* Message of the last failed call on this host thread ("" if none). */
 CKV_API const char* ckv_last_error(void);

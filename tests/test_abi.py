@@ -176,6 +176,11 @@ CASES = [
     ("dense ws", lambda: ckv.lib.ckv_dense_decode(ctypes.byref(_cache()), FAKE, 100, FAKE, FAKE, 8, None),
      WORKSPACE),
     ("null cache", lambda: ckv.lib.ckv_dense_decode(None, FAKE, 100, FAKE, FAKE, 1 << 40, None), INVALID),
+    ("device error null graph", lambda: ckv.lib.ckv_get_device_error(None, None, ctypes.byref(ctypes.c_int32()), 0),
+     INVALID),
+    ("device error null code", lambda: ckv.lib.ckv_get_device_error(ctypes.byref(_graph()), None, None, 0), INVALID),
+    ("device error null word", lambda: ckv.lib.ckv_get_device_error(ctypes.byref(_graph(dev_err=None)), None,
+                                                                     ctypes.byref(ctypes.c_int32()), 0), INVALID),
 ]
 
 

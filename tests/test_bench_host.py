@@ -90,3 +90,9 @@ def test_assignment_drift_on_a_hand_built_layer():
     # members 2..5: 0, 1/2, 0, 1/2 -> 1/4
     assert d["member_rel_dist"] == pytest.approx(0.25)
     assert d["rule"] == "score"
+
+
+def test_cpu_baseline_reports_single_and_all_core_oracle_rates():
+    cb = bench.cpu_baseline(synth.WORKLOADS["tiny"], 128, torch.device("cpu"), 4)
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0
+    assert cb["all_cores"]["cores"] == (os.cpu_count() or 1) and cb["all_cores"]["value"] > 0

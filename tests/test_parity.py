@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import graph_community_sparse_b200 as ckv
 import oracle.ckv_oracle as O
 import synth
 from parity_util import BAND, TOL, Case, Report
@@ -184,6 +185,10 @@ def test_bad_labels_are_flagged_and_skipped():
     case = Case(wl, labels=bad, Cmax=C)
     err = int(case.st.graph.dev_err.item())
     assert err & 1 and err & 2
+    # the same word through the library's reader, which can also clear it
+    assert ckv.ckv_get_device_error(case.st.graph) == err
+    assert ckv.ckv_get_device_error(case.st.graph, reset=True) == err
+    assert ckv.ckv_get_device_error(case.st.graph) == 0 and int(case.st.graph.dev_err.item()) == 0
     comm_of = case.st.graph.comm_of.cpu().numpy()
     assert comm_of[0, 1] == -1 and comm_of[1, 100] == -1
     assert int(case.st.graph.cnt.sum().item()) == wl.B * wl.G * (wl.T - wl.S) - 1
