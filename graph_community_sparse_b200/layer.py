@@ -38,9 +38,13 @@ class LayerState:
                                             device=K.device)
         self.ws = new_workspace(ckv_workspace_size(self.cache, self.graph, self.sel), device=K.device)
         B, Hq_, d = self.cache.B, Hq, self.cache.d
-        self.out = torch.empty((B, Hq_, d), dtype=torch.float32, device=K.device)
-        self.nbr8 = torch.full((self.graph.U, NEIGHBOURS), -1, dtype=torch.int32, device=K.device)
-        self.assigned = torch.full((self.graph.U,), -1, dtype=torch.int32, device=K.device)
+        # the step's results share one allocation (out, then nbr8, then
+        # assigned; all 4-byte types), so a caller reads them back with one copy
+        n_out, U = B * Hq_ * d, self.graph.U
+        self.results = torch.full((n_out + U * NEIGHBOURS + U,), -1, dtype=torch.int32, device=K.device)
+        self.out = self.results[:n_out].view(torch.float32).view(B, Hq_, d)
+        self.nbr8 = self.results[n_out: n_out + U * NEIGHBOURS].view(U, NEIGHBOURS)
+        self.assigned = self.results[n_out + U * NEIGHBOURS:]
         self.T = 0
 
     @property
