@@ -401,10 +401,11 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         # and the new K/V rows copied into the cache
         dec_bytes = dec_bytes + ntok * 8 + n_layers * (U * (8 * 4 + 8 * wl.d * 4 + 2 * wl.d * 4)
                                                        + 4 * wl.B * wl.Hkv * wl.d * esz)
-    # the scoring pass reads every centre in bf16; the selected communities
-    # (at least) are re-scored from the fp32 centres; per community a size is
-    # read and a score bound written and read back; the token list is written
-    sel_bytes = ncomm * wl.d * 2 + nsel * wl.d * 4 + q_bytes + ncomm * 4 * 3 + ntok * 4
+    # the scoring pass reads every centre's int8 codes and scale; the selected
+    # communities (at least) are re-scored from the fp32 centres; per
+    # community a size is read and a score bound written and read back; the
+    # token list is written
+    sel_bytes = ncomm * (wl.d + 4) + nsel * wl.d * 4 + q_bytes + ncomm * 4 * 3 + ntok * 4
     peak, peak_src = measured_peaks()
 
     def gbs(bytes_, ms):

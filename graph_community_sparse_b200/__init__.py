@@ -67,7 +67,7 @@ class CacheDesc(ctypes.Structure):
 
 class GraphDesc(ctypes.Structure):
     _fields_ = [("mode", _i32), ("S", _i32), ("Cmax", _i32), ("max_tail", _i32), ("T_cap", _i32),
-                ("assign_rule", _i32), ("comm_of", _p), ("offs", _p), ("tok", _p), ("cnt", _p), ("cent", _p), ("cent_lp", _p),
+                ("assign_rule", _i32), ("comm_of", _p), ("offs", _p), ("tok", _p), ("cnt", _p), ("cent", _p), ("cent_q", _p), ("cent_qs", _p),
                 ("num_comm", _p), ("tail_tok", _p), ("tail_comm", _p), ("tail_len", _p),
                 ("dev_err", _p)]
 
@@ -156,7 +156,8 @@ class Graph:
     tok: torch.Tensor
     cnt: torch.Tensor
     cent: torch.Tensor
-    cent_lp: torch.Tensor
+    cent_q: torch.Tensor
+    cent_qs: torch.Tensor
     num_comm: torch.Tensor
     tail_tok: torch.Tensor
     tail_comm: torch.Tensor
@@ -189,7 +190,8 @@ def new_graph(cache: CacheDesc, mode: int, S: int, Cmax: int, max_tail: int, dev
         tok=torch.zeros((U, cache.T_cap), **i32),
         cnt=torch.zeros((U, Cmax), **i32),
         cent=torch.zeros((U, Cmax, cache.d), dtype=torch.float32, device=device),
-        cent_lp=torch.zeros((U, Cmax, cache.d), dtype=torch.bfloat16, device=device),
+        cent_q=torch.zeros((U, Cmax, cache.d), dtype=torch.int8, device=device),
+        cent_qs=torch.zeros((U, Cmax), dtype=torch.float32, device=device),
         num_comm=torch.zeros((U,), **i32),
         tail_tok=torch.zeros((U, max(max_tail, 1)), **i32),
         tail_comm=torch.zeros((U, max(max_tail, 1)), **i32),
@@ -197,7 +199,7 @@ def new_graph(cache: CacheDesc, mode: int, S: int, Cmax: int, max_tail: int, dev
         dev_err=torch.zeros((1,), **i32),
     )
     desc = GraphDesc(mode, S, Cmax, max_tail, cache.T_cap, rule, *(t[k].data_ptr() for k in (
-        "comm_of", "offs", "tok", "cnt", "cent", "cent_lp", "num_comm", "tail_tok", "tail_comm", "tail_len",
+        "comm_of", "offs", "tok", "cnt", "cent", "cent_q", "cent_qs", "num_comm", "tail_tok", "tail_comm", "tail_len",
         "dev_err")))
     return Graph(desc, **t)
 

@@ -78,11 +78,12 @@ ckv_status check_graph(const ckv_cache_desc* c, const ckv_graph_desc* g) {
     if (g->S > g->T_cap) return fail(CKV_ERR_CAPACITY, "S > T_cap");
     const int64_t U = (int64_t)c->B * graphs_per_seq(c, g);
     if (U > ckv::MAX_UNITS) return fail(CKV_ERR_UNSUPPORTED, "B*G = %lld above %d", (long long)U, ckv::MAX_UNITS);
-    if (!g->comm_of || !g->offs || !g->tok || !g->cnt || !g->cent || !g->cent_lp || !g->num_comm || !g->tail_len ||
+    if (!g->comm_of || !g->offs || !g->tok || !g->cnt || !g->cent || !g->cent_q || !g->cent_qs || !g->num_comm ||
+        !g->tail_len ||
         !g->dev_err || (g->max_tail > 0 && (!g->tail_tok || !g->tail_comm)))
         return fail(CKV_ERR_INVALID_ARG, "a graph array pointer is NULL");
-    if (!aligned16(g->cent) || !aligned16(g->cent_lp))
-        return fail(CKV_ERR_MISALIGNED, "cent and cent_lp must be 16-byte aligned");
+    if (!aligned16(g->cent) || !aligned16(g->cent_q) || !aligned16(g->cent_qs))
+        return fail(CKV_ERR_MISALIGNED, "cent, cent_q and cent_qs must be 16-byte aligned");
     if (U * (int64_t)g->T_cap > (int64_t)1 << 31 || U * (int64_t)g->Cmax * c->d > (int64_t)1 << 40)
         return fail(CKV_ERR_UNSUPPORTED, "graph arrays too large");
     return CKV_OK;
@@ -137,7 +138,8 @@ ckv::GraphView graph_view(const ckv_cache_desc* c, const ckv_graph_desc* g) {
     v.tok = g->tok;
     v.cnt = g->cnt;
     v.cent = g->cent;
-    v.cent_lp = reinterpret_cast<__nv_bfloat16*>(g->cent_lp);
+    v.cent_q = g->cent_q;
+    v.cent_qs = g->cent_qs;
     v.num_comm = g->num_comm;
     v.tail_tok = g->tail_tok;
     v.tail_comm = g->tail_comm;

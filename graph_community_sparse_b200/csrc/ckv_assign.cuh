@@ -36,7 +36,8 @@ struct AssignParams {
     int32_t* comm_of;
     int32_t* cnt;
     float* cent;
-    __nv_bfloat16* cent_lp;
+    int8_t* cent_q;
+    float* cent_qs;
     int32_t* tail_tok;
     int32_t* tail_comm;
     int32_t* tail_len;
@@ -83,7 +84,8 @@ inline AssignParams make_assign_params(const CacheView& c, const GraphView& g, i
     p.comm_of = g.comm_of;
     p.cnt = g.cnt;
     p.cent = g.cent;
-    p.cent_lp = g.cent_lp;
+    p.cent_q = g.cent_q;
+    p.cent_qs = g.cent_qs;
     p.tail_tok = g.tail_tok;
     p.tail_comm = g.tail_comm;
     p.tail_len = g.tail_len;
@@ -100,6 +102,7 @@ inline AssignParams make_assign_params(const CacheView& c, const GraphView& g, i
 template <typename T, int D, int NW, typename Sync>
 __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const int* nbrpos, int tid, Sync sync) {
     constexpr int E = D / 32;
+    static_assert(E == 2 || E == 4, "d is 64 or 128");
     __shared__ int s_cand[CKV_NEIGHBOURS];
     __shared__ float s_score[CKV_NEIGHBOURS];
     __shared__ int s_cnt[CKV_NEIGHBOURS];
@@ -207,17 +210,29 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     if (best < 0 || warp != 0) return;
     // running mean: c <- c + (k - c) / (n + 1), from the copy of the centre
     // taken while scoring
-    float* cr = p.cent + ((size_t)u * p.Cmax + best) * D + lane * E;
-    __nv_bfloat16* clp = p.cent_lp + ((size_t)u * p.Cmax + best) * D + lane * E;
+    const size_t row = (size_t)u * p.Cmax + best;
+    float* cr = p.cent + row * D + lane * E;
     const float* c0r = s_row[s_bi] + lane * E;
     const float denom = (float)(s_n + 1);
+    float c1[E], amax = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const float c0 = c0r[e];
-        const float c1 = c0 + (kx[e] - c0) / denom;
-        cr[e] = c1;
-        clp[e] = __float2bfloat16_rn(c1);  // the scoring copy follows the centre
+        c1[e] = c0 + (kx[e] - c0) / denom;
+        cr[e] = c1[e];
+        amax = fmaxf(amax, fabsf(c1[e]));
     }
+    // the int8 scoring copy follows the centre: new scale, new codes
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+    const float sc = q8_scale(amax);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) packed |= (uint32_t)(q8_code(c1[e], sc) & 0xff) << (8 * e);
+    int8_t* qr = p.cent_q + row * D + lane * E;
+    if constexpr (E == 4) *reinterpret_cast<uint32_t*>(qr) = packed;
+    else *reinterpret_cast<uint16_t*>(qr) = (uint16_t)packed;
+    if (lane == 0) p.cent_qs[row] = sc;
 }
 
 }  // namespace ckv

@@ -15,7 +15,8 @@
 //                 members end up sorted by (community, position).
 // build_mean: one block per (unit, community); 8 warps sum member rows in a
 //   fixed interleaving in fp64 and combine in warp order: deterministic, and
-//   the fp32 centre is the correctly rounded mean up to fp64 summation error.
+//   the fp32 centre is the correctly rounded mean up to fp64 summation error;
+//   the row's int8 scoring copy (scale and codes) is written with it.
 #include "ckv_internal.cuh"
 
 namespace ckv {
@@ -32,7 +33,8 @@ struct BuildParams {
     int32_t* tok;
     int32_t* cnt;
     float* cent;
-    __nv_bfloat16* cent_lp;
+    int8_t* cent_q;
+    float* cent_qs;
     int32_t* num_comm;
     int32_t* tail_len;
     int32_t* dev_err;
@@ -163,14 +165,27 @@ __global__ void __launch_bounds__(256) build_mean(BuildParams p) {
 #pragma unroll
     for (int e = 0; e < E; ++e) part[warp][lane * E + e] = acc[e];
     __syncthreads();
+    float m = 0.f;
     if (threadIdx.x < D) {
         double s = 0.0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) s += part[w][threadIdx.x];
-        const float m = n > 0 ? (float)(s / (double)n) : 0.f;
+        m = n > 0 ? (float)(s / (double)n) : 0.f;
         p.cent[((size_t)u * p.Cmax + c) * D + threadIdx.x] = m;
-        p.cent_lp[((size_t)u * p.Cmax + c) * D + threadIdx.x] = __float2bfloat16_rn(m);
     }
+    // the int8 scoring copy: the row's scale from its largest magnitude
+    __shared__ float s_amax[8];
+    float a = fabsf(m);  // 0 on the threads past D
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, o));
+    if (lane == 0) s_amax[warp] = a;
+    __syncthreads();
+    float amax = s_amax[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_amax[w]);
+    const float sc = q8_scale(amax);
+    if (threadIdx.x < D) p.cent_q[((size_t)u * p.Cmax + c) * D + threadIdx.x] = (int8_t)q8_code(m, sc);
+    if (threadIdx.x == 0) p.cent_qs[(size_t)u * p.Cmax + c] = sc;
 }
 
 size_t build_ws_bytes(int U, int Cmax, int T_cap) {
@@ -202,7 +217,8 @@ cudaError_t launch_build(const CacheView& c, const GraphView& g, const int32_t* 
     p.tok = g.tok;
     p.cnt = g.cnt;
     p.cent = g.cent;
-    p.cent_lp = g.cent_lp;
+    p.cent_q = g.cent_q;
+    p.cent_qs = g.cent_qs;
     p.num_comm = g.num_comm;
     p.tail_len = g.tail_len;
     p.dev_err = g.dev_err;

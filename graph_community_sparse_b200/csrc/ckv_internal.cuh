@@ -58,6 +58,18 @@ __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // ---------------------------------------------------------------------------
+// The int8 scoring copy of a centre row: scale s = max_i |c_i| / 127 and code
+// round-half-even(c_i / s) (0 for an all-zero row), both divisions IEEE.
+// |c_i - s code_i| <= s (1/2 + 2^-17): the quotient's rounding adds at most
+// 127 ulp(1)/2 to the half unit of the integer rounding.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float q8_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f; }
+__device__ __forceinline__ int q8_code(float c, float s) {
+    if (!(s > 0.f)) return 0;
+    return max(-127, min(127, __float2int_rn(__fdiv_rn(c, s))));
+}
+
+// ---------------------------------------------------------------------------
 // cp.async (global -> shared, L2 only); size 0 means zero-fill, nothing read
 // ---------------------------------------------------------------------------
 
@@ -191,7 +203,8 @@ struct GraphView {
     int32_t* tok;
     int32_t* cnt;
     float* cent;
-    __nv_bfloat16* cent_lp;
+    int8_t* cent_q;
+    float* cent_qs;
     int32_t* num_comm;
     int32_t* tail_tok;
     int32_t* tail_comm;

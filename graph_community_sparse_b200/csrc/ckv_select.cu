@@ -8,14 +8,16 @@
 //
 // The score is s_c = max over the graph's query heads of q_h . cent_c /
 // sqrt(d) in fp32, and the selection is exactly the one those scores give;
-// but the centres are streamed only once, in bf16 (cent_lp), which halves
-// the bytes of the pass over every community:
+// but the pass over every community streams the centres' int8 copy (codes
+// cent_q with one fp32 scale s_c per row, cent_qs), a quarter of the fp32
+// bytes:
 //  * score_kernel, grid (centre blocks of 128, units): a streaming
-//    matrix-vector product over the bf16 centres (one half-warp per row,
-//    16-byte loads, the value-exchanging butterfly of the attention kernel
-//    for the head sums) gives s~_c and a rigorous bound e_c >= |s_c - s~_c|
-//    from sum |q| |cent_lp| (LP_REL_BOUND).  The upper bound s~ + e is
-//    stored; the community's size is added, with a global atomic, to a
+//    matrix-vector product over the codes (16-byte loads; one query head:
+//    8 lanes per row; several heads: tensor cores for a bf16 q, else a
+//    half-warp per row with the value-exchanging butterfly of the attention
+//    kernel for the head sums) gives s~_c = s_c q . code_c / sqrt(d) and a
+//    rigorous bound e_c >= |s_c - s~_c| from s_c |q|_1 (Q8_BOUND).  The
+//    upper bound s~ + e is stored; the community's size is added, with a global atomic, to a
 //    per-unit histogram over the top 12 bits of the key of the lower bound
 //    s~ - e, key = (orderable score << 32) | ~id (unique; orders communities
 //    by score desc, id asc);
@@ -48,18 +50,21 @@ template <int GQ> struct ScoreBlockRows { static constexpr int v = GQ == 1 ? SCO
 constexpr int SEL_HBITS = HIST_BITS;
 constexpr int SEL_HBINS = HIST_BINS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
-// Bound on |fp32 score from cent - fp32 score from cent_lp| per unit of
-// sum_i |q_i| |cent_lp_i| / sqrt(d): bf16 rounding contributes at most 2^-9
-// (1 + 2^-9), the two fp32 dot products' rounding (depth <= 13 for d <= 128)
-// about 2^-19 each; 2^-8 leaves a factor 1.9 of margin.  The absolute term
-// covers bf16 subnormals.
-constexpr float LP_REL_BOUND = 1.0f / 256.0f;
-constexpr float LP_ABS_BOUND = 1e-30f;
+// Bound on |fp32 score from cent - fp32 score from the int8 copy| per unit
+// of s_c |q|_1 / sqrt(d) (s_c the row's scale): the codes contribute at most
+// 1/2 + 2^-17 (see q8_scale); the fp32 dot products, of depth <= 19 over
+// terms summing to at most 127 |q|_1 (codes) or 127 s_c |q|_1 (fp32 centre),
+// about 2^-12.8 and 2^-13.8; the products by s_c and 1/sqrt(d) 2^-16.  So
+// 1/2 + 2^-7 leaves a margin of 10 over the rounding terms.  The absolute
+// term covers scales in the subnormal range.
+constexpr float Q8_BOUND = 0.5f + 1.0f / 128.0f;
+constexpr float Q8_ABS_BOUND = 1e-30f;
 
 struct SelectParams {
     const void* q;
     const float* cent;
-    const __nv_bfloat16* cent_lp;
+    const int8_t* cent_q;       // [U, Cmax, D] int8 scoring copy of cent
+    const float* cent_qs;       // [U, Cmax] its row scales
     float* scores;              // [U, Cmax] upper bound of each score (first pass)
     int32_t* hist;              // [U, SEL_HBINS]
     unsigned long long* gkey;   // [U, npow_max] scratch for large candidate sets
@@ -110,71 +115,53 @@ __device__ int block_scan_inplace(int* a, int n, int* s_warp) {
     return total;
 }
 
-// Raw bf16 row part of a lane (E elements, 2E bytes), kept packed until used.
-template <int E> struct RawPart;
-template <> struct RawPart<8> {
-    uint4 w;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint4*>(p); }
-    __device__ __forceinline__ void zero() { w = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[8]) const {
-        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-        x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
-    }
-};
-template <> struct RawPart<16> {
-    uint4 w0, w1;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
-        w0 = reinterpret_cast<const uint4*>(p)[0];
-        w1 = reinterpret_cast<const uint4*>(p)[1];
-    }
-    __device__ __forceinline__ void zero() { w0 = w1 = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[16]) const {
-        const uint32_t v[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            x[2 * i] = bf16_lo(v[i]);
-            x[2 * i + 1] = bf16_hi(v[i]);
-        }
-    }
-};
-template <> struct RawPart<32> {
-    uint4 w[4];
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = reinterpret_cast<const uint4*>(p)[i];
-    }
-    __device__ __forceinline__ void zero() {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    __device__ __forceinline__ void unpack(float (&x)[32]) const {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t v[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                x[8 * i + 2 * k] = bf16_lo(v[k]);
-                x[8 * i + 2 * k + 1] = bf16_hi(v[k]);
-            }
-        }
-    }
-};
-template <> struct RawPart<4> {
-    uint2 w;
-    __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = *reinterpret_cast<const uint2*>(p); }
-    __device__ __forceinline__ void zero() { w = make_uint2(0u, 0u); }
+// A lane's E int8 codes of a row (E bytes), kept packed until used.
+__device__ __forceinline__ float q8_byte(uint32_t w, int k) {  // signed byte k of w
+    return (float)((int)(w << (24 - 8 * k)) >> 24);
+}
+template <int E> struct Q8Part;
+template <> struct Q8Part<4> {
+    uint32_t w;
+    __device__ __forceinline__ void load(const int8_t* p) { w = *reinterpret_cast<const uint32_t*>(p); }
+    __device__ __forceinline__ void zero() { w = 0u; }
     __device__ __forceinline__ void unpack(float (&x)[4]) const {
-        x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = q8_byte(w, k);
+    }
+};
+template <> struct Q8Part<8> {
+    uint2 w;
+    __device__ __forceinline__ void load(const int8_t* p) { w = *reinterpret_cast<const uint2*>(p); }
+    __device__ __forceinline__ void zero() { w = make_uint2(0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[8]) const {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            x[k] = q8_byte(w.x, k);
+            x[4 + k] = q8_byte(w.y, k);
+        }
+    }
+};
+template <> struct Q8Part<16> {
+    uint4 w;
+    __device__ __forceinline__ void load(const int8_t* p) { w = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void zero() { w = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void unpack(float (&x)[16]) const {
+        const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[4 * i + k] = q8_byte(v[i], k);
     }
 };
 
-// First-pass scores of this block's (up to) SCORE_ROWS centres of unit u:
-// a warp owns SCORE_ROWS / SEL_WARPS consecutive rows, a half-warp every
-// other one; all of a lane's row parts are loaded (packed) before any is
-// used, so each warp keeps SCORE_ROWS / SEL_WARPS bf16 rows in flight.
-// One query head per graph: SC_LPR lanes per row (D/SC_LPR elements each),
-// so a warp instruction covers 32/SC_LPR rows and a row's sums take
-// log2(SC_LPR) shuffle levels.
+// First-pass scores of this block's (up to) SCORE_ROWS centres of unit u,
+// from the int8 copy: a warp owns SCORE_ROWS / SEL_WARPS consecutive rows;
+// all of a lane's row parts (and the rows' scales) are loaded before any is
+// used, so each warp keeps its rows in flight.  The score is
+// s~ = s_c (q . code_c) / sqrt(d) and its bound e = Q8_BOUND s_c |q|_1 / sqrt(d).
+// One query head per graph: SC_LPR lanes per row (D/SC_LPR codes each, one
+// 16-byte load for d = 128), so a warp instruction covers 32/SC_LPR rows and
+// a row's sum takes log2(SC_LPR) shuffle levels.
 constexpr int SC_LPR = 8;
 template <typename T, int D>
 __device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int C) {
@@ -186,56 +173,66 @@ __device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int
     const int oct = lane / SC_LPR, l8 = lane % SC_LPR;
     const int row0 = blockIdx.x * SCORE_ROWS_GQ1 + warp * RW;
     if (row0 >= C) return;
-    RawPart<E> raw[RQ];
+    Q8Part<E> raw[RQ];
+    float rs[RQ];
+    int wv[RQ];  // sizes, for the histogram
 #pragma unroll
     for (int j = 0; j < RQ; ++j) {
         const int c = row0 + GR * j + oct;
-        if (c < C) raw[j].load(p.cent_lp + ((size_t)u * p.Cmax + c) * D + l8 * E);
-        else raw[j].zero();
+        if (c < C) {
+            raw[j].load(p.cent_q + ((size_t)u * p.Cmax + c) * D + l8 * E);
+            rs[j] = p.cent_qs[(size_t)u * p.Cmax + c];
+            wv[j] = p.cnt[(size_t)u * p.Cmax + c];
+        } else {
+            raw[j].zero();
+            rs[j] = 0.f;
+            wv[j] = 0;
+        }
     }
-    const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
     const int b = u / p.G, g = u - b * p.G;
-    float qr[E];
+    float qr[E], qn = 0.f;
     {
         const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + g) * D + l8 * E;  // head g
 #pragma unroll
-        for (int e = 0; e < E; ++e) qr[e] = to_f32(qp[e]);
+        for (int e = 0; e < E; ++e) {
+            qr[e] = to_f32(qp[e]);
+            qn += fabsf(qr[e]);
+        }
     }
+#pragma unroll
+    for (int o = SC_LPR / 2; o >= 1; o >>= 1) qn += __shfl_xor_sync(FULL, qn, o);  // |q|_1
+    const float ebase = Q8_BOUND * qn * p.inv_sqrt_d;
     int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
 #pragma unroll
     for (int j = 0; j < RQ; ++j) {
         float x[E];
         raw[j].unpack(x);
-        float a = 0.f, m = 0.f;
+        float a = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            a = fmaf(qr[e], x[e], a);
-            m = fmaf(fabsf(qr[e]), fabsf(x[e]), m);
-        }
+        for (int e = 0; e < E; ++e) a = fmaf(qr[e], x[e], a);
 #pragma unroll
-        for (int o = SC_LPR / 2; o >= 1; o >>= 1) {
-            a += __shfl_xor_sync(FULL, a, o);
-            m += __shfl_xor_sync(FULL, m, o);
-        }
-        const float sc = a * p.inv_sqrt_d;
-        // |exact score - sc| <= 2^-8 m / sqrt(d) (see LP_REL_BOUND)
-        const float err = fmaf(LP_REL_BOUND, m * p.inv_sqrt_d, LP_ABS_BOUND);
+        for (int o = SC_LPR / 2; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+        const float sc = a * rs[j] * p.inv_sqrt_d;
+        const float err = fmaf(ebase, rs[j], Q8_ABS_BOUND);
         const int c = row0 + GR * j + oct;
-        const int w = __shfl_sync(FULL, wc, GR * j + oct);
         if (l8 == 0 && c < C) {
             p.scores[(size_t)u * p.Cmax + c] = sc + err;
-            if (w > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), w);
+            if (wv[j] > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), wv[j]);
         }
     }
 }
 
-// Several query heads per graph with a bf16 q: both products on the tensor
-// cores (mma.sync m16n8k16), heads as the A rows (padded with zeros), eight
-// communities per n-tile as the B columns, loaded straight from global
-// memory in fragment order: S = Q C~^T and the bound's M = |Q| |C~|^T, whose
-// operands are the same registers with the sign bits cleared.  A warp takes
-// two n-tiles (16 communities); the 4 lanes of quad 0 then hold, per
-// community, the max over the group's heads of both.
+// Several query heads per graph with a bf16 q: the products on the tensor
+// cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), heads as the A rows
+// (padded with zeros), eight communities per n-tile as the B columns.  The
+// int8 codes are exact in bf16, so S = Q code^T is the same sum as in the
+// one-head path.  Lane (g, tq) owns dims [LB tq, LB tq + LB) of its rows
+// (LB = D/4 bytes, one or two 16-byte loads) and of its head's q; k-step kk
+// takes dims LB tq + 4kk .. +3 of every lane, which the fragment sees as
+// k = 2tq, 2tq + 1 (register b0 / a0) and 2tq + 8, 2tq + 9 (b1 / a2): the
+// same map on both operands, and over the k-steps every dim once.  A warp
+// takes two n-tiles (16 communities); the 4 lanes of quad 0 then hold, per
+// community, the max over the group's heads.
 __device__ __forceinline__ void mma_sc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -244,66 +241,91 @@ __device__ __forceinline__ void mma_sc(float (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(0u), "r"(a1), "r"(0u), "r"(b0), "r"(b1));
 }
 
+// two signed bytes of w (k, k + 1) as a bf16 pair, low half first (exact)
+__device__ __forceinline__ uint32_t q8_pair_bf16(uint32_t w, int k) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(q8_byte(w, k), q8_byte(w, k + 1));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <int D, int GQ>
 __device__ __forceinline__ void score_rows_mma(const SelectParams& p, int u, int C) {
-    constexpr int KS = D / 16;
+    constexpr int KS = D / 16;   // k-steps
+    constexpr int LB = D / 4;    // dims (bytes of codes) per lane and row
+    constexpr int NV = LB / 16;  // 16-byte loads per lane and row
     constexpr int RW = SCORE_ROWS / SEL_WARPS;  // 16 communities per warp
-    static_assert(RW == 16, "two n-tiles of 8 per warp");
-    constexpr uint32_t ABS = 0x7fff7fffu;
+    static_assert(RW == 16 && KS == LB / 4, "two n-tiles of 8 per warp; 4 dims per lane and k-step");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, tq = lane & 3;
     const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
     if (row0 >= C) return;
-    // B fragments of both n-tiles: community row0 + 8t + g, dims kk*16 + 2tq (+8)
-    uint32_t bf[2][KS][2];
+    // codes of both n-tiles (community row0 + 8t + g) and the scales of the
+    // four communities whose results this lane ends up holding (2tq + e)
+    uint4 bw[2][NV];
+    float rs[2][2];
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const int c = row0 + 8 * t + g;
-        const __nv_bfloat16* row = p.cent_lp + ((size_t)u * p.Cmax + min(c, C - 1)) * D + 2 * tq;
+        const int8_t* row = p.cent_q + ((size_t)u * p.Cmax + min(c, C - 1)) * D + LB * tq;
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-            const uint32_t x0 = *reinterpret_cast<const uint32_t*>(row + kk * 16);
-            const uint32_t x1 = *reinterpret_cast<const uint32_t*>(row + kk * 16 + 8);
-            bf[t][kk][0] = c < C ? x0 : 0u;
-            bf[t][kk][1] = c < C ? x1 : 0u;
+        for (int v = 0; v < NV; ++v) {
+            const uint4 x = reinterpret_cast<const uint4*>(row)[v];
+            bw[t][v] = c < C ? x : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int ce = row0 + 8 * t + 2 * tq + e;
+            rs[t][e] = ce < C ? p.cent_qs[(size_t)u * p.Cmax + ce] : 0.f;
         }
     }
     const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
     const int b = u / p.G, gg = u - b * p.G;
     const int h0 = gg * GQ;  // per-group graphs (several heads)
-    uint32_t qa[KS][2];
+    // this lane's dims of head g's q (bf16 pairs), and |q_g|_1 over the quad
+    uint32_t qa[LB / 2];
+    float qn = 0.f;
     {
-        const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + h0 + min(g, GQ - 1)) * D + 2 * tq;
+        const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + h0 + min(g, GQ - 1)) * D + LB * tq;
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-            const uint32_t x0 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16);
-            const uint32_t x1 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 8);
-            qa[kk][0] = g < GQ ? x0 : 0u;
-            qa[kk][1] = g < GQ ? x1 : 0u;
+        for (int v = 0; v < LB / 8; ++v) {
+            const uint4 x = reinterpret_cast<const uint4*>(qrow)[v];
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                qa[4 * v + k] = g < GQ ? xs[k] : 0u;
+                qn += fabsf(bf16_lo(qa[4 * v + k])) + fabsf(bf16_hi(qa[4 * v + k]));
+            }
         }
     }
+    qn += __shfl_xor_sync(FULL, qn, 1);
+    qn += __shfl_xor_sync(FULL, qn, 2);
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) qn = fmaxf(qn, __shfl_xor_sync(FULL, qn, o));  // max over heads
+    const float ebase = Q8_BOUND * qn * p.inv_sqrt_d;
     int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, macc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t wd[4 * NV];  // code word kk: dims LB tq + 4kk .. +3
 #pragma unroll
-        for (int kk = 0; kk < KS; ++kk) {
-            mma_sc(sacc, qa[kk][0], qa[kk][1], bf[t][kk][0], bf[t][kk][1]);
-            mma_sc(macc, qa[kk][0] & ABS, qa[kk][1] & ABS, bf[t][kk][0] & ABS, bf[t][kk][1] & ABS);
+        for (int v = 0; v < NV; ++v) {
+            wd[4 * v] = bw[t][v].x;
+            wd[4 * v + 1] = bw[t][v].y;
+            wd[4 * v + 2] = bw[t][v].z;
+            wd[4 * v + 3] = bw[t][v].w;
         }
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk)
+            mma_sc(sacc, qa[2 * kk], qa[2 * kk + 1], q8_pair_bf16(wd[kk], 0), q8_pair_bf16(wd[kk], 2));
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             // max over the group's heads (rows g < GQ)
-            float sv = g < GQ ? sacc[e] : -INFINITY, mv = g < GQ ? macc[e] : 0.f;
+            float sv = g < GQ ? sacc[e] : -INFINITY;
 #pragma unroll
-            for (int o = 4; o <= 16; o <<= 1) {
-                sv = fmaxf(sv, __shfl_xor_sync(FULL, sv, o));
-                mv = fmaxf(mv, __shfl_xor_sync(FULL, mv, o));
-            }
+            for (int o = 4; o <= 16; o <<= 1) sv = fmaxf(sv, __shfl_xor_sync(FULL, sv, o));
             const int r = 8 * t + 2 * tq + e;  // community row within the warp's 16
             const int w = __shfl_sync(FULL, wc, r);
-            const float sc = sv * p.inv_sqrt_d;
-            const float err = fmaf(LP_REL_BOUND, mv * p.inv_sqrt_d, LP_ABS_BOUND);
+            const float sc = sv * rs[t][e] * p.inv_sqrt_d;
+            const float err = fmaf(ebase, rs[t][e], Q8_ABS_BOUND);
             const int c = row0 + r;
             if (g == 0 && c < C) {
                 p.scores[(size_t)u * p.Cmax + c] = sc + err;
@@ -330,44 +352,49 @@ __device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) 
     const int half = lane >> 4, l16 = lane & 15;
     const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
     if (row0 >= C) return;
-    RawPart<E> raw[RH];
+    Q8Part<E> raw[RH];
+    float rs[RH];
 #pragma unroll
     for (int j = 0; j < RH; ++j) {
         const int c = row0 + 2 * j + half;
-        if (c < C) raw[j].load(p.cent_lp + ((size_t)u * p.Cmax + c) * D + l16 * E);
-        else raw[j].zero();
+        if (c < C) {
+            raw[j].load(p.cent_q + ((size_t)u * p.Cmax + c) * D + l16 * E);
+            rs[j] = p.cent_qs[(size_t)u * p.Cmax + c];
+        } else {
+            raw[j].zero();
+            rs[j] = 0.f;
+        }
     }
     const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
     const int b = u / p.G, g = u - b * p.G;
     const int h0 = p.per_head ? g : g * GQ;
-    float qr[GQ][E];
+    float qr[GQ][E], qn[GQ];
 #pragma unroll
-    for (int h = 0; h < GQ; ++h)
+    for (int h = 0; h < GQ; ++h) {
         load_row_part<T, E>(static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h0 + h) * D + l16 * E, qr[h]);
+        qn[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) qn[h] += fabsf(qr[h][e]);
+    }
+    // max over the heads of |q_h|_1
+    const float ebase = Q8_BOUND * halfwarp_max_over_heads<GQ>(halfwarp_reduce_heads<GQ>(qn, lane)) * p.inv_sqrt_d;
 
     int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
 #pragma unroll
     for (int j = 0; j < RH; ++j) {
         float x[E];
         raw[j].unpack(x);
-        float part[GQ], mag[GQ];
+        float part[GQ];
 #pragma unroll
         for (int h = 0; h < GQ; ++h) {
-            float a = 0.f, m = 0.f;
+            float a = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                a = fmaf(qr[h][e], x[e], a);
-                m = fmaf(fabsf(qr[h][e]), fabsf(x[e]), m);
-            }
+            for (int e = 0; e < E; ++e) a = fmaf(qr[h][e], x[e], a);
             part[h] = a;
-            mag[h] = m;
         }
         float s = halfwarp_reduce_heads<GQ>(part, lane);
-        s = halfwarp_max_over_heads<GQ>(s) * p.inv_sqrt_d;
-        float m = halfwarp_reduce_heads<GQ>(mag, lane);
-        m = halfwarp_max_over_heads<GQ>(m) * p.inv_sqrt_d;
-        // |exact score - s| <= 2^-8 m (see LP_REL_BOUND)
-        const float err = fmaf(LP_REL_BOUND, m, LP_ABS_BOUND);
+        s = halfwarp_max_over_heads<GQ>(s) * rs[j] * p.inv_sqrt_d;
+        const float err = fmaf(ebase, rs[j], Q8_ABS_BOUND);
         const int c = row0 + 2 * j + half;
         const int w = __shfl_sync(FULL, wc, 2 * j + half);
         if (l16 == 0 && c < C) {
@@ -827,7 +854,8 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     SelectParams p{};
     p.q = q;
     p.cent = g.cent;
-    p.cent_lp = g.cent_lp;
+    p.cent_q = g.cent_q;
+    p.cent_qs = g.cent_qs;
     p.scores = reinterpret_cast<float*>(w + l.scores);
     p.hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + WS_RESERVED);  // zero on entry
     p.gkey = reinterpret_cast<unsigned long long*>(w + l.gkey);

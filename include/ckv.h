@@ -64,7 +64,7 @@ extern "C" {
 #define CKV_API
 #endif
 
-#define CKV_ABI_VERSION 3
+#define CKV_ABI_VERSION 4
 #define CKV_NEIGHBOURS 8
 
 typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
@@ -125,10 +125,14 @@ typedef struct {
  *   tok      int32 [U, T_cap]   members sorted by (community, position)
  *   cnt      int32 [U, Cmax]    member count, including tail members
  *   cent     fp32  [U, Cmax, d] running-mean centre of each community
- *   cent_lp  bf16  [U, Cmax, d] cent rounded to nearest, kept in step by the
- *                  build and the update: the scoring streams it (half the
- *                  bytes) and re-scores only the communities whose bounds
- *                  reach the budget cut from cent (see ckv_score_select)
+ *   cent_q   int8  [U, Cmax, d] cent quantised per row: with
+ *                  s = max_i |cent_i| / 127 (fp32 division), cent_q_i =
+ *                  round-half-even(cent_i / s), 0 where s = 0
+ *   cent_qs  fp32  [U, Cmax]    that row scale s
+ *                  Both are kept in step with cent by the build and the
+ *                  update.  The scoring streams them (a quarter of cent's
+ *                  bytes) and re-scores from cent only the communities whose
+ *                  score bounds reach the budget cut (see ckv_score_select)
  *   num_comm int32 [U]          1 + largest community id present
  *   tail_tok, tail_comm int32 [U, max_tail]  tokens joined after the build
  *   tail_len int32 [U]
@@ -149,7 +153,8 @@ typedef struct {
     int32_t* tok;
     int32_t* cnt;
     float* cent;
-    uint16_t* cent_lp;  /* bf16 bits [U, Cmax, d]: cent rounded, for the first scoring pass */
+    int8_t* cent_q;     /* [U, Cmax, d] cent quantised per row, for the first scoring pass */
+    float* cent_qs;     /* [U, Cmax] the rows' quantisation scales */
     int32_t* num_comm;
     int32_t* tail_tok;
     int32_t* tail_comm;
@@ -208,9 +213,10 @@ CKV_API ckv_status ckv_build_centroids(const ckv_cache_desc* cache, const int32_
  *           longest ranked prefix whose cnt sum is <= budget, and at least the
  *           top community; the sinks come on top of the budget.
  * Writes every field of `sel`.  budget >= 0.  The pass over all communities
- * reads the bf16 copy cent_lp with a rigorous error bound per score; only
- * the communities whose bound reaches the budget cut are re-scored from the
- * fp32 cent, so the selection is the one the fp32 scores give.
+ * reads the int8 copy (cent_q, cent_qs) with a rigorous error bound per score
+ * (|q . (cent - s cent_q)| <= s |q|_1 / 2 plus rounding); only the
+ * communities whose bound reaches the budget cut are re-scored from the fp32
+ * cent, so the selection is the one the fp32 scores give.
  */
 CKV_API ckv_status ckv_score_select(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
                             const void* q, int32_t budget, const ckv_selection_desc* sel,

@@ -66,7 +66,7 @@ def _cache(**kw):
 
 def _graph(**kw):
     g = dict(mode=0, S=4, Cmax=128, max_tail=16, T_cap=4096)
-    for i, f in enumerate(["comm_of", "offs", "tok", "cnt", "cent", "cent_lp", "num_comm", "tail_tok",
+    for i, f in enumerate(["comm_of", "offs", "tok", "cnt", "cent", "cent_q", "cent_qs", "num_comm", "tail_tok",
                            "tail_comm", "tail_len", "dev_err"]):
         g[f] = FAKE + (i + 2) * (1 << 28)
     g.update(kw)
@@ -131,8 +131,10 @@ CASES = [
                                                               ctypes.byref(_graph(assign_rule=-1)), 5, FAKE, FAKE,
                                                               None), INVALID),
     ("null graph array", lambda: _call_build(_cache(), _graph(cent=None)), INVALID),
-    ("null cent_lp", lambda: _call_build(_cache(), _graph(cent_lp=None)), INVALID),
-    ("misaligned cent_lp", lambda: _call_build(_cache(), _graph(cent_lp=FAKE + 8)), MISALIGNED),
+    ("null cent_q", lambda: _call_build(_cache(), _graph(cent_q=None)), INVALID),
+    ("null cent_qs", lambda: _call_build(_cache(), _graph(cent_qs=None)), INVALID),
+    ("misaligned cent_q", lambda: _call_build(_cache(), _graph(cent_q=FAKE + 8)), MISALIGNED),
+    ("misaligned cent_qs", lambda: _call_build(_cache(), _graph(cent_qs=FAKE + 4)), MISALIGNED),
     ("too many units", lambda: _call_build(_cache(B=400), _graph(mode=1)), UNSUPPORTED),
     ("null labels", lambda: _call_build(_cache(), _graph(), labels=None), INVALID),
     ("T > T_cap", lambda: _call_build(_cache(), _graph(), T=5000, stride=5000), CAPACITY),

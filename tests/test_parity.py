@@ -274,23 +274,39 @@ def test_fused_decode_append_matches_separate_calls():
                 assert torch.equal(getattr(a.st.graph, name), getattr(b.st.graph, name)), (wl.key, name)
 
 
+def _int8_copy(cent: torch.Tensor):
+    """The scoring copy's definition, in float32 numpy (IEEE divisions): per
+    row s = max |c| / 127, code = round-half-even(c / s), 0 for an all-zero
+    row."""
+    c = cent.cpu().numpy()
+    s = np.abs(c).max(axis=-1) / np.float32(127.0)
+    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    codes = np.where(s[..., None] > 0, np.rint(c / safe[..., None]), 0.0)
+    return (torch.from_numpy(np.clip(codes, -127, 127).astype(np.int8)).to(cent.device),
+            torch.from_numpy(s.astype(np.float32)).to(cent.device))
+
+
 def test_scoring_copy_tracks_centres():
-    """cent_lp is cent rounded to bf16 (round to nearest even), after the
+    """(cent_q, cent_qs) is cent quantised per row, bit for bit, after the
     build and after every update."""
-    wl = small("cent_lp", 42, steps=3)
-    case = Case(wl)
-    assert torch.equal(case.st.graph.cent_lp, case.st.graph.cent.to(torch.bfloat16))
-    for _ in range(wl.steps):
-        case.step(wl.budget)
-        assert torch.equal(case.st.graph.cent_lp, case.st.graph.cent.to(torch.bfloat16))
+    for wl in (small("cent_q", 42, steps=3), small("cent_q_f32_d64", 48, dtype="f32", d=64, mode="head",
+                                                  Hq=8, Hkv=4, steps=3)):
+        case = Case(wl)
+        for i in range(wl.steps + 1):
+            if i:
+                case.step(wl.budget)
+            codes, s = _int8_copy(case.st.graph.cent)
+            assert torch.equal(case.st.graph.cent_qs, s), (wl.key, i)
+            assert torch.equal(case.st.graph.cent_q, codes), (wl.key, i)
 
 
-def test_cut_among_scores_closer_than_bf16():
-    """Every community's keys are one vector scaled by 1 + 1e-4 * id, so
-    neighbouring communities' scores differ by ~1e-3, far below what the bf16
-    scoring pass resolves (~2e-2) and far above the 1e-5 tie band: the exact
-    re-scoring alone decides the ranking and the cut, which must equal the
-    oracle's."""
+def test_cut_among_scores_closer_than_the_int8_pass():
+    """Every community's keys are v + 1e-4 id w (v, w fixed per graph), so
+    neighbouring communities' scores differ by ~1e-4, far below what the int8
+    scoring pass resolves (its codes barely change from one community to the
+    next; its bounds are ~1e-1 wide) and far above the 1e-5 tie band: the
+    exact re-scoring alone decides the ranking and the cut, which must equal
+    the oracle's."""
     wl = small("near_ties", 43, dtype="f32", B=1, T=3000, budgets=(1000,), steps=1, update=False)
     case = Case(wl)
     q = synth.draw_queries(wl, case.draw, 0)
@@ -299,7 +315,8 @@ def test_cut_among_scores_closer_than_bf16():
     for g in range(wl.G):
         lab = torch.from_numpy(labels[0, g].astype(np.int64)).cuda()
         v = q[0, g * gq].float()
-        rows = v[None, :] * (1.0 + 1e-4 * lab.clamp(min=0).float())[:, None]
+        w = torch.roll(v, 1)
+        rows = v[None, :] + (1e-4 * lab.clamp(min=0).float())[:, None] * w[None, :]
         keep = lab < 0  # sinks keep their keys
         case.st.K[0, g, : wl.T] = torch.where(keep[:, None], case.st.K[0, g, : wl.T], rows)
     case.st.build(torch.from_numpy(labels.reshape(case.U, wl.T).astype(np.int32)).cuda(), wl.T)
