@@ -208,27 +208,28 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     sync();
     const int best = s_best;
     if (best < 0 || warp != 0) return;
-    // running mean: c <- c + (k - c) / (n + 1), from the copy of the centre
+    // running mean: c <- c + (k - c) / (n + 1) (as (k - c) * (1/(n + 1)) + c,
+    // one rounding more than a division), from the copy of the centre
     // taken while scoring
     const size_t row = (size_t)u * p.Cmax + best;
     float* cr = p.cent + row * D + lane * E;
     const float* c0r = s_row[s_bi] + lane * E;
-    const float denom = (float)(s_n + 1);
+    const float inv_n1 = __frcp_rn((float)(s_n + 1));  // one reciprocal, then products
     float c1[E], amax = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const float c0 = c0r[e];
-        c1[e] = c0 + (kx[e] - c0) / denom;
+        c1[e] = fmaf(kx[e] - c0, inv_n1, c0);
         cr[e] = c1[e];
         amax = fmaxf(amax, fabsf(c1[e]));
     }
     // the int8 scoring copy follows the centre: new scale, new codes
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-    const float sc = q8_scale(amax);
+    const float sc = q8_scale(amax), rc = q8_recip(amax);
     uint32_t packed = 0;
 #pragma unroll
-    for (int e = 0; e < E; ++e) packed |= (uint32_t)(q8_code(c1[e], sc) & 0xff) << (8 * e);
+    for (int e = 0; e < E; ++e) packed |= (uint32_t)(q8_code(c1[e], rc) & 0xff) << (8 * e);
     int8_t* qr = p.cent_q + row * D + lane * E;
     if constexpr (E == 4) *reinterpret_cast<uint32_t*>(qr) = packed;
     else *reinterpret_cast<uint16_t*>(qr) = (uint16_t)packed;

@@ -183,8 +183,8 @@ __global__ void __launch_bounds__(256) build_mean(BuildParams p) {
     float amax = s_amax[0];
 #pragma unroll
     for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_amax[w]);
-    const float sc = q8_scale(amax);
-    if (threadIdx.x < D) p.cent_q[((size_t)u * p.Cmax + c) * D + threadIdx.x] = (int8_t)q8_code(m, sc);
+    const float sc = q8_scale(amax), rc = q8_recip(amax);
+    if (threadIdx.x < D) p.cent_q[((size_t)u * p.Cmax + c) * D + threadIdx.x] = (int8_t)q8_code(m, rc);
     if (threadIdx.x == 0) p.cent_qs[(size_t)u * p.Cmax + c] = sc;
 }
 

@@ -59,14 +59,14 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162flo
 
 // ---------------------------------------------------------------------------
 // The int8 scoring copy of a centre row: scale s = max_i |c_i| / 127 and code
-// round-half-even(c_i / s) (0 for an all-zero row), both divisions IEEE.
-// |c_i - s code_i| <= s (1/2 + 2^-17): the quotient's rounding adds at most
-// 127 ulp(1)/2 to the half unit of the integer rounding.
+// round-half-even(c_i * r) with r = 127 / max_i |c_i| (both divisions IEEE,
+// the product fp32; 0 for an all-zero row).  c_i r is within 127 * 2^-23 of
+// c_i / s, so |c_i - s code_i| <= s (1/2 + 2^-16).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float q8_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f; }
-__device__ __forceinline__ int q8_code(float c, float s) {
-    if (!(s > 0.f)) return 0;
-    return max(-127, min(127, __float2int_rn(__fdiv_rn(c, s))));
+__device__ __forceinline__ float q8_recip(float amax) { return amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f; }
+__device__ __forceinline__ int q8_code(float c, float r) {
+    return max(-127, min(127, __float2int_rn(c * r)));
 }
 
 // ---------------------------------------------------------------------------

@@ -52,7 +52,7 @@ constexpr int SEL_HBINS = HIST_BINS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
 // Bound on |fp32 score from cent - fp32 score from the int8 copy| per unit
 // of s_c |q|_1 / sqrt(d) (s_c the row's scale): the codes contribute at most
-// 1/2 + 2^-17 (see q8_scale); the fp32 dot products, of depth <= 19 over
+// 1/2 + 2^-16 (see q8_scale); the fp32 dot products, of depth <= 19 over
 // terms summing to at most 127 |q|_1 (codes) or 127 s_c |q|_1 (fp32 centre),
 // about 2^-12.8 and 2^-13.8; the products by s_c and 1/sqrt(d) 2^-16.  So
 // 1/2 + 2^-7 leaves a margin of 10 over the rounding terms.  The absolute

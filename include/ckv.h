@@ -126,8 +126,9 @@ typedef struct {
  *   cnt      int32 [U, Cmax]    member count, including tail members
  *   cent     fp32  [U, Cmax, d] running-mean centre of each community
  *   cent_q   int8  [U, Cmax, d] cent quantised per row: with
- *                  s = max_i |cent_i| / 127 (fp32 division), cent_q_i =
- *                  round-half-even(cent_i / s), 0 where s = 0
+ *                  s = max_i |cent_i| / 127 and r = 127 / max_i |cent_i|
+ *                  (fp32 divisions), cent_q_i = round-half-even(cent_i * r)
+ *                  (fp32 product), 0 where s = 0
  *   cent_qs  fp32  [U, Cmax]    that row scale s
  *                  Both are kept in step with cent by the build and the
  *                  update.  The scoring streams them (a quarter of cent's

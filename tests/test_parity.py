@@ -275,13 +275,14 @@ def test_fused_decode_append_matches_separate_calls():
 
 
 def _int8_copy(cent: torch.Tensor):
-    """The scoring copy's definition, in float32 numpy (IEEE divisions): per
-    row s = max |c| / 127, code = round-half-even(c / s), 0 for an all-zero
-    row."""
+    """The scoring copy's definition, in float32 numpy (IEEE arithmetic): per
+    row s = max |c| / 127, r = 127 / max |c|, code = round-half-even(c * r),
+    0 for an all-zero row."""
     c = cent.cpu().numpy()
-    s = np.abs(c).max(axis=-1) / np.float32(127.0)
-    safe = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
-    codes = np.where(s[..., None] > 0, np.rint(c / safe[..., None]), 0.0)
+    amax = np.abs(c).max(axis=-1)
+    s = amax / np.float32(127.0)
+    r = np.float32(127.0) / np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    codes = np.where(amax[..., None] > 0, np.rint(c * r[..., None]), 0.0)
     return (torch.from_numpy(np.clip(codes, -127, 127).astype(np.int8)).to(cent.device),
             torch.from_numpy(s.astype(np.float32)).to(cent.device))
 
