@@ -107,7 +107,7 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     __shared__ float s_score[CKV_NEIGHBOURS];
     __shared__ int s_cnt[CKV_NEIGHBOURS];
     __shared__ float s_row[CKV_NEIGHBOURS][D];  // candidate centres, reused by the update
-    __shared__ int s_best, s_bi, s_n, s_tl;
+    __shared__ int s_tl;
     const int lane = tid & 31, warp = tid >> 5;
     const int b = u / p.G, g = u - b * p.G;
     const int gq = p.Hq / p.Hkv;
@@ -165,38 +165,43 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
         if (lane == 0) s_score[i] = use ? s : -INFINITY;
     }
     sync();
-    if (tid == 0) {
-        // each distinct candidate carries its score at its first slot; under
-        // the vote rule the number of slots naming it comes first
-        int best = -1, bi = -1, bv = 0;
-        float bs = -INFINITY;
-        for (int i = 0; i < CKV_NEIGHBOURS; ++i) {
-            const int ci = s_cand[i];
-            if (ci < 0 || s_score[i] == -INFINITY) continue;
-            int v = 0;
-            if (p.vote) {
-                for (int j = i; j < CKV_NEIGHBOURS; ++j) v += s_cand[j] == ci;
-            }
-            if (best < 0 || v > bv || (v == bv && (s_score[i] > bs || (s_score[i] == bs && ci < best)))) {
-                best = ci;
-                bi = i;
-                bv = v;
-                bs = s_score[i];
-            }
+    if (warp != 0) return;  // warp 0 picks the winner and updates its row
+    // Lane i < 8 holds slot i.  Each distinct candidate carries its score at
+    // its first slot; the winner is the largest (votes, score, -id), votes
+    // (the slots naming the community) counting only under the vote rule:
+    // one 64-bit key per lane, reduced over the warp.  The slot rides in the
+    // low bits below the id, which is unique among the keys.
+    unsigned long long key = 0ull;  // 0: no candidate
+    if (lane < CKV_NEIGHBOURS) {
+        const int ci = s_cand[lane];
+        const float sc = s_score[lane];
+        const unsigned same = __match_any_sync(0xffu, ci);  // lanes 0..7 naming the same community
+        if (ci >= 0 && sc != -INFINITY) {
+            const unsigned v = p.vote ? (unsigned)__popc(same) : 0u;
+            unsigned b = __float_as_uint(sc + 0.0f);  // -0 ranks as +0
+            b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+            key = ((unsigned long long)v << 60) | ((unsigned long long)b << 16) |
+                  ((unsigned long long)(MAX_CMAX - 1 - ci) << 3) | (unsigned long long)lane;
         }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const unsigned long long k2 = __shfl_xor_sync(FULL, key, o);
+        key = k2 > key ? k2 : key;
+    }
+    int best = key ? MAX_CMAX - 1 - (int)((key >> 3) & 0x1fffu) : -1;
+    const int bi = (int)(key & 7u);
+    if (best >= 0 && s_tl >= p.max_tail) {
+        if (lane == 0) atomicOr(p.dev_err, CKV_DEVERR_TAIL_FULL);
+        best = -1;
+    }
+    const int n = best >= 0 ? s_cnt[bi] : 0;  // written by the candidate's warp above
+    if (lane == 0) {
         int32_t* cpos = p.comm_of + (size_t)u * p.T_cap + p.pos;
-        if (best >= 0 && s_tl >= p.max_tail) {
-            atomicOr(p.dev_err, CKV_DEVERR_TAIL_FULL);
-            best = -1;
-        }
-        s_best = best;
-        s_bi = bi;
         if (best < 0) {
             *cpos = -1;
             if (p.assigned) p.assigned[u] = -1;
         } else {
-            const int n = s_cnt[bi];  // read by the candidate's warp above
-            s_n = n;
             p.cnt[(size_t)u * p.Cmax + best] = n + 1;
             *cpos = best;
             p.tail_tok[(size_t)u * p.max_tail + s_tl] = p.pos;
@@ -205,16 +210,14 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
             if (p.assigned) p.assigned[u] = best;
         }
     }
-    sync();
-    const int best = s_best;
-    if (best < 0 || warp != 0) return;
+    if (best < 0) return;
     // running mean: c <- c + (k - c) / (n + 1) (as (k - c) * (1/(n + 1)) + c,
     // one rounding more than a division), from the copy of the centre
     // taken while scoring
     const size_t row = (size_t)u * p.Cmax + best;
     float* cr = p.cent + row * D + lane * E;
-    const float* c0r = s_row[s_bi] + lane * E;
-    const float inv_n1 = __frcp_rn((float)(s_n + 1));  // one reciprocal, then products
+    const float* c0r = s_row[bi] + lane * E;
+    const float inv_n1 = __frcp_rn((float)(n + 1));  // one reciprocal, then products
     float c1[E], amax = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
