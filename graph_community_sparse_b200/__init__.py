@@ -74,7 +74,7 @@ class GraphDesc(ctypes.Structure):
 
 class SelectionDesc(ctypes.Structure):
     _fields_ = [("tok_cap", _i32), ("sel_comm", _p), ("n_sel", _p), ("sel_tok", _p), ("n_tok", _p),
-                ("unit_prefix", _p)]
+                ("tok_prefix", _p), ("tail_sel", _p), ("unit_prefix", _p)]
 
 
 _P = ctypes.POINTER
@@ -176,6 +176,8 @@ class Selection:
     n_sel: torch.Tensor
     sel_tok: torch.Tensor
     n_tok: torch.Tensor
+    tok_prefix: torch.Tensor
+    tail_sel: torch.Tensor
     unit_prefix: torch.Tensor
 
 
@@ -209,9 +211,11 @@ def new_selection(cache: CacheDesc, graph: Graph, tok_cap: int, device="cuda") -
     i32 = dict(dtype=torch.int32, device=device)
     t = dict(sel_comm=torch.zeros((U, Cmax), **i32), n_sel=torch.zeros((U,), **i32),
              sel_tok=torch.zeros((U, tok_cap), **i32), n_tok=torch.zeros((U,), **i32),
+             tok_prefix=torch.zeros((U, Cmax + 1), **i32),
+             tail_sel=torch.zeros((U, max(graph.desc.max_tail, 1)), **i32),
              unit_prefix=torch.zeros((U + 1,), **i32))
     desc = SelectionDesc(tok_cap, *(t[k].data_ptr() for k in ("sel_comm", "n_sel", "sel_tok", "n_tok",
-                                                               "unit_prefix")))
+                                                               "tok_prefix", "tail_sel", "unit_prefix")))
     return Selection(desc, **t)
 
 

@@ -91,7 +91,7 @@ ckv_status check_graph(const ckv_cache_desc* c, const ckv_graph_desc* g) {
 
 ckv_status check_sel(const ckv_graph_desc* g, const ckv_selection_desc* s, int64_t U) {
     if (!s) return fail(CKV_ERR_INVALID_ARG, "selection descriptor is NULL");
-    if (!s->sel_comm || !s->n_sel || !s->sel_tok || !s->n_tok || !s->unit_prefix)
+    if (!s->sel_comm || !s->n_sel || !s->sel_tok || !s->n_tok || !s->tok_prefix || !s->tail_sel || !s->unit_prefix)
         return fail(CKV_ERR_INVALID_ARG, "a selection array pointer is NULL");
     if (s->tok_cap < 1 || s->tok_cap < g->S) return fail(CKV_ERR_INVALID_ARG, "tok_cap must be >= max(S, 1)");
     if (U * (int64_t)s->tok_cap > (int64_t)1 << 30)
@@ -156,6 +156,8 @@ ckv::SelView sel_view(const ckv_selection_desc* s) {
     v.sel_tok = s->sel_tok;
     v.n_tok = s->n_tok;
     v.unit_prefix = s->unit_prefix;
+    v.tok_prefix = s->tok_prefix;
+    v.tail_sel = s->tail_sel;
     return v;
 }
 

@@ -219,6 +219,8 @@ struct SelView {
     int32_t* sel_tok;
     int32_t* n_tok;
     int32_t* unit_prefix;
+    int32_t* tok_prefix;
+    int32_t* tail_sel;
 };
 
 // workspace carving

@@ -82,6 +82,8 @@ struct SelectParams {
     int32_t* sel_tok;
     int32_t* n_tok;
     int32_t* unit_prefix;
+    int32_t* tok_prefix;        // [U, Cmax + 1] run offsets of the list
+    int32_t* tail_sel;          // [U, max(max_tail, 1)] communities of the list's tail part
     int Hq, G, per_head;
     float inv_sqrt_d;
     int U, Cmax, npow_max, S, T_cap, max_tail, tok_cap, budget;
@@ -672,6 +674,12 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     // tokens of the selected runs; their inclusive prefix (the small path
     // ranked it already)
     const int nb = small ? (kstar > 0 ? s_bsz[kstar - 1] : 0) : block_scan_inplace(bsz, kstar, s_warp);
+    {
+        // the runs' offsets in the list, for callers (and the attention's
+        // update) that map a list entry back to its community
+        int32_t* tp = p.tok_prefix + (size_t)u * (p.Cmax + 1);
+        for (int k = tid; k <= kstar; k += nt) tp[k] = k ? bsz[k - 1] : 0;
+    }
 
     int32_t* out = p.sel_tok + (size_t)u * p.tok_cap;
     const int32_t* tk = p.tok + (size_t)u * p.T_cap;
@@ -753,6 +761,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
             const int off = block_exclusive_scan(in, s_warp, &total);
             if (in) {
                 const int dst = base + off;
+                p.tail_sel[(size_t)u * max(p.max_tail, 1) + (dst - p.S - nb)] = tc[i];
                 if (dst < p.tok_cap) out[dst] = tt[i];
                 else overflow = true;
             }
@@ -873,6 +882,8 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     p.sel_tok = s.sel_tok;
     p.n_tok = s.n_tok;
     p.unit_prefix = s.unit_prefix;
+    p.tok_prefix = s.tok_prefix;
+    p.tail_sel = s.tail_sel;
     p.Hq = c.Hq;
     p.G = g.G;
     p.per_head = g.mode == CKV_GRAPH_PER_HEAD;

@@ -64,7 +64,7 @@ extern "C" {
 #define CKV_API
 #endif
 
-#define CKV_ABI_VERSION 4
+#define CKV_ABI_VERSION 5
 #define CKV_NEIGHBOURS 8
 
 typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
@@ -173,6 +173,14 @@ typedef struct {
  *                                   community in rank order, then its tail
  *                                   members
  *   n_tok       int32 [U]           length of each sel_tok row
+ *   tok_prefix  int32 [U, Cmax+1]   the list's runs: the build-time members of
+ *                                   sel_comm[k] are entries [S + tok_prefix[k],
+ *                                   S + tok_prefix[k+1]) of sel_tok;
+ *                                   tok_prefix[0] = 0 (values before any
+ *                                   truncation to tok_cap)
+ *   tail_sel    int32 [U, max(max_tail, 1)]  the community of each tail
+ *                                   member in the list, in list order (list
+ *                                   entries from S + tok_prefix[n_sel] on)
  *   unit_prefix int32 [U+1]         exclusive prefix sum of n_tok, written by
  *                                   ckv_sparse_decode (its work split)
  * tok_cap >= T_cap can never overflow; tok_cap >= S + max(budget, largest
@@ -184,6 +192,8 @@ typedef struct {
     int32_t* n_sel;
     int32_t* sel_tok;
     int32_t* n_tok;
+    int32_t* tok_prefix;
+    int32_t* tail_sel;
     int32_t* unit_prefix;
 } ckv_selection_desc;
 

@@ -159,6 +159,8 @@ class Case:
         sel_tok = self.st.sel.sel_tok.cpu().numpy()
         n_tok = self.st.sel.n_tok.cpu().numpy()
         prefix = self.st.sel.unit_prefix.cpu().numpy()
+        tok_prefix = self.st.sel.tok_prefix.cpu().numpy()
+        tail_sel = self.st.sel.tail_sel.cpu().numpy()
         nbr = self.st.nbr8.cpu().numpy()
         cnt_gpu = self.st.graph.cnt.cpu().numpy()
         assert prefix[0] == 0 and np.array_equal(np.diff(prefix), n_tok), "unit_prefix is not the scan of n_tok"
@@ -185,6 +187,15 @@ class Case:
             if not check_selection(gsel, scores, cnt, budget):
                 rep.band_selections += 1
             toks = O.token_set(gsel, members, wl.S)
+            # the list's runs: build-time member counts of the ranked
+            # communities, cumulated; then the tail members' communities in
+            # tail (position) order
+            T0 = wl.T
+            built = np.bincount(st.comm_of[wl.S: T0][st.comm_of[wl.S: T0] >= 0], minlength=self.Cmax)
+            runs = np.concatenate([[0], np.cumsum(built[gsel])]) if gsel else np.zeros(1, dtype=np.int64)
+            assert np.array_equal(tok_prefix[u, : len(gsel) + 1], runs), f"unit {u}: run offsets differ"
+            tails = [int(st.comm_of[t]) for t in range(T0, st.T) if int(st.comm_of[t]) in set(gsel)]
+            assert np.array_equal(tail_sel[u, : len(tails)], tails), f"unit {u}: tail communities differ"
             gt = sel_tok[u, : n_tok[u]]
             tok_cap = self.st.sel.desc.tok_cap
             if len(toks) <= tok_cap:

@@ -75,7 +75,7 @@ def _graph(**kw):
 
 def _sel(**kw):
     s = dict(tok_cap=4096)
-    for i, f in enumerate(["sel_comm", "n_sel", "sel_tok", "n_tok", "unit_prefix"]):
+    for i, f in enumerate(["sel_comm", "n_sel", "sel_tok", "n_tok", "tok_prefix", "tail_sel", "unit_prefix"]):
         s[f] = FAKE + (i + 20) * (1 << 28)
     s.update(kw)
     return ckv.SelectionDesc(**s)
@@ -148,6 +148,8 @@ CASES = [
     ("misaligned q", lambda: _call_select(_cache(), _graph(), _sel(), q=FAKE + 4), MISALIGNED),
     ("tok_cap < S", lambda: _call_select(_cache(), _graph(), _sel(tok_cap=2)), INVALID),
     ("null selection array", lambda: _call_select(_cache(), _graph(), _sel(unit_prefix=None)), INVALID),
+    ("null run offsets", lambda: _call_select(_cache(), _graph(), _sel(tok_prefix=None)), INVALID),
+    ("null tail communities", lambda: _call_decode(_cache(), _graph(), _sel(tail_sel=None)), INVALID),
     ("select ws small", lambda: _call_select(_cache(), _graph(), _sel(), ws_bytes=100), WORKSPACE),
     ("null out", lambda: _call_decode(_cache(), _graph(), _sel(), out=None), INVALID),
     ("misaligned out", lambda: _call_decode(_cache(), _graph(), _sel(), out=FAKE + 4), MISALIGNED),
