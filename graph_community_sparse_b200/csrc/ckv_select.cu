@@ -50,6 +50,7 @@ template <int GQ> struct ScoreBlockRows { static constexpr int v = GQ == 1 ? SCO
 constexpr int SEL_HBITS = HIST_BITS;
 constexpr int SEL_HBINS = HIST_BINS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
+constexpr int RANK_LOOP_MAX = 128;          // up to this many: quadratic ranking; more: sorting network
 // Bound on |fp32 score from cent - fp32 score from the int8 copy| per unit
 // of s_c |q|_1 / sqrt(d) (s_c the row's scale): the codes contribute at most
 // 1/2 + 2^-16 (see q8_scale); the fp32 dot products, of depth <= 19 over
@@ -115,6 +116,39 @@ __device__ int block_scan_inplace(int* a, int n, int* s_warp) {
     }
     __syncthreads();
     return total;
+}
+
+// Exclusive scan of one 64-bit value per thread over the block (s_w64: 33
+// entries of shared memory).
+__device__ unsigned long long block_exclusive_scan_u64(unsigned long long x, unsigned long long* s_w64) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    unsigned long long inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(FULL, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_w64[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const unsigned long long w = lane < nw ? s_w64[lane] : 0ull;
+        unsigned long long wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(FULL, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nw) s_w64[lane] = wi - w;
+    }
+    __syncthreads();
+    return s_w64[warp] + inc - x;
+}
+
+// The token copy reads a selected run next: start fetching its first lines
+// into L2.
+__device__ __forceinline__ void prefetch_run(const int32_t* run, int len) {
+    const int lines = min((len + 31) >> 5, 8);
+    for (int l = 0; l < lines; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(run + 32 * l));
 }
 
 // A lane's E int8 codes of a row (E bytes), kept packed until used.
@@ -586,27 +620,79 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     int* bsz = small ? s_bsz : p.gw + (size_t)u * p.npow_max;
     if (small) {
         bool in = false;
-        if (tid < nc) {
-            const unsigned long long k = s_key[tid];
-            const int w = s_w[tid];
-            // rank, the size ranked above (for the cut) and the run length
-            // ranked above (the run's place in the token list)
-            int rank = 0, above = 0, above_len = 0;
-            for (int j = 0; j < nc; ++j) {
-                const bool gt = s_key[j] > k;
-                rank += gt;
-                above += gt ? s_w[j] : 0;
-                above_len += gt ? s_len[j] : 0;
+        if (nc <= RANK_LOOP_MAX) {  // uniform over the block
+            if (tid < nc) {
+                const unsigned long long k = s_key[tid];
+                const int w = s_w[tid];
+                // rank, the size ranked above (for the cut) and the run length
+                // ranked above (the run's place in the token list)
+                int rank = 0, above = 0, above_len = 0;
+                for (int j = 0; j < nc; ++j) {
+                    const bool gt = s_key[j] > k;
+                    rank += gt;
+                    above += gt ? s_w[j] : 0;
+                    above_len += gt ? s_len[j] : 0;
+                }
+                in = above + w <= p.budget;
+                s_runs[rank] = k;
+                s_bsz[rank] = above_len + (o1 - o0);  // inclusive prefix in rank order
+                s_ofs[rank] = o0;
+                if (in || rank == 0) prefetch_run(p.tok + (size_t)u * p.T_cap + o0, o1 - o0);
             }
-            in = above + w <= p.budget;
-            s_runs[rank] = k;
-            s_bsz[rank] = above_len + (o1 - o0);  // inclusive prefix in rank order
-            s_ofs[rank] = o0;
-            if (in || rank == 0) {
-                // the token copy reads this run next: start fetching it into L2
-                const int32_t* run = p.tok + (size_t)u * p.T_cap + o0;
-                const int lines = min((o1 - o0 + 31) >> 5, 8);
-                for (int l = 0; l < lines; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(run + 32 * l));
+        } else {
+            // More candidates than the quadratic ranking pays for: the exact
+            // keys are sorted best first in registers, a thread per entry, by
+            // a bitonic network over next_pow2(nc) entries (partners in the
+            // same warp exchange by shuffles, across warps through shared
+            // memory); the low bits of a sort key carry the candidate's slot
+            // next to its id, which keeps the tie order (lower id first).
+            // One scan in rank order then gives the sizes and run lengths
+            // ranked above each entry.
+            __shared__ int s_o0[SEL_FAST];
+            __shared__ unsigned long long s_w64[33];
+            static_assert(SEL_FAST <= 256 && MAX_CMAX <= (1 << 24), "slot and id fit the key's low 32 bits");
+            unsigned long long v = 0;  // below every real key
+            if (tid < nc) {
+                const unsigned long long k = s_key[tid];
+                s_o0[tid] = o0;
+                v = (k & 0xffffffff00000000ull) | ((unsigned long long)(MAX_CMAX - 1 - key_id(k)) << 8) |
+                    (unsigned long long)tid;
+            }
+            int npow = 32;
+            while (npow < nc) npow <<= 1;
+            for (int k = 2; k <= npow; k <<= 1) {
+                for (int j = k >> 1; j > 0; j >>= 1) {
+                    unsigned long long o;
+                    if (j >= 32) {  // uniform over the block
+                        s_key[tid] = v;  // each thread read only its own entry above
+                        __syncthreads();
+                        o = s_key[tid ^ j];
+                        __syncthreads();
+                    } else {
+                        o = __shfl_xor_sync(FULL, v, j);
+                    }
+                    const unsigned long long hi = v > o ? v : o, lo = v > o ? o : v;
+                    v = (((tid & k) == 0) == ((tid & j) == 0)) ? hi : lo;
+                }
+            }
+            int w = 0, len = 0, slot = 0;
+            if (tid < nc) {
+                slot = (int)(v & 0xffu);
+                w = s_w[slot];
+                len = s_len[slot];
+            }
+            // sizes and run lengths are each at most T_cap < 2^31: one 64-bit scan
+            const unsigned long long pre =
+                block_exclusive_scan_u64(((unsigned long long)w << 32) | (unsigned)len, s_w64);
+            if (tid < nc) {
+                const int above = (int)(pre >> 32), above_len = (int)(pre & 0xffffffffu);
+                const int id = MAX_CMAX - 1 - (int)((v >> 8) & 0xffffffu);
+                const int o0r = s_o0[slot];
+                in = above + w <= p.budget;
+                s_runs[tid] = (v & 0xffffffff00000000ull) | (unsigned long long)(0xffffffffu - (unsigned)id);
+                s_bsz[tid] = above_len + len;  // inclusive prefix in rank order
+                s_ofs[tid] = o0r;
+                if (in || tid == 0) prefetch_run(p.tok + (size_t)u * p.T_cap + o0r, len);
             }
         }
         kstar = __syncthreads_count(in);

@@ -249,6 +249,22 @@ def test_many_candidates_global_sort(budget_frac):
     assert int(case.st.sel.n_sel.max().item()) > 256
 
 
+@pytest.mark.parametrize("budget", [6000, 9000])
+def test_candidates_between_the_two_rankings(budget):
+    """Between 129 and 256 candidates: the selection ranks them with its
+    sorting network instead of the quadratic loop (one head per graph, ~65
+    tokens per community; by the oracle these budgets select 61-155 and
+    101-206 communities in the four graphs)."""
+    T = 40000
+    wl = small(f"mid_cand_{budget}", 49, B=1, Hq=4, Hkv=1, T=T, mode="head", budgets=(budget,), steps=2,
+               update=True)
+    case = Case(wl)
+    for _ in range(wl.steps):
+        case.step(wl.budget)
+    n_sel = case.st.sel.n_sel.cpu().numpy()
+    assert n_sel.max() > 128 and n_sel.max() <= 230, n_sel
+
+
 def test_fused_decode_append_matches_separate_calls():
     """ckv_sparse_decode_append (update run by the merge kernel) gives the
     same outputs, neighbours, cache and graph state, bit for bit, as
