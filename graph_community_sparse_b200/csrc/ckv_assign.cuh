@@ -98,7 +98,7 @@ inline AssignParams make_assign_params(const CacheView& c, const GraphView& g, i
 // the unit's 8 neighbour positions (-1: none) in nbrpos, readable by all of
 // them.  sync() is a barrier over exactly these NW warps.  Candidates are
 // scored NW at a time, one warp each, so all their centres are fetched in
-// one or two rounds; one thread picks the winner; warp 0 moves its centre.
+// one or two rounds; warp 0 picks the winner and moves its centre.
 template <typename T, int D, int NW, typename Sync>
 __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const int* nbrpos, int tid, Sync sync) {
     constexpr int E = D / 32;
