@@ -265,6 +265,21 @@ def test_candidates_between_the_two_rankings(budget):
     assert n_sel.max() > 128 and n_sel.max() <= 230, n_sel
 
 
+def test_largest_community_count():
+    """Cmax = 8192 communities (the largest supported) of 1-3 tokens each in
+    one graph, with updates: the scoring grid's last row block is full, the
+    histogram and the re-scoring see every community, and the selection of
+    ~300 communities takes the global-memory sort."""
+    wl = small("max_comm", 50, B=1, Hq=4, Hkv=1, T=8192 * 2 + 4, sizes="multinomial", n_comm=8192,
+               min_size=1, budgets=(600,), steps=2, update=True)
+    case = Case(wl)
+    assert case.C == 8192 and case.Cmax == 8192
+    for _ in range(wl.steps):
+        case.step(wl.budget)
+    assert int(case.st.graph.dev_err.item()) == 0
+    assert int(case.st.sel.n_sel.max().item()) > 256
+
+
 def test_fused_decode_append_matches_separate_calls():
     """ckv_sparse_decode_append (update run by the merge kernel) gives the
     same outputs, neighbours, cache and graph state, bit for bit, as
