@@ -24,7 +24,8 @@
  *  - All pointers in the descriptors and arguments are DEVICE pointers owned
  *    by the caller, except the descriptors themselves (host structs, read
  *    during the call only).  The library keeps no pointer after returning.
- *  - Calls are asynchronous on `stream` and never synchronise the device;
+ *  - Calls are asynchronous on `stream` and never synchronise the device
+ *    (ckv_get_device_error, which reads the error word, excepted);
  *    they may be captured into a CUDA graph after one uncaptured call per
  *    device and kernel shape (the first call caches device attributes).
  *  - No call allocates device memory.  Scratch comes from the caller's

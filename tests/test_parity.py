@@ -376,3 +376,32 @@ def test_vote_rule_is_decisive_and_matches_oracle():
     assert any(not torch.equal(a, b) for a, b in zip(picks_v, picks_s))
     assert int(vote.st.graph.dev_err.item()) == 0
     print(rep)
+
+
+def test_cuda_graph_capture_replays_the_step():
+    """After one eager call, the selection and the attention can be captured
+    in a CUDA graph (no call allocates or synchronises, and the launches carry
+    their programmatic dependencies); replays with new queries in the
+    captured buffer give the eager results bit for bit."""
+    wl = small("graph_capture", 51, update=False, steps=3)
+    case = Case(wl)
+    st = case.st
+    qs = [synth.draw_queries(wl, case.draw, i) for i in range(wl.steps)]
+    eager = []
+    for q in qs:
+        st.decode(q, wl.budget)
+        eager.append((st.out.clone(), st.nbr8.clone(), st.sel.sel_tok.clone(), st.sel.n_tok.clone()))
+    q_static = qs[0].clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        st.decode(q_static, wl.budget)
+    for q, (out, nbr, tok, ntok) in zip(qs, eager):
+        q_static.copy_(q)
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(st.out, out) and torch.equal(st.nbr8, nbr)
+        assert torch.equal(st.sel.n_tok, ntok)
+        for u in range(st.U):  # the token lists (entries past n_tok are stale by design)
+            n = int(ntok[u])
+            assert torch.equal(st.sel.sel_tok[u, :n], tok[u, :n]), u
+    assert int(st.graph.dev_err.item()) == 0
