@@ -380,6 +380,23 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         nsel_hist.append(sum(L.st.sel.n_sel.long().sum() for L in layers))
     torch.cuda.synchronize()
     check_dev_err("timed steps")
+    # per-kernel durations: the library brackets each launch with CUDA events
+    # on its stream in a pass of its own (the events cost the programmatic
+    # overlap between a call's kernels, so neither the timed steps nor the
+    # per-call pass carry them)
+    import graph_community_sparse_b200 as ckv
+    ckv.ckv_kernel_times()  # drop anything recorded before
+    ckv.ckv_kernel_timing(True)
+    try:
+        for j in range(B_steps):
+            new_episode_if_due()
+            flush()
+            one_step(W_steps + K_steps + j)
+        torch.cuda.synchronize()
+    finally:
+        ckv.ckv_kernel_timing(False)
+    ktimes = ckv.ckv_kernel_times()
+    check_dev_err("kernel timing pass")
     drift = assignment_drift(layers, wl, wl.T) if wl.update else None
     # per step, summed over the layers: each selection from the previous
     # layer's attention end (or the step start), each attention from its
@@ -435,14 +452,38 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
                                             for e in bevs])) * 1e3, 2) for li in range(n_layers)],
             "attn_us": [round(float(np.mean([e[1 + 2 * li].elapsed_time(e[2 + 2 * li]) for e in bevs])) * 1e3, 2)
                         for li in range(n_layers)]}
-    dom = max((dec_name, "ckv_score_select"), key=lambda k: kernels[k]["ms"])
-    roofline = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": peak, "unit": "GB/s",
-                "frac": kernels[dom]["GB/s"] / peak, "peak_source": peak_src,
-                "traffic": profile_traffic(dom, wl.key) if n_layers == 1 else None,
-                "bytes_per_launch": kernels[dom]["bytes"] / n_layers,
-                "timing": "CUDA events around the library call on its stream, mean over a pass of "
-                          f"{B_steps} steps right after the timed ones{per} (the timed steps carry no "
-                          "events between calls, which would break the programmatic-launch chain)"}
+    # the kernels one by one (per step, summed over the layers): the attention
+    # kernel's algorithmic bytes are the distinct selected K/V rows, their
+    # indices, q and (with neighbours) the logit of every list entry; the
+    # split-K partials it writes for the merge are not algorithmic
+    attn_bytes = rows * row_bytes + ntok * 4 + q_bytes + (ntok * 4 if wl.update else 0)
+    per_kernel = {}
+    for kind, (tot_ms, nlaunch) in ktimes.items():
+        if nlaunch:
+            per_kernel[kind] = {"ms": tot_ms / B_steps, "launches_per_step": nlaunch / B_steps,
+                                "share": tot_ms / B_steps / float(np.mean(step_ms))}
+    if "attention" in per_kernel:
+        a = per_kernel["attention"]
+        a["bytes"] = float(np.mean(attn_bytes))
+        a["GB/s"] = a["bytes"] / (a["ms"] * 1e-3) / 1e9
+        a["frac"] = a["GB/s"] / peak
+    dom_kind = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
+    if dom_kind == "attention":
+        a = per_kernel["attention"]
+        roofline = {"kernel": "decode_main (the split-K attention kernel of " + dec_name + ")", "bound": "hbm",
+                    "achieved": a["GB/s"], "peak": peak, "unit": "GB/s", "frac": a["frac"], "peak_source": peak_src,
+                    "traffic": profile_traffic("decode_main", wl.key) if n_layers == 1 else None,
+                    "bytes_per_launch": a["bytes"] / n_layers,
+                    "timing": "CUDA events the library records around each launch (ckv_kernel_timing) on the "
+                              f"launching stream, mean over a pass of {B_steps} steps after the timed ones{per}"}
+    else:
+        dom = max((dec_name, "ckv_score_select"), key=lambda k: kernels[k]["ms"])
+        roofline = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": peak, "unit": "GB/s",
+                    "frac": kernels[dom]["GB/s"] / peak, "peak_source": peak_src,
+                    "traffic": profile_traffic(dom, wl.key) if n_layers == 1 else None,
+                    "bytes_per_launch": kernels[dom]["bytes"] / n_layers,
+                    "timing": "CUDA events around the library call on its stream, mean over a pass of "
+                              f"{B_steps} steps right after the timed ones{per}"}
 
     # dense comparator on the same caches and queries
     dense_out = torch.empty_like(st0.out)
@@ -543,6 +584,7 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "tokens_per_s": value * wl.B,
         "roofline": roofline,
         "kernels": kernels,
+        "per_kernel": per_kernel,
         "step_roofline": step_roofline,
         "per_layer": per_layer,
         "dense": dense,

@@ -21,7 +21,8 @@ __all__ = [
     "Graph", "Selection", "cache_desc", "new_graph", "new_selection", "new_workspace",
     "ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
     "ckv_sparse_decode_noalloc", "NOALLOC_SCRATCH_BYTES", "ckv_assign_update", "ckv_append_assign",
-    "ckv_sparse_decode_append", "ckv_get_device_error",
+    "ckv_sparse_decode_append", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times",
+    "KERNEL_KINDS",
     "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "ASSIGN_SCORE", "ASSIGN_VOTE",
@@ -38,9 +39,10 @@ PER_GROUP, PER_HEAD = 0, 1
 ASSIGN_SCORE, ASSIGN_VOTE = 0, 1
 DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
 NEIGHBOURS = 8
+KERNEL_KINDS = ("build", "score", "select", "attention", "merge", "update")
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
             "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
-            "ckv_get_device_error",
+            "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times",
             "ckv_dense_decode",
             "ckv_status_string", "ckv_last_error", "ckv_abi_version")
 NOALLOC_SCRATCH_BYTES = 32 << 20
@@ -89,9 +91,11 @@ lib.ckv_sparse_decode_append.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(Se
                                          _p, _p, _p, _sz, _p]
 lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
 lib.ckv_get_device_error.argtypes = [_P(GraphDesc), _p, _P(ctypes.c_int32), _i32]
+lib.ckv_kernel_timing.argtypes = [_i32]
+lib.ckv_kernel_times.argtypes = [_P(ctypes.c_float), _P(ctypes.c_int32), _i32]
 for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
            "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
-           "ckv_dense_decode", "ckv_get_device_error"):
+           "ckv_dense_decode", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times"):
     getattr(lib, _f).restype = ctypes.c_int
 lib.ckv_status_string.argtypes = [ctypes.c_int]
 lib.ckv_status_string.restype = ctypes.c_char_p
@@ -298,6 +302,20 @@ def ckv_sparse_decode_append(cache: CacheDesc, q: torch.Tensor, graph: Graph, se
                                         v_new.data_ptr(), _ptr(assigned), ws.data_ptr(), ws.numel(),
                                         _stream(stream)),
            "ckv_sparse_decode_append")
+
+
+def ckv_kernel_timing(enable: bool) -> None:
+    """Bracket every later launch with CUDA events (diagnostic; see ckv.h)."""
+    _check(lib.ckv_kernel_timing(int(bool(enable))), "ckv_kernel_timing")
+
+
+def ckv_kernel_times() -> dict:
+    """{kind: (total ms, launches)} of the launches timed since the last read."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_float * n)()
+    cnt = (ctypes.c_int32 * n)()
+    _check(lib.ckv_kernel_times(ms, cnt, n), "ckv_kernel_times")
+    return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
 
 
 def ckv_get_device_error(graph: Graph, reset: bool = False, stream=None) -> int:

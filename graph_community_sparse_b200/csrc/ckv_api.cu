@@ -173,6 +173,21 @@ extern "C" {
 
 int32_t ckv_abi_version(void) { return CKV_ABI_VERSION; }
 
+static_assert(ckv::KK_COUNT == CKV_KERNEL_KINDS && ckv::KK_ATTENTION == CKV_KERNEL_ATTENTION &&
+                  ckv::KK_UPDATE == CKV_KERNEL_UPDATE,
+              "kernel kinds match the header");
+
+ckv_status ckv_kernel_timing(int32_t enable) {
+    ckv::timing_set(enable != 0);
+    return ok();
+}
+
+ckv_status ckv_kernel_times(float* total_ms, int32_t* launches, int32_t n) {
+    if (!total_ms || !launches) return fail(CKV_ERR_INVALID_ARG, "total_ms or launches is NULL");
+    if (n < CKV_KERNEL_KINDS) return fail(CKV_ERR_INVALID_ARG, "n = %d < %d kernel kinds", n, CKV_KERNEL_KINDS);
+    return cuda_status(ckv::timing_read(total_ms, launches), "ckv_kernel_times");
+}
+
 ckv_status ckv_get_device_error(const ckv_graph_desc* graph, ckv_stream_t stream, int32_t* code, int32_t reset) {
     if (!graph || !graph->dev_err) return fail(CKV_ERR_INVALID_ARG, "graph descriptor or its dev_err is NULL");
     if (!code) return fail(CKV_ERR_INVALID_ARG, "code is NULL");

@@ -760,9 +760,10 @@ cudaError_t launch_decode_t(DecodeParams p, cudaStream_t st) {
     int blocks = sms * per_sm;
     if (blocks * DEC_WARPS > MAX_DECODE_WARPS) blocks = MAX_DECODE_WARPS / DEC_WARPS;
     p.W = blocks * DEC_WARPS;
-    e = launch_pdl(kern, dim3(blocks), dim3(DEC_WARPS * 32), smem, st, p);
+    e = launch_pdl(KK_ATTENTION, kern, dim3(blocks), dim3(DEC_WARPS * 32), smem, st, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_merge<T, D, GQ, DENSE>, dim3(p.U), dim3(D + (DENSE ? 0 : 32 * NBR_WARPS)), 0, st, p);
+    return launch_pdl(KK_MERGE, decode_merge<T, D, GQ, DENSE>, dim3(p.U), dim3(D + (DENSE ? 0 : 32 * NBR_WARPS)),
+                      0, st, p);
 }
 
 template <bool DENSE>

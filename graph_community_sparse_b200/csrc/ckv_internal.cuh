@@ -285,9 +285,24 @@ inline size_t ws_head_bytes(int B, int Hq) { return WS_RESERVED + align256((size
 // 63 -> 71 us per call on a 128K-context batch of 8).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Diagnostic kernel timing (ckv_kernel_timing): while it is on, every
+// launch is bracketed by two CUDA events on its stream, and the durations are
+// summed per kind when they are read (ckv_kernel_times).  Off by default; the
+// events also cost the programmatic overlap between a call's kernels.
+enum KernelKind { KK_BUILD = 0, KK_SCORE, KK_SELECT, KK_ATTENTION, KK_MERGE, KK_UPDATE, KK_COUNT };
+bool timing_enabled();
+cudaError_t timing_mark(int kind, bool start, cudaStream_t st);
+void timing_set(bool on);
+cudaError_t timing_read(float* total_ms, int32_t* launches);
+
 template <typename... Params, typename... Args>
-inline cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                              Args&&... args) {
+inline cudaError_t launch_pdl(int kind, void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    const bool timed = timing_enabled();
+    if (timed) {
+        const cudaError_t e = timing_mark(kind, true, st);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
@@ -298,7 +313,9 @@ inline cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, si
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (timed && e == cudaSuccess) e = timing_mark(kind, false, st);
+    return e;
 }
 
 

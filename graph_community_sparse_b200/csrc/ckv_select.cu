@@ -933,9 +933,9 @@ template <typename T, int D, int GQ>
 cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
     constexpr int rows = ScoreBlockRows<GQ>::v;
     dim3 grid((p.Cmax + rows - 1) / rows, p.U);
-    cudaError_t e = launch_pdl(score_kernel<T, D, GQ>, grid, dim3(SEL_THREADS), 0, st, p);
+    cudaError_t e = launch_pdl(KK_SCORE, score_kernel<T, D, GQ>, grid, dim3(SEL_THREADS), 0, st, p);
     if (e != cudaSuccess) return e;
-    return launch_pdl(select_kernel<T, D, GQ>, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
+    return launch_pdl(KK_SELECT, select_kernel<T, D, GQ>, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
 }
 }  // namespace
 

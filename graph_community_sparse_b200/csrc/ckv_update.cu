@@ -25,11 +25,11 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
     if (p.U <= 0) return cudaSuccess;
     const dim3 grid(p.U), block(CKV_NEIGHBOURS * 32);
     if (c.dtype == CKV_DTYPE_BF16) {
-        if (c.d == 128) return launch_pdl(assign_kernel<__nv_bfloat16, 128>, grid, block, 0, st, p);
-        return launch_pdl(assign_kernel<__nv_bfloat16, 64>, grid, block, 0, st, p);
+        if (c.d == 128) return launch_pdl(KK_UPDATE, assign_kernel<__nv_bfloat16, 128>, grid, block, 0, st, p);
+        return launch_pdl(KK_UPDATE, assign_kernel<__nv_bfloat16, 64>, grid, block, 0, st, p);
     }
-    if (c.d == 128) return launch_pdl(assign_kernel<float, 128>, grid, block, 0, st, p);
-    return launch_pdl(assign_kernel<float, 64>, grid, block, 0, st, p);
+    if (c.d == 128) return launch_pdl(KK_UPDATE, assign_kernel<float, 128>, grid, block, 0, st, p);
+    return launch_pdl(KK_UPDATE, assign_kernel<float, 64>, grid, block, 0, st, p);
 }
 
 }  // namespace ckv

@@ -343,6 +343,28 @@ CKV_API ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, 
 CKV_API ckv_status ckv_get_device_error(const ckv_graph_desc* graph, ckv_stream_t stream, int32_t* code,
                                         int32_t reset);
 
+/*
+ * Diagnostic kernel timing; no result depends on it.  With enable != 0, every
+ * kernel that later calls on this host thread launch is bracketed by two
+ * CUDA events on its stream; ckv_kernel_times() waits for the recorded
+ * events and fills the HOST arrays total_ms[kind] (summed duration, ms) and
+ * launches[kind] for the launches since its previous call, then forgets
+ * them.  The events cost the programmatic overlap between a call's kernels,
+ * so time the step itself without them.  n < CKV_KERNEL_KINDS or NULL
+ * arrays: CKV_ERR_INVALID_ARG; a failed event call: CKV_ERR_CUDA.
+ */
+typedef enum {
+    CKV_KERNEL_BUILD = 0,      /* the four kernels of ckv_build_centroids, as one */
+    CKV_KERNEL_SCORE = 1,      /* first scoring pass (ckv_score_select) */
+    CKV_KERNEL_SELECT = 2,     /* selection and token list (ckv_score_select) */
+    CKV_KERNEL_ATTENTION = 3,  /* split-K attention (sparse and dense decode) */
+    CKV_KERNEL_MERGE = 4,      /* merge, neighbours and fused update */
+    CKV_KERNEL_UPDATE = 5      /* ckv_assign_update / ckv_append_assign */
+} ckv_kernel_kind;
+#define CKV_KERNEL_KINDS 6
+CKV_API ckv_status ckv_kernel_timing(int32_t enable);
+CKV_API ckv_status ckv_kernel_times(float* total_ms, int32_t* launches, int32_t n);
+
 CKV_API const char* ckv_status_string(ckv_status status);
 /* Message of the last failed call on this host thread ("" if none). */
 CKV_API const char* ckv_last_error(void);

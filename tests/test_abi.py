@@ -180,6 +180,9 @@ CASES = [
     ("dense ws", lambda: ckv.lib.ckv_dense_decode(ctypes.byref(_cache()), FAKE, 100, FAKE, FAKE, 8, None),
      WORKSPACE),
     ("null cache", lambda: ckv.lib.ckv_dense_decode(None, FAKE, 100, FAKE, FAKE, 1 << 40, None), INVALID),
+    ("kernel times null", lambda: ckv.lib.ckv_kernel_times(None, None, 6), INVALID),
+    ("kernel times short", lambda: ckv.lib.ckv_kernel_times((ctypes.c_float * 6)(), (ctypes.c_int32 * 6)(), 5),
+     INVALID),
     ("device error null graph", lambda: ckv.lib.ckv_get_device_error(None, None, ctypes.byref(ctypes.c_int32()), 0),
      INVALID),
     ("device error null code", lambda: ckv.lib.ckv_get_device_error(ctypes.byref(_graph()), None, None, 0), INVALID),
@@ -200,3 +203,12 @@ def test_python_binding_raises():
     with pytest.raises(ckv.CKVError) as e:
         ckv._check(UNSUPPORTED, "x")
     assert e.value.status == UNSUPPORTED
+
+
+def test_kernel_timing_is_host_side_until_used():
+    """Turning timing on and off and reading an empty record touch no device."""
+    assert ckv.lib.ckv_kernel_timing(1) == 0 and ckv.lib.ckv_kernel_timing(0) == 0
+    times = ckv.ckv_kernel_times()
+    assert list(times) == list(ckv.KERNEL_KINDS) and all(v == (0.0, 0) for v in times.values())
+    hdr = open(HEADER).read()
+    assert int(re.search(r"#define CKV_KERNEL_KINDS (\d+)", hdr).group(1)) == len(ckv.KERNEL_KINDS)
