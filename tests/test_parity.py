@@ -405,3 +405,25 @@ def test_cuda_graph_capture_replays_the_step():
             n = int(ntok[u])
             assert torch.equal(st.sel.sel_tok[u, :n], tok[u, :n]), u
     assert int(st.graph.dev_err.item()) == 0
+
+
+def test_kernel_timing_counts_each_launch():
+    """With timing on, one step records one launch of each of its kernels
+    (positive durations); with it off nothing more is recorded."""
+    wl = small("kernel_timing", 52, steps=1)
+    case = Case(wl)
+    q = synth.draw_queries(wl, case.draw, 0)
+    kn, vn = synth.draw_new_tokens(wl, case.draw, 0)
+    ckv.ckv_kernel_times()
+    ckv.ckv_kernel_timing(True)
+    try:
+        case.st.select(q, wl.budget)
+        case.st.attend_append(q, kn.to(case.st.K.dtype), vn.to(case.st.V.dtype))
+    finally:
+        ckv.ckv_kernel_timing(False)
+    t = ckv.ckv_kernel_times()
+    for kind in ("score", "select", "attention", "merge"):
+        assert t[kind][1] == 1 and t[kind][0] > 0.0, (kind, t[kind])
+    assert t["build"][1] == 0 and t["update"][1] == 0
+    case.st.select(q, wl.budget)
+    assert all(v[1] == 0 for v in ckv.ckv_kernel_times().values())
