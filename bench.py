@@ -459,7 +459,8 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     attn_bytes = rows * row_bytes + ntok * 4 + q_bytes + (ntok * 4 if wl.update else 0)
     per_kernel = {}
     for kind, (tot_ms, nlaunch) in ktimes.items():
-        if nlaunch:
+        # the episodes' rebuilds between steps are not part of the step
+        if nlaunch and kind != "build":
             per_kernel[kind] = {"ms": tot_ms / B_steps, "launches_per_step": nlaunch / B_steps,
                                 "share": tot_ms / B_steps / float(np.mean(step_ms))}
     if "attention" in per_kernel:
