@@ -96,3 +96,18 @@ def test_cpu_baseline_reports_single_and_all_core_oracle_rates():
     cb = bench.cpu_baseline(synth.WORKLOADS["tiny"], 128, torch.device("cpu"), 4)
     assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] > 0
     assert cb["all_cores"]["cores"] == (os.cpu_count() or 1) and cb["all_cores"]["value"] > 0
+
+
+def test_reference_arm_prints_one_contract_line(capsys):
+    """`bench.py --impl reference` (the CPU oracle) on the tiny workload: one
+    JSON line with the base contract's keys and the reference arm's."""
+    assert bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3"]) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
