@@ -25,14 +25,17 @@
 //    dependent: the lower-bound histogram gives a bin edge t with more than
 //    the budget's weight of communities certainly scoring >= t, so every
 //    selected community scores >= t; the candidates are the communities
-//    whose upper bound reaches t (typically a few dozen), and only they are
+//    whose upper bound reaches t (tens to a few hundred), and only they are
 //    re-scored exactly in fp32 from cent.  A non-candidate scores below t
-//    and so below every selected one, so ranking the candidates alone, each
-//    against the others in shared memory (which also gives the size above
-//    it and so the cut, at least the top community, with no sort), gives
-//    the exact selection.  Then the unit's token list: sinks, build-time
-//    members of each selected community (from the community-contiguous CSR),
-//    then the selected tail members.
+//    and so below every selected one, so ranking the candidates alone gives
+//    the exact selection: up to 128 each against the others in shared
+//    memory (which also gives the size ranked above it, so the cut needs no
+//    sort), more by a sorting network in registers and one scan, more than
+//    256 by a block-wide sort in global scratch; at least the top community
+//    is taken.  Then the unit's token list: sinks, build-time members of
+//    each selected community (from the community-contiguous CSR), then the
+//    selected tail members; and the runs' offsets and the tail entries'
+//    communities.
 // The histograms live in the workspace head: zero on entry, and each
 // selection block clears its unit's histogram after reading it.
 #include <math.h>
