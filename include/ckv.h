@@ -25,7 +25,8 @@
  *    by the caller, except the descriptors themselves (host structs, read
  *    during the call only).  The library keeps no pointer after returning.
  *  - Calls are asynchronous on `stream` and never synchronise the device
- *    (ckv_get_device_error, which reads the error word, excepted);
+ *    (ckv_get_device_error and the diagnostic ckv_kernel_times, which wait
+ *    for what they read, excepted);
  *    they may be captured into a CUDA graph after one uncaptured call per
  *    device and kernel shape (the first call caches device attributes).
  *  - No call allocates device memory.  Scratch comes from the caller's
@@ -106,8 +107,8 @@ typedef enum { CKV_ASSIGN_SCORE = 0, CKV_ASSIGN_VOTE = 1 } ckv_assign_rule;
  * The full KV cache of one layer: K and V are [B, Hkv, T_cap, d] with the d
  * elements of a row contiguous; strides are in elements and their byte
  * values must be multiples of 16 (as must the base pointers).  The library
- * only reads it, except ckv_append_assign, which writes row `pos` of K and V
- * and nothing else.  [R-A] paragraph 5: the cache stays whole so any
+ * only reads it, except ckv_append_assign and ckv_sparse_decode_append,
+ * which write row `pos` of K and V and nothing else.  [R-A] paragraph 5: the cache stays whole so any
  * fragment can be selected again later.
  */
 typedef struct {
@@ -302,7 +303,8 @@ CKV_API ckv_status ckv_assign_update(const ckv_cache_desc* cache, const ckv_grap
  * token's rows k_new and v_new (each [B, Hkv, d] in the cache dtype,
  * contiguous, 16-byte aligned) at position `pos` of K and V, then updates
  * every graph unit exactly as ckv_assign_update does, taking the new key from
- * k_new.  One launch; the only call that writes the cache, and only row pos
+ * k_new.  One launch; with ckv_sparse_decode_append the only calls that
+ * write the cache, and only row pos
  * (the selection of the step that produced nbr8 never holds pos, so no
  * read of this step races with the write).  0 <= pos < T_cap.
  */
