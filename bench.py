@@ -95,12 +95,13 @@ def measured_peaks():
 
 def csrc_digest() -> str:
     """sha256 over the library's kernel sources (every .cu and .cuh file but
-    the host-only argument checking in ckv_api.cu; names and contents, in name
-    order): any kernel or launch change alters it."""
+    the host-only ckv_api.cu (argument checks) and ckv_timing.cu (diagnostic
+    events); names and contents, in name order): any kernel or launch change
+    alters it."""
     d = os.path.join(ROOT, "graph_community_sparse_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")) and f != "ckv_api.cu":
+        if f.endswith((".cu", ".cuh", ".h")) and f not in ("ckv_api.cu", "ckv_timing.cu"):
             h.update(f.encode() + b"\0" + open(os.path.join(d, f), "rb").read())
     return h.hexdigest()
 

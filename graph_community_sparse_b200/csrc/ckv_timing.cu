@@ -46,13 +46,22 @@ cudaError_t timing_mark(int kind, bool start, cudaStream_t st) {
     e = cudaEventRecord(ev, st);
     if (e != cudaSuccess) return e;
     if (start) {
+        if (t_open) {  // a launch failed after its start mark: reuse that event
+            std::lock_guard<std::mutex> lk(g_mu);
+            g_pool.push_back(t_open);
+        }
         t_open = ev;
         t_open_kind = kind;
         return cudaSuccess;
     }
-    if (t_open && t_open_kind == kind) {
+    {
         std::lock_guard<std::mutex> lk(g_mu);
-        g_done.push_back(Mark{kind, t_open, ev});
+        if (t_open && t_open_kind == kind) {
+            g_done.push_back(Mark{kind, t_open, ev});
+        } else {  // no matching start: nothing to time
+            if (t_open) g_pool.push_back(t_open);
+            g_pool.push_back(ev);
+        }
     }
     t_open = nullptr;
     t_open_kind = -1;
