@@ -9,7 +9,9 @@ mutation tests at the end plant plausible mistakes in copies of the oracle's
 functions and check that some pin catches each one.
 """
 import itertools
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -17,6 +19,19 @@ import torch
 
 import oracle.ckv_oracle as O
 import synth
+
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")))
+
+
+def _num(x):
+    """A fixture number: floats as written, plus "ln3" and "-inf"."""
+    return {"ln3": math.log(3.0), "-inf": -math.inf}.get(x, x) if isinstance(x, str) else x
+
+
+def _arr(a):
+    return np.array([[_num(x) for x in row] for row in a] if a and isinstance(a[0], list) else [_num(x) for x in a],
+                    dtype=np.float64)
 
 
 def _sdpa(q, K, V):
@@ -40,21 +55,17 @@ def _random_graph(rng, T=160, S=4, C=7, d=16):
 # ----------------------------------------------------------------------------
 
 def check_attention_closed_form(attention):
-    # d = 4: q = (2,0,0,0); k1 = (ln 3,0,0,0) -> logit ln 3; k2 = 0 -> logit 0;
-    # weights 3/4, 1/4; o = 3/4 (1,0,0,0) + 1/4 (0,4,0,0) = (0.75, 1, 0, 0)
-    K = np.array([[math.log(3.0), 0, 0, 0], [0, 0, 0, 0]], dtype=np.float64)
-    V = np.array([[1, 0, 0, 0], [0, 4, 0, 0]], dtype=np.float64)
-    o = attention(np.array([2.0, 0, 0, 0]), K, V, np.array([0, 1]))
-    return np.allclose(o, [0.75, 1.0, 0.0, 0.0], atol=1e-14)
+    # tests/golden/worked_examples.json "attention" (worked by hand there)
+    g = GOLDEN["attention"]
+    o = attention(_arr(g["q"]), _arr(g["K"]), _arr(g["V"]), np.array(g["positions"]))
+    return np.allclose(o, _arr(g["out"]), atol=1e-14)
 
 
 def check_scores_closed_form(community_scores):
-    # d = 4, two heads; community 0: dots 2 and -1 -> max 2 -> 2/sqrt(4) = 1.0
-    # community 1: dots -2 and 3 -> 1.5; community 2 empty -> -inf
-    q = np.array([[2.0, 0, 0, 0], [0, -1.0, 0, 0]])
-    cent = np.array([[1.0, 1, 0, 0], [-1.0, -3, 0, 0], [5.0, 5, 5, 5]])
-    s = community_scores(q, cent, np.array([3, 2, 0]))
-    return s[0] == 1.0 and s[1] == 1.5 and s[2] == -np.inf
+    # tests/golden/worked_examples.json "scores" (worked by hand there)
+    g = GOLDEN["scores"]
+    s = community_scores(_arr(g["q"]), _arr(g["cent"]), np.array(g["cnt"]))
+    return bool(np.array_equal(s, _arr(g["scores"])))
 
 
 def _brute_select(scores, cnt, budget):
@@ -90,12 +101,10 @@ def check_select_bruteforce(select, trials=300, seed=3):
 
 
 def check_select_worked(select):
-    s = np.array([3.0, 1.0, 2.0, 2.0])
-    n = np.array([5, 4, 3, 2])
-    # rank: 0 (3), 2 (2, lower id), 3 (2), 1 (1); prefix sizes 5, 8, 10, 14
-    return (select(s, n, 10) == [0, 2, 3] and select(s, n, 9) == [0, 2]
-            and select(s, n, 4) == [0] and select(s, n, 14) == [0, 2, 3, 1]
-            and select(s, n, 0) == [0])
+    # tests/golden/worked_examples.json "select" (worked by hand there)
+    g = GOLDEN["select"]
+    s, n = _arr(g["scores"]), np.array(g["cnt"])
+    return all(list(select(s, n, budget)) == expect for budget, expect in g["cases"])
 
 
 def _brute_neighbours(q_heads, K, positions, S, k=8):
@@ -233,18 +242,13 @@ def test_assign_bruteforce_ties_and_one_update():
 def check_assign_vote(fn) -> bool:
     """The majority-vote rule: most frequent neighbour community, then the
     larger score, then the lower id; worked cases, then brute force."""
-    d = 4
-    cent = np.array([[1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0], [2, 0, 0, 0]], dtype=np.float64)
-    k = np.array([1.0, 0.5, 0.0, 0.0])
+    # tests/golden/worked_examples.json "assign_vote" (worked by hand there)
+    g = GOLDEN["assign_vote"]
+    cent = _arr(g["cent"])
+    d = cent.shape[1]
     ok = True
-    # worked by hand: votes {2: 3, 0: 2, 1: 2} -> 2 wins although its score (0) is the lowest
-    ok &= fn(k, cent, [2, 0, 2, 1, 0, 2, 1, -1]) == 2
-    # equal votes {0: 2, 3: 2}: scores 1/2 and 2/2 -> 3
-    ok &= fn(k, cent, [0, 3, 0, 3]) == 3
-    # equal votes and equal scores (cent[1] and cent[2] seen from k2) -> the lower id
-    k2 = np.array([0.0, 1.0, 1.0, 0.0])
-    ok &= fn(k2, cent, [2, 1]) == 1
-    ok &= fn(k, cent, [-1, -1]) == -1 and fn(k, cent, []) == -1
+    for kname, nb, expect in g["cases"]:
+        ok &= fn(_arr(g[kname]), cent, nb) == expect
     rng = np.random.default_rng(23)
     C = 6
     for _ in range(200):
