@@ -30,10 +30,14 @@ in that order:
    communities of the 8 non-sink selected tokens with the largest graph logit
    (max over the graph's heads of q_h . k_t / sqrt(d); ties to the lower
    position); the token joins the candidate c maximising k_new . c / sqrt(d)
-   (ties to the lower id).
+   (ties to the lower id), or, under the other reading (assign_vote), the
+   community holding the most of the 8 neighbours, ties to the larger
+   k_new . c / sqrt(d) and then the lower id.
 
 Every centre is recomputed from the member lists whenever it is needed; the
-oracle never updates a mean incrementally.  Pins: see tests/test_oracle.py.
+oracle never updates a mean incrementally.  Pins: see tests/test_oracle.py
+and the hand-worked cases in tests/golden/worked_examples.json; every
+function here has one.
 """
 from __future__ import annotations
 
