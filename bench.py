@@ -38,9 +38,9 @@ import synth  # noqa: E402
 METRIC = "sparse decode steps/s at 128K ctx; achieved HBM GB/s vs B200 peak"
 DEFAULT_WORKLOAD = "qwen3_8b_128k_head"
 FALLBACK_HBM_GBS = 6650.0
-# score, select, attention, merge (the update runs inside the merge kernel)
-KERNELS_PER_STEP_UPDATE = 4
-KERNELS_PER_STEP_STATIC = 4
+# score+select, attention, merge (the update runs inside the merge kernel)
+KERNELS_PER_STEP_UPDATE = 3
+KERNELS_PER_STEP_STATIC = 3
 
 
 # ----------------------------------------------------------------------------

@@ -312,9 +312,15 @@ ckv_status ckv_sparse_decode_noalloc(const ckv_cache_desc* cache, const void* q,
     size_t have = 0;
     cudaError_t e = ckv::static_decode_scratch(&scratch, &have);
     if (e != cudaSuccess) return cuda_status(e, "ckv_sparse_decode_noalloc: scratch address lookup");
-    return cuda_status(ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q,
-                                                 out, nbr8, scratch, nullptr, reinterpret_cast<cudaStream_t>(stream)),
-                       "ckv_sparse_decode_noalloc");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    e = ckv::launch_sparse_decode(cache_view(cache), graph_view(cache, graph), sel_view(sel), q, out, nbr8, scratch,
+                                  nullptr, st);
+    if (e != cudaSuccess) {
+        // a kernel enqueued before the failed launch may leave the head's
+        // counters nonzero; zero them so later calls start clean
+        (void)cudaMemsetAsync(scratch, 0, ckv::ws_head_bytes(cache->B, cache->Hq), st);
+    }
+    return cuda_status(e, "ckv_sparse_decode_noalloc");
 }
 
 ckv_status ckv_assign_update(const ckv_cache_desc* cache, const ckv_graph_desc* graph, int32_t pos,

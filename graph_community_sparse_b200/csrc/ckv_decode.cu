@@ -464,29 +464,6 @@ __device__ __forceinline__ int nbr_pos(unsigned long long k) {
     return 0x7fffffff - (int)(unsigned)(k & 0xffffffffu);
 }
 
-// Bitonic sort of one key per lane, descending across the warp.
-__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
-#pragma unroll
-    for (int k = 2; k <= 32; k <<= 1) {
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            const unsigned long long y = __shfl_xor_sync(FULL, x, j);
-            const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
-            x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
-        }
-    }
-    return x;
-}
-
-__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x) {
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        const unsigned long long y = __shfl_xor_sync(FULL, x, o);
-        x = x > y ? x : y;
-    }
-    return x;
-}
-
 // The fused community update of unit u by the merge block's NBR_WARPS
 // neighbour warps (thread xt of 32 NBR_WARPS), given its neighbour positions.
 template <typename T, int D>

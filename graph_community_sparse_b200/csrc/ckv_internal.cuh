@@ -85,6 +85,10 @@ __device__ __forceinline__ void cp_async_8(void* smem, const void* gmem, bool pr
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(s), "l"(gmem), "r"(sz)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async_4(void* smem, const void* gmem) {
+    unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
@@ -150,6 +154,29 @@ template <int GQ>
 __device__ __forceinline__ float halfwarp_max_over_heads(float x) {
 #pragma unroll
     for (int o = 16 >> Log2<GQ>::v; o <= 8; o <<= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
+    return x;
+}
+
+// Bitonic sort of one key per lane, descending across the warp.
+__device__ __forceinline__ unsigned long long warp_sort_desc(unsigned long long x, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(FULL, x, j);
+            const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
+            x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+        }
+    }
+    return x;
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(FULL, x, o);
+        x = x > y ? x : y;
+    }
     return x;
 }
 
@@ -226,13 +253,9 @@ struct SelView {
 // workspace carving
 // Workspace head, shared by every call on a workspace and zero before its
 // first use: the attention kernels' work ticket (WS_RESERVED bytes), then one
-// score histogram of HIST_BINS counters per possible graph unit (B * Hq).
-// Every call leaves the head zero (the attention's merge returns the ticket,
-// the selection clears each histogram after reading it).  The other parts of
-// each call start after the head.
+// arrival counter per possible graph unit (B * Hq ints).  Every call leaves
+// the head zero.  The other parts of each call start after the head.
 constexpr size_t WS_RESERVED = 256;
-constexpr int HIST_BITS = 12;
-constexpr int HIST_BINS = 1 << HIST_BITS;
 
 struct DecodeWs {
     int* ticket;   // dynamic chunk counter (the workspace's first bytes)
@@ -273,7 +296,7 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
                                  const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline size_t ws_head_bytes(int B, int Hq) { return WS_RESERVED + align256((size_t)B * Hq * HIST_BINS * 4); }
+inline size_t ws_head_bytes(int B, int Hq) { return WS_RESERVED + align256((size_t)B * Hq * 4); }
 
 // Programmatic dependent launch.  Kernels launched by launch_pdl() start
 // with pdl_wait(), so they read and write nothing before the previous kernel

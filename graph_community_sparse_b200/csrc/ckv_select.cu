@@ -1,4 +1,4 @@
-// Community scoring and budgeted selection for sm_100a.
+// Community scoring and budgeted selection for sm_100a, in one kernel.
 //
 // During generation each query is first matched against the community
 // centres alone, and only the chosen communities are then read from the KV
@@ -7,37 +7,34 @@
 // "The speed-up depends on how many graphs the model stores").
 //
 // The score is s_c = max over the graph's query heads of q_h . cent_c /
-// sqrt(d) in fp32, and the selection is exactly the one those scores give;
-// but the pass over every community streams the centres' int8 copy (codes
-// cent_q with one fp32 scale s_c per row, cent_qs), a quarter of the fp32
-// bytes:
-//  * score_kernel, grid (centre blocks of 128, units): a streaming
-//    matrix-vector product over the codes (16-byte loads; one query head:
-//    8 lanes per row; several heads: tensor cores for a bf16 q, else a
-//    half-warp per row with the value-exchanging butterfly of the attention
-//    kernel for the head sums) gives s~_c = s_c q . code_c / sqrt(d) and a
-//    rigorous bound e_c >= |s_c - s~_c| from s_c |q|_1 (Q8_BOUND).  The
-//    upper bound s~ + e is stored; the community's size is added, with a global atomic, to a
-//    per-unit histogram over the top 12 bits of the key of the lower bound
-//    s~ - e, key = (orderable score << 32) | ~id (unique; orders communities
-//    by score desc, id asc);
-//  * select_kernel, one block per unit, launched as a programmatic
-//    dependent: the lower-bound histogram gives a bin edge t with more than
-//    the budget's weight of communities certainly scoring >= t, so every
-//    selected community scores >= t; the candidates are the communities
-//    whose upper bound reaches t (tens to a few hundred), and only they are
-//    re-scored exactly in fp32 from cent.  A non-candidate scores below t
-//    and so below every selected one, so ranking the candidates alone gives
-//    the exact selection: up to 128 each against the others in shared
-//    memory (which also gives the size ranked above it, so the cut needs no
-//    sort), more by a sorting network in registers and one scan, more than
-//    256 by a block-wide sort in global scratch; at least the top community
-//    is taken.  Then the unit's token list: sinks, build-time members of
-//    each selected community (from the community-contiguous CSR), then the
-//    selected tail members; and the runs' offsets and the tail entries'
-//    communities.
-// The histograms live in the workspace head: zero on entry, and each
-// selection block clears its unit's histogram after reading it.
+// sqrt(d) in fp32, and the selection is exactly the one those scores give.
+// score_select_kernel: one block of SEL_THREADS per graph unit, all of its
+// state in shared memory, no global atomics and no kernel boundary:
+//  1. first pass over every community, streaming the centres' int8 copy
+//     (codes cent_q with one fp32 scale s_c per row, cent_qs: a quarter of
+//     the fp32 bytes).  The query of each head is split exactly into two
+//     int8 vectors, q ~ sq (128 hi + lo) with |q_i - sq (128 hi_i + lo_i)|
+//     <= 0.51 sq, so every product is an exact integer dot product (dp4a on
+//     the CUDA cores, 8 lanes per centre row, one 16-byte load per lane).
+//     That gives s~_c = s_c sq (q_int . code_c) / sqrt(d) and a rigorous
+//     bound e_c >= |s_c - s~_c| (Q8_BOUND, QSPLIT_BOUND).  Each community's
+//     upper bound s~ + e goes to shared memory, and its size is added to a
+//     shared 4096-bin histogram over the top 12 bits of the key of its lower
+//     bound s~ - e, key = (orderable score << 32) | ~id (unique; orders
+//     communities by score desc, id asc);
+//  2. the histogram gives a bin edge t with more than the budget's weight of
+//     communities certainly scoring >= t, so every selected community scores
+//     >= t; the candidates are the communities whose upper bound reaches t
+//     (tens to a few hundred), and only they are re-scored exactly in fp32
+//     from cent.  A non-candidate scores below t and so below every selected
+//     one, so ranking the candidates alone gives the exact selection: each
+//     warp sorts 32 of them and a candidate's rank (and the sizes ranked
+//     above it) is its place in its own run plus binary searches in the
+//     others; more than SEL_FAST candidates are sorted block-wide in global
+//     scratch; at least the top community is taken;
+//  3. the unit's token list: sinks, build-time members of each selected
+//     community (from the community-contiguous CSR), then the selected tail
+//     members; and the runs' offsets and the tail entries' communities.
 #include <math.h>
 #include <type_traits>
 
@@ -45,23 +42,30 @@
 
 namespace ckv {
 
-constexpr int SEL_WARPS = 8;
+constexpr int SEL_WARPS = 16;
 constexpr int SEL_THREADS = SEL_WARPS * 32;
-constexpr int SCORE_ROWS = SEL_WARPS * 16;      // centres per block (several heads per graph)
-constexpr int SCORE_ROWS_GQ1 = SEL_WARPS * 16;  // centres per block (one head per graph)
-template <int GQ> struct ScoreBlockRows { static constexpr int v = GQ == 1 ? SCORE_ROWS_GQ1 : SCORE_ROWS; };
-constexpr int SEL_HBITS = HIST_BITS;
-constexpr int SEL_HBINS = HIST_BINS;
+constexpr int SEL_HBITS = 12;
+constexpr int SEL_HBINS = 1 << SEL_HBITS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
-constexpr int RANK_LOOP_MAX = 128;          // up to this many: quadratic ranking; more: sorting network
+constexpr int SC_LPR = 8;                   // lanes per centre row in the first pass
+constexpr int SC_RPI = 32 / SC_LPR;         // rows per warp instruction
+template <int GQ> struct ScRq { static constexpr int v = GQ == 1 ? 8 : GQ == 2 ? 4 : 2; };  // row groups per lane in flight
+// Range of the integer query: q_i ~ sq Q_i with |Q_i| <= 127 * 128, so
+// Q_i = 128 hi_i + lo_i with hi_i in [-127, 127] and lo_i in [-64, 63].
+constexpr int Q_SPLIT = 127 * 128;
 // Bound on |fp32 score from cent - fp32 score from the int8 copy| per unit
 // of s_c |q|_1 / sqrt(d) (s_c the row's scale): the codes contribute at most
-// 1/2 + 2^-16 (see q8_scale); the fp32 dot products, of depth <= 19 over
-// terms summing to at most 127 |q|_1 (codes) or 127 s_c |q|_1 (fp32 centre),
-// about 2^-12.8 and 2^-13.8; the products by s_c and 1/sqrt(d) 2^-16.  So
-// 1/2 + 2^-7 leaves a margin of 10 over the rounding terms.  The absolute
-// term covers scales in the subnormal range.
+// 1/2 + 2^-16 (see q8_scale); the fp32 dot products of the exact re-score,
+// of depth <= 19 over terms summing to at most 127 s_c |q|_1, about 2^-13.8;
+// the conversion of the integer dot product and the products by sq, s_c and
+// 1/sqrt(d), relative 2^-22 of a value below 127 s_c (|q|_1 + d sq / 2),
+// about 2^-15.  So 1/2 + 2^-7 leaves a margin of 10 over the rounding terms.
 constexpr float Q8_BOUND = 0.5f + 1.0f / 128.0f;
+// The integer query: Q_i = rn(q_i * fl(Q_SPLIT / amax)) is within 1/2 +
+// 2^-10 of q_i / sq, sq = fl(amax / Q_SPLIT), so |q_i - sq Q_i| <= 0.503 sq,
+// and |code . (q - sq Q)| <= 127 d 0.51 sq per unit of s_c.
+constexpr float QSPLIT_BOUND = 0.51f;
+// Covers scales in the subnormal range.
 constexpr float Q8_ABS_BOUND = 1e-30f;
 
 struct SelectParams {
@@ -69,8 +73,6 @@ struct SelectParams {
     const float* cent;
     const int8_t* cent_q;       // [U, Cmax, D] int8 scoring copy of cent
     const float* cent_qs;       // [U, Cmax] its row scales
-    float* scores;              // [U, Cmax] upper bound of each score (first pass)
-    int32_t* hist;              // [U, SEL_HBINS]
     unsigned long long* gkey;   // [U, npow_max] scratch for large candidate sets
     int32_t* gw;                // [U, npow_max]
     const int32_t* cnt;
@@ -85,7 +87,6 @@ struct SelectParams {
     int32_t* n_sel;
     int32_t* sel_tok;
     int32_t* n_tok;
-    int32_t* unit_prefix;
     int32_t* tok_prefix;        // [U, Cmax + 1] run offsets of the list
     int32_t* tail_sel;          // [U, max(max_tail, 1)] communities of the list's tail part
     int Hq, G, per_head;
@@ -154,299 +155,85 @@ __device__ __forceinline__ void prefetch_run(const int32_t* run, int len) {
     for (int l = 0; l < lines; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(run + 32 * l));
 }
 
-// A lane's E int8 codes of a row (E bytes), kept packed until used.
-__device__ __forceinline__ float q8_byte(uint32_t w, int k) {  // signed byte k of w
-    return (float)((int)(w << (24 - 8 * k)) >> 24);
-}
-template <int E> struct Q8Part;
-template <> struct Q8Part<4> {
-    uint32_t w;
-    __device__ __forceinline__ void load(const int8_t* p) { w = *reinterpret_cast<const uint32_t*>(p); }
-    __device__ __forceinline__ void zero() { w = 0u; }
-    __device__ __forceinline__ void unpack(float (&x)[4]) const {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = q8_byte(w, k);
-    }
+// A lane's share of an int8 code row: D / SC_LPR bytes (16 for d = 128).
+template <int D> struct CodePart;
+template <> struct CodePart<128> {
+    static constexpr int W = 4;  // 32-bit words
+    uint4 v;
+    __device__ __forceinline__ void load(const int8_t* p) { v = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ uint32_t word(int k) const { return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w; }
 };
-template <> struct Q8Part<8> {
-    uint2 w;
-    __device__ __forceinline__ void load(const int8_t* p) { w = *reinterpret_cast<const uint2*>(p); }
-    __device__ __forceinline__ void zero() { w = make_uint2(0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[8]) const {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            x[k] = q8_byte(w.x, k);
-            x[4 + k] = q8_byte(w.y, k);
-        }
-    }
-};
-template <> struct Q8Part<16> {
-    uint4 w;
-    __device__ __forceinline__ void load(const int8_t* p) { w = *reinterpret_cast<const uint4*>(p); }
-    __device__ __forceinline__ void zero() { w = make_uint4(0u, 0u, 0u, 0u); }
-    __device__ __forceinline__ void unpack(float (&x)[16]) const {
-        const uint32_t v[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int k = 0; k < 4; ++k) x[4 * i + k] = q8_byte(v[i], k);
-    }
+template <> struct CodePart<64> {
+    static constexpr int W = 2;
+    uint2 v;
+    __device__ __forceinline__ void load(const int8_t* p) { v = *reinterpret_cast<const uint2*>(p); }
+    __device__ __forceinline__ uint32_t word(int k) const { return k == 0 ? v.x : v.y; }
 };
 
-// First-pass scores of this block's (up to) SCORE_ROWS centres of unit u,
-// from the int8 copy: a warp owns SCORE_ROWS / SEL_WARPS consecutive rows;
-// all of a lane's row parts (and the rows' scales) are loaded before any is
-// used, so each warp keeps its rows in flight.  The score is
-// s~ = s_c (q . code_c) / sqrt(d) and its bound e = Q8_BOUND s_c |q|_1 / sqrt(d).
-// One query head per graph: SC_LPR lanes per row (D/SC_LPR codes each, one
-// 16-byte load for d = 128), so a warp instruction covers 32/SC_LPR rows and
-// a row's sum takes log2(SC_LPR) shuffle levels.
-constexpr int SC_LPR = 8;
-template <typename T, int D>
-__device__ __forceinline__ void score_rows_gq1(const SelectParams& p, int u, int C) {
-    constexpr int E = D / SC_LPR;
-    constexpr int GR = 32 / SC_LPR;             // rows per warp instruction
-    constexpr int RW = SCORE_ROWS_GQ1 / SEL_WARPS;  // rows per warp
-    constexpr int RQ = RW / GR;                 // rows per lane group
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int oct = lane / SC_LPR, l8 = lane % SC_LPR;
-    const int row0 = blockIdx.x * SCORE_ROWS_GQ1 + warp * RW;
-    if (row0 >= C) return;
-    Q8Part<E> raw[RQ];
-    float rs[RQ];
-    int wv[RQ];  // sizes, for the histogram
+// Sum of GQ per-head integers over the SC_LPR lanes of a row group with value
+// exchange: afterwards lane lr holds the full sum of head lr >> (3 - log2 GQ).
+template <int GQ>
+__device__ __forceinline__ int rowgroup_reduce_heads(int (&v)[GQ], int lr) {
+    static_assert(GQ <= SC_LPR, "one head per lane at least");
+    int cur[GQ];
 #pragma unroll
-    for (int j = 0; j < RQ; ++j) {
-        const int c = row0 + GR * j + oct;
-        if (c < C) {
-            raw[j].load(p.cent_q + ((size_t)u * p.Cmax + c) * D + l8 * E);
-            rs[j] = p.cent_qs[(size_t)u * p.Cmax + c];
-            wv[j] = p.cnt[(size_t)u * p.Cmax + c];
+    for (int i = 0; i < GQ; ++i) cur[i] = v[i];
+    int n = GQ;
+#pragma unroll
+    for (int o = SC_LPR / 2; o >= 1; o >>= 1) {
+        if (n > 1) {
+            const bool upper = (lr & o) != 0;
+            const int h = n >> 1;
+#pragma unroll
+            for (int i = 0; i < h; ++i) {
+                const int send = upper ? cur[i] : cur[i + h];
+                const int keep = upper ? cur[i + h] : cur[i];
+                cur[i] = keep + __shfl_xor_sync(FULL, send, o);
+            }
+            n = h;
         } else {
-            raw[j].zero();
-            rs[j] = 0.f;
-            wv[j] = 0;
+            cur[0] += __shfl_xor_sync(FULL, cur[0], o);
         }
     }
-    const int b = u / p.G, g = u - b * p.G;
-    float qr[E], qn = 0.f;
-    {
-        const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + g) * D + l8 * E;  // head g
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            qr[e] = to_f32(qp[e]);
-            qn += fabsf(qr[e]);
-        }
-    }
-#pragma unroll
-    for (int o = SC_LPR / 2; o >= 1; o >>= 1) qn += __shfl_xor_sync(FULL, qn, o);  // |q|_1
-    const float ebase = Q8_BOUND * qn * p.inv_sqrt_d;
-    int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
-#pragma unroll
-    for (int j = 0; j < RQ; ++j) {
-        float x[E];
-        raw[j].unpack(x);
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) a = fmaf(qr[e], x[e], a);
-#pragma unroll
-        for (int o = SC_LPR / 2; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
-        const float sc = a * rs[j] * p.inv_sqrt_d;
-        const float err = fmaf(ebase, rs[j], Q8_ABS_BOUND);
-        const int c = row0 + GR * j + oct;
-        if (l8 == 0 && c < C) {
-            p.scores[(size_t)u * p.Cmax + c] = sc + err;
-            if (wv[j] > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), wv[j]);
-        }
-    }
+    return cur[0];
 }
 
-// Several query heads per graph with a bf16 q: the products on the tensor
-// cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), heads as the A rows
-// (padded with zeros), eight communities per n-tile as the B columns.  The
-// int8 codes are exact in bf16, so S = Q code^T is the same sum as in the
-// one-head path.  Lane (g, tq) owns dims [LB tq, LB tq + LB) of its rows
-// (LB = D/4 bytes, one or two 16-byte loads) and of its head's q; k-step kk
-// takes dims LB tq + 4kk .. +3 of every lane, which the fragment sees as
-// k = 2tq, 2tq + 1 (register b0 / a0) and 2tq + 8, 2tq + 9 (b1 / a2): the
-// same map on both operands, and over the k-steps every dim once.  A warp
-// takes two n-tiles (16 communities); the 4 lanes of quad 0 then hold, per
-// community, the max over the group's heads.
-__device__ __forceinline__ void mma_sc(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(0u), "r"(a1), "r"(0u), "r"(b0), "r"(b1));
+// Thread i < SEL_PREFETCH warms one page that the unit's selection reads or
+// writes after the first pass (token list, members, CSR offsets, ranked ids,
+// fp32 centres, tail), so the address translations are done before they are
+// needed; issued before waiting for the previous kernel.
+constexpr int SEL_PREFETCH = 10;
+__device__ __forceinline__ void select_prefetch(const SelectParams& p, int u, int i, int D) {
+    const size_t crow = (size_t)u * p.Cmax * D;
+    const void* a = nullptr;
+    switch (i) {
+        case 0: a = p.sel_tok + (size_t)u * p.tok_cap; break;
+        case 1: a = p.tok + (size_t)u * p.T_cap; break;
+        case 2: a = p.tok + (size_t)u * p.T_cap + p.T_cap - 1; break;
+        case 3: a = p.offs + (size_t)u * (p.Cmax + 1); break;
+        case 4: a = p.sel_comm + (size_t)u * p.Cmax; break;
+        case 5: a = p.cent + crow; break;
+        case 6: a = p.cent + crow + (size_t)(p.Cmax - 1) * D; break;
+        case 7: a = p.max_tail > 0 ? p.tail_tok + (size_t)u * p.max_tail : nullptr; break;
+        case 8: a = p.max_tail > 0 ? p.tail_comm + (size_t)u * p.max_tail : nullptr; break;
+        case 9: a = p.tail_len + u; break;
+        default: break;
+    }
+    if (a) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
 }
 
-// two signed bytes of w (k, k + 1) as a bf16 pair, low half first (exact)
-__device__ __forceinline__ uint32_t q8_pair_bf16(uint32_t w, int k) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(q8_byte(w, k), q8_byte(w, k + 1));
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-template <int D, int GQ>
-__device__ __forceinline__ void score_rows_mma(const SelectParams& p, int u, int C) {
-    constexpr int KS = D / 16;   // k-steps
-    constexpr int LB = D / 4;    // dims (bytes of codes) per lane and row
-    constexpr int NV = LB / 16;  // 16-byte loads per lane and row
-    constexpr int RW = SCORE_ROWS / SEL_WARPS;  // 16 communities per warp
-    static_assert(RW == 16 && KS == LB / 4, "two n-tiles of 8 per warp; 4 dims per lane and k-step");
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, tq = lane & 3;
-    const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
-    if (row0 >= C) return;
-    // codes of both n-tiles (community row0 + 8t + g) and the scales of the
-    // four communities whose results this lane ends up holding (2tq + e)
-    uint4 bw[2][NV];
-    float rs[2][2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int c = row0 + 8 * t + g;
-        const int8_t* row = p.cent_q + ((size_t)u * p.Cmax + min(c, C - 1)) * D + LB * tq;
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const uint4 x = reinterpret_cast<const uint4*>(row)[v];
-            bw[t][v] = c < C ? x : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int ce = row0 + 8 * t + 2 * tq + e;
-            rs[t][e] = ce < C ? p.cent_qs[(size_t)u * p.Cmax + ce] : 0.f;
-        }
-    }
-    const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
-    const int b = u / p.G, gg = u - b * p.G;
-    const int h0 = gg * GQ;  // per-group graphs (several heads)
-    // this lane's dims of head g's q (bf16 pairs), and |q_g|_1 over the quad
-    uint32_t qa[LB / 2];
-    float qn = 0.f;
-    {
-        const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + h0 + min(g, GQ - 1)) * D + LB * tq;
-#pragma unroll
-        for (int v = 0; v < LB / 8; ++v) {
-            const uint4 x = reinterpret_cast<const uint4*>(qrow)[v];
-            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                qa[4 * v + k] = g < GQ ? xs[k] : 0u;
-                qn += fabsf(bf16_lo(qa[4 * v + k])) + fabsf(bf16_hi(qa[4 * v + k]));
-            }
-        }
-    }
-    qn += __shfl_xor_sync(FULL, qn, 1);
-    qn += __shfl_xor_sync(FULL, qn, 2);
-#pragma unroll
-    for (int o = 4; o <= 16; o <<= 1) qn = fmaxf(qn, __shfl_xor_sync(FULL, qn, o));  // max over heads
-    const float ebase = Q8_BOUND * qn * p.inv_sqrt_d;
-    int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        uint32_t wd[4 * NV];  // code word kk: dims LB tq + 4kk .. +3
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            wd[4 * v] = bw[t][v].x;
-            wd[4 * v + 1] = bw[t][v].y;
-            wd[4 * v + 2] = bw[t][v].z;
-            wd[4 * v + 3] = bw[t][v].w;
-        }
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < KS; ++kk)
-            mma_sc(sacc, qa[2 * kk], qa[2 * kk + 1], q8_pair_bf16(wd[kk], 0), q8_pair_bf16(wd[kk], 2));
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            // max over the group's heads (rows g < GQ)
-            float sv = g < GQ ? sacc[e] : -INFINITY;
-#pragma unroll
-            for (int o = 4; o <= 16; o <<= 1) sv = fmaxf(sv, __shfl_xor_sync(FULL, sv, o));
-            const int r = 8 * t + 2 * tq + e;  // community row within the warp's 16
-            const int w = __shfl_sync(FULL, wc, r);
-            const float sc = sv * rs[t][e] * p.inv_sqrt_d;
-            const float err = fmaf(ebase, rs[t][e], Q8_ABS_BOUND);
-            const int c = row0 + r;
-            if (g == 0 && c < C) {
-                p.scores[(size_t)u * p.Cmax + c] = sc + err;
-                if (w > 0) atomicAdd(hist + (int)(score_key(sc - err, c) >> (64 - SEL_HBITS)), w);
-            }
-        }
-    }
+// Dynamic shared memory of the kernel: the histogram, then per community its
+// upper score bound and its size.
+__host__ __device__ inline size_t sel_dyn_smem(int Cmax) {
+    return (size_t)SEL_HBINS * 4 + 2 * (((size_t)Cmax * 4 + 15) & ~size_t(15));
 }
 
 template <typename T, int D, int GQ>
-__device__ __forceinline__ void score_rows(const SelectParams& p, int u, int C) {
-    if constexpr (GQ == 1) {
-        score_rows_gq1<T, D>(p, u, C);
-        return;
-    }
-    if constexpr (GQ > 1 && std::is_same<T, __nv_bfloat16>::value) {
-        score_rows_mma<D, GQ>(p, u, C);
-        return;
-    }
-    constexpr int E = D / 16;
-    constexpr int RW = SCORE_ROWS / SEL_WARPS;  // rows per warp
-    constexpr int RH = RW / 2;                  // rows per half-warp
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int half = lane >> 4, l16 = lane & 15;
-    const int row0 = blockIdx.x * SCORE_ROWS + warp * RW;
-    if (row0 >= C) return;
-    Q8Part<E> raw[RH];
-    float rs[RH];
-#pragma unroll
-    for (int j = 0; j < RH; ++j) {
-        const int c = row0 + 2 * j + half;
-        if (c < C) {
-            raw[j].load(p.cent_q + ((size_t)u * p.Cmax + c) * D + l16 * E);
-            rs[j] = p.cent_qs[(size_t)u * p.Cmax + c];
-        } else {
-            raw[j].zero();
-            rs[j] = 0.f;
-        }
-    }
-    const int wc = (lane < RW && row0 + lane < C) ? p.cnt[(size_t)u * p.Cmax + row0 + lane] : 0;
-    const int b = u / p.G, g = u - b * p.G;
-    const int h0 = p.per_head ? g : g * GQ;
-    float qr[GQ][E], qn[GQ];
-#pragma unroll
-    for (int h = 0; h < GQ; ++h) {
-        load_row_part<T, E>(static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h0 + h) * D + l16 * E, qr[h]);
-        qn[h] = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) qn[h] += fabsf(qr[h][e]);
-    }
-    // max over the heads of |q_h|_1
-    const float ebase = Q8_BOUND * halfwarp_max_over_heads<GQ>(halfwarp_reduce_heads<GQ>(qn, lane)) * p.inv_sqrt_d;
-
-    int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
-#pragma unroll
-    for (int j = 0; j < RH; ++j) {
-        float x[E];
-        raw[j].unpack(x);
-        float part[GQ];
-#pragma unroll
-        for (int h = 0; h < GQ; ++h) {
-            float a = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) a = fmaf(qr[h][e], x[e], a);
-            part[h] = a;
-        }
-        float s = halfwarp_reduce_heads<GQ>(part, lane);
-        s = halfwarp_max_over_heads<GQ>(s) * rs[j] * p.inv_sqrt_d;
-        const float err = fmaf(ebase, rs[j], Q8_ABS_BOUND);
-        const int c = row0 + 2 * j + half;
-        const int w = __shfl_sync(FULL, wc, 2 * j + half);
-        if (l16 == 0 && c < C) {
-            p.scores[(size_t)u * p.Cmax + c] = s + err;
-            if (w > 0) atomicAdd(hist + (int)(score_key(s - err, c) >> (64 - SEL_HBITS)), w);
-        }
-    }
-}
-
-// Selection for unit u after all its scores are in (see the file comment).
-// Score bounds and the histogram were written by other blocks: read through L2.
-template <typename T, int D, int GQ>
-__device__ void select_unit(const SelectParams& p, int u, int C) {
+__global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectParams p) {
+    extern __shared__ __align__(16) unsigned char sel_dyn[];
+    int* s_hist = reinterpret_cast<int*>(sel_dyn);
+    float* s_ub = reinterpret_cast<float*>(sel_dyn + SEL_HBINS * 4);
+    int* s_sz = reinterpret_cast<int*>(sel_dyn + SEL_HBINS * 4 + (((size_t)p.Cmax * 4 + 15) & ~size_t(15)));
     __shared__ unsigned long long s_key[SEL_FAST];
     __shared__ int s_w[SEL_FAST];
     __shared__ unsigned long long s_runs[SEL_FAST];
@@ -456,60 +243,165 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     __shared__ unsigned s_mask[MAX_CMAX / 32];
     __shared__ int s_warp[33];
     __shared__ int s_bstar, s_nc, s_nt, s_cnt;
+    // the graph's queries: fp32 (exact re-scoring) and the int8 split words
+    // (hi, then lo) of the first pass, with each head's scale and bound term
+    __shared__ __align__(16) float s_qf[GQ][D];
+    __shared__ __align__(16) uint32_t s_qw[GQ][2][D / 4];
+    __shared__ float s_sq[GQ], s_eb[GQ];
 
+    constexpr int EW = D / 32;  // q elements per lane
+    const int u = blockIdx.x;
     const int tid = threadIdx.x, nt = blockDim.x;
     const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
-    const float* sc = p.scores + (size_t)u * p.Cmax;
-    const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
-    const int32_t* hist = p.hist + (size_t)u * SEL_HBINS;
+    if (tid < SEL_PREFETCH) select_prefetch(p, u, tid, D);
+    {
+        int4* h4 = reinterpret_cast<int4*>(s_hist);
+        for (int i = tid; i < SEL_HBINS / 4; i += nt) h4[i] = make_int4(0, 0, 0, 0);
+    }
     for (int i = tid; i < (p.Cmax + 31) / 32; i += nt) s_mask[i] = 0u;
     if (tid == 0) {
         s_bstar = -1;
         s_nc = 0;
         s_cnt = 0;
     }
+    pdl_wait();  // q, the centres and the counts may come from the kernels before
 
-    // Every load that depends on nothing but u is issued first, together:
-    // the histogram (16 bins per thread as four 16-byte loads) and the first
-    // round of community sizes and scores (from clamped in-range ids, masked
-    // by c < C later).
-    constexpr int RND = 8;
-    constexpr int per = SEL_HBINS / SEL_THREADS;
-    static_assert(per == 16, "four int4 histogram loads per thread");
-    int4 hv[4];
+    const int b = u / p.G, g = u - b * p.G;
+    const int h0 = p.per_head ? g : g * GQ;
+    if (warp < GQ) {
+        // head `warp`: fp32 copy, |q|_1, and the integer split
+        const T* qp = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + h0 + warp) * D + lane * EW;
+        float x[EW];
+        float amax = 0.f, qn = 0.f;
+#pragma unroll
+        for (int e = 0; e < EW; ++e) {
+            x[e] = to_f32(qp[e]);
+            s_qf[warp][lane * EW + e] = x[e];
+            amax = fmaxf(amax, fabsf(x[e]));
+            qn += fabsf(x[e]);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+            qn += __shfl_xor_sync(FULL, qn, o);
+        }
+        const float sq = amax > 0.f ? __fdiv_rn(amax, (float)Q_SPLIT) : 0.f;
+        const float rq = amax > 0.f ? __fdiv_rn((float)Q_SPLIT, amax) : 0.f;
+        uint32_t hw = 0u, lw = 0u;
+#pragma unroll
+        for (int e = 0; e < EW; ++e) {
+            const int Q = max(-Q_SPLIT, min(Q_SPLIT, __float2int_rn(x[e] * rq)));
+            const int hi = (Q + 64) >> 7;  // floor((Q + 64) / 128)
+            const int lo = Q - 128 * hi;
+            hw |= (uint32_t)(hi & 0xff) << (8 * e);
+            lw |= (uint32_t)(lo & 0xff) << (8 * e);
+        }
+        if constexpr (EW == 4) {
+            s_qw[warp][0][lane] = hw;
+            s_qw[warp][1][lane] = lw;
+        } else {
+            reinterpret_cast<uint16_t*>(s_qw[warp][0])[lane] = (uint16_t)hw;
+            reinterpret_cast<uint16_t*>(s_qw[warp][1])[lane] = (uint16_t)lw;
+        }
+        if (lane == 0) {
+            s_sq[warp] = sq;
+            s_eb[warp] = fmaf(Q8_BOUND, qn, (127.0f * D * QSPLIT_BOUND) * sq);
+        }
+    }
+    __syncthreads();
+    const int C = min(p.num_comm[u], p.Cmax);
+    const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
+
+    // 1. first pass: lane lr of row group `sub` owns D/8 dims of one row
     {
-        int4* h4 = reinterpret_cast<int4*>(const_cast<int32_t*>(hist) + per * tid);
+        using CP = CodePart<D>;
+        constexpr int W = CP::W;
+        const int sub = lane / SC_LPR, lr = lane % SC_LPR;
+        constexpr int LG = GQ == 1 ? 0 : GQ == 2 ? 1 : GQ == 4 ? 2 : 3;
+        const int hl = lr >> (3 - LG);  // head whose sum this lane ends up with
+        const float sq_mine = s_sq[hl];
+        float eb = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) hv[i] = __ldcg(h4 + i);
-        // leave the histogram zero for the next call (each thread clears the
-        // bins it alone read)
+        for (int h = 0; h < GQ; ++h) eb = fmaxf(eb, s_eb[h]);
+        const float ebase = eb * p.inv_sqrt_d;
+        // the lane's query words: registers for one or two heads, else read
+        // from shared memory per row group
+        uint32_t qreg[GQ <= 2 ? GQ : 1][2][W];
+        if constexpr (GQ <= 2) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) h4[i] = make_int4(0, 0, 0, 0);
+            for (int h = 0; h < GQ; ++h)
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    qreg[h][0][k] = s_qw[h][0][lr * W + k];
+                    qreg[h][1][k] = s_qw[h][1][lr * W + k];
+                }
+        }
+        const int8_t* codes = p.cent_q + (size_t)u * p.Cmax * D + lr * (D / SC_LPR);
+        // the rows' scales and sizes go to shared memory (s_ub, s_sz) while
+        // the first codes load; each row's upper bound later replaces its scale
+        {
+            const float* scales = p.cent_qs + (size_t)u * p.Cmax;
+            for (int c = tid; c < C; c += nt) {
+                cp_async_4(s_ub + c, scales + c);
+                cp_async_4(s_sz + c, cn + c);
+            }
+            cp_async_commit();
+        }
+        constexpr int RQ = ScRq<GQ>::v;
+        constexpr int STEP = SEL_WARPS * RQ * SC_RPI;
+        CP cv[RQ];
+        auto load_codes = [&](int b0) {
+#pragma unroll
+            for (int j = 0; j < RQ; ++j) cv[j].load(codes + (size_t)min(b0 + j * SC_RPI + sub, C - 1) * D);
+        };
+        int base = warp * RQ * SC_RPI;
+        if (base < C) load_codes(base);
+        cp_async_wait<0>();
+        __syncthreads();
+        for (; base < C; base += STEP) {
+#pragma unroll
+            for (int j = 0; j < RQ; ++j) {
+                int acc[GQ];
+#pragma unroll
+                for (int h = 0; h < GQ; ++h) {
+                    int ah = 0, al = 0;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        uint32_t qh, ql;
+                        if constexpr (GQ <= 2) {
+                            qh = qreg[h][0][k];
+                            ql = qreg[h][1][k];
+                        } else {
+                            qh = s_qw[h][0][lr * W + k];
+                            ql = s_qw[h][1][lr * W + k];
+                        }
+                        ah = __dp4a((int)cv[j].word(k), (int)qh, ah);
+                        al = __dp4a((int)cv[j].word(k), (int)ql, al);
+                    }
+                    acc[h] = ah * 128 + al;  // exact: |acc| < 2^29
+                }
+                float f = (float)rowgroup_reduce_heads<GQ>(acc, lr) * sq_mine;
+#pragma unroll
+                for (int o = SC_LPR >> LG; o < SC_LPR; o <<= 1) f = fmaxf(f, __shfl_xor_sync(FULL, f, o));
+                const int c = base + j * SC_RPI + sub;
+                if (lr == 0 && c < C) {
+                    const float rs = s_ub[c];
+                    const int w = s_sz[c];
+                    const float sc = f * rs * p.inv_sqrt_d;
+                    const float err = fmaf(ebase, rs, Q8_ABS_BOUND);
+                    s_ub[c] = w > 0 ? sc + err : -INFINITY;
+                    if (w > 0) atomicAdd(&s_hist[(int)(score_key(sc - err, c) >> (64 - SEL_HBITS))], w);
+                }
+            }
+            if (base + STEP < C) load_codes(base + STEP);
+        }
     }
-    int wv[RND];
-    float sv[RND];
-#pragma unroll
-    for (int r = 0; r < RND; ++r) {
-        const int c = min(tid + r * nt, p.Cmax - 1);
-        wv[r] = cn[c];
-        sv[r] = __ldcg(sc + c);
-    }
-    // this lane's part of the graph's queries, for the exact re-scoring
-    constexpr int EW = D / 32;
-    float qw[GQ][EW];
-    {
-        const int b = u / p.G, g = u - b * p.G;
-        const int h0 = p.per_head ? g : g * GQ;
-#pragma unroll
-        for (int h = 0; h < GQ; ++h)
-#pragma unroll
-            for (int e = 0; e < EW; ++e)
-                qw[h][e] = to_f32(static_cast<const T*>(p.q)[((size_t)b * p.Hq + h0 + h) * D + lane * EW + e]);
-    }
+    __syncthreads();
+
     // exact fp32 scores, from cent, of the n candidates whose keys (built
     // from the upper bounds) are in keys[]: one warp per candidate, RSC
     // candidates' rows in flight per warp; the keys are replaced in place
-    constexpr int RSC = 8;
+    constexpr int RSC = GQ >= 4 ? 4 : 8;
     auto rescore = [&](unsigned long long* keys, int n) {
         for (int i0 = warp; i0 < n; i0 += RSC * nw) {
             float row[RSC][EW];
@@ -518,8 +410,13 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
             for (int r = 0; r < RSC; ++r) {
                 cid[r] = key_id(keys[min(i0 + r * nw, n - 1)]);
                 const float* cr = p.cent + ((size_t)u * p.Cmax + cid[r]) * D + lane * EW;
+                if constexpr (EW == 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(cr);
+                    row[r][0] = v.x; row[r][1] = v.y; row[r][2] = v.z; row[r][3] = v.w;
+                } else {
 #pragma unroll
-                for (int e = 0; e < EW; ++e) row[r][e] = cr[e];
+                    for (int e = 0; e < EW; ++e) row[r][e] = cr[e];
+                }
             }
             unsigned long long nk[RSC];
 #pragma unroll
@@ -529,7 +426,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
                 for (int h = 0; h < GQ; ++h) {
                     float a = 0.f;
 #pragma unroll
-                    for (int e = 0; e < EW; ++e) a = fmaf(qw[h][e], row[r][e], a);
+                    for (int e = 0; e < EW; ++e) a = fmaf(s_qf[h][lane * EW + e], row[r][e], a);
 #pragma unroll
                     for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
                     best = fmaxf(best, a);
@@ -545,15 +442,22 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         }
     };
 
-    // 1. crossing bin: thread t owns bins [per*t, per*t + per)
+    // 2a. crossing bin: thread t owns bins [per*t, per*t + per)
+    constexpr int per = SEL_HBINS / SEL_THREADS;
+    static_assert(per == 8, "two int4 histogram loads per thread");
     {
-        const int hw[per] = {hv[0].x, hv[0].y, hv[0].z, hv[0].w, hv[1].x, hv[1].y, hv[1].z, hv[1].w,
-                             hv[2].x, hv[2].y, hv[2].z, hv[2].w, hv[3].x, hv[3].y, hv[3].z, hv[3].w};
+        int hw[per];
+        {
+            const int4* h4 = reinterpret_cast<const int4*>(s_hist) + 2 * tid;
+            const int4 a = h4[0], c = h4[1];
+            hw[0] = a.x; hw[1] = a.y; hw[2] = a.z; hw[3] = a.w;
+            hw[4] = c.x; hw[5] = c.y; hw[6] = c.z; hw[7] = c.w;
+        }
         int own = 0;
 #pragma unroll
         for (int i = 0; i < per; ++i) own += hw[i];
         int total;
-        const int pre = block_exclusive_scan(own, s_warp, &total);  // also orders the inits above
+        const int pre = block_exclusive_scan(own, s_warp, &total);
         int above = total - pre - own;  // weight of every bin above this thread's
 #pragma unroll
         for (int i = per - 1; i >= 0; --i) {
@@ -567,12 +471,24 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     __syncthreads();
     const int bstar = max(s_bstar, 0);  // no crossing: every key is a candidate
 
-    // 2. candidates: keys from the crossing bin up, with their sizes
-    auto offer = [&](int c, int w, float sval) {
-        if (c >= C || w <= 0) return;
-        const unsigned long long k = score_key(sval, c);
-        if ((int)(k >> (64 - SEL_HBITS)) >= bstar) {
-            const int i = atomicAdd(&s_nc, 1);
+    // 2b. candidates: keys from the crossing bin up, with their sizes; one
+    //     shared-memory atomic per warp and round
+    for (int c0 = 0; c0 < C; c0 += nt) {
+        const int c = c0 + tid;
+        bool cand = false;
+        int w = 0;
+        unsigned long long k = 0ull;
+        if (c < C) {
+            w = s_sz[c];
+            k = score_key(s_ub[c], c);
+            cand = w > 0 && (int)(k >> (64 - SEL_HBITS)) >= bstar;
+        }
+        const unsigned m = __ballot_sync(FULL, cand);
+        int first = 0;
+        if (lane == 0 && m) first = atomicAdd(&s_nc, __popc(m));
+        first = __shfl_sync(FULL, first, 0);
+        if (cand) {
+            const int i = first + __popc(m & ((1u << lane) - 1u));
             if (i < SEL_FAST) {
                 s_key[i] = k;
                 s_w[i] = w;
@@ -582,18 +498,6 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
                 for (int l = 0; l < D * 4 / 128; ++l) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + 128 * l));
             }
         }
-    };
-#pragma unroll
-    for (int r = 0; r < RND; ++r) offer(tid + r * nt, wv[r], sv[r]);
-    for (int c0 = tid + RND * nt; c0 < C; c0 += RND * nt) {
-#pragma unroll
-        for (int r = 0; r < RND; ++r) {
-            const int c = min(c0 + r * nt, p.Cmax - 1);
-            wv[r] = cn[c];
-            sv[r] = __ldcg(sc + c);
-        }
-#pragma unroll
-        for (int r = 0; r < RND; ++r) offer(c0 + r * nt, wv[r], sv[r]);
     }
     __syncthreads();
     const int nc = s_nc;
@@ -612,91 +516,77 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         __syncthreads();
     }
 
-    // 3. the cut.  Few candidates (the usual case): no sort; candidate i's
-    //    rank is the number of larger keys and the weight above it their size
-    //    sum, so it is selected iff that sum plus its own size fits the budget
-    //    (sizes are positive, so the selected set is a prefix of the ranking).
-    //    Each candidate's CSR run is looked up meanwhile and stored at its rank.
+    // 2c. the cut, from each candidate's rank and the sizes ranked above it
+    //     (sizes are positive, so the selected set is a prefix of the
+    //     ranking): candidate i is in iff the size above it plus its own fits
+    //     the budget.  Warp r sorts candidates [32r, 32r + 32) best first and
+    //     scans their sizes and run lengths in that order; an entry's rank is
+    //     its place in its own run plus, in every other run, the number of
+    //     entries above it (binary search), and the sizes above it the
+    //     matching prefixes.  Sort values carry the candidate's slot below the
+    //     id, which keeps the tie order (lower id first) and finds the payload.
     int kstar;
     const unsigned long long* sorted;
     const bool small = nc <= SEL_FAST;
     int* bsz = small ? s_bsz : p.gw + (size_t)u * p.npow_max;
     if (small) {
-        bool in = false;
-        if (nc <= RANK_LOOP_MAX) {  // uniform over the block
-            if (tid < nc) {
-                const unsigned long long k = s_key[tid];
-                const int w = s_w[tid];
-                // rank, the size ranked above (for the cut) and the run length
-                // ranked above (the run's place in the token list)
-                int rank = 0, above = 0, above_len = 0;
-                for (int j = 0; j < nc; ++j) {
-                    const bool gt = s_key[j] > k;
-                    rank += gt;
-                    above += gt ? s_w[j] : 0;
-                    above_len += gt ? s_len[j] : 0;
-                }
-                in = above + w <= p.budget;
-                s_runs[rank] = k;
-                s_bsz[rank] = above_len + (o1 - o0);  // inclusive prefix in rank order
-                s_ofs[rank] = o0;
-                if (in || rank == 0) prefetch_run(p.tok + (size_t)u * p.T_cap + o0, o1 - o0);
-            }
-        } else {
-            // More candidates than the quadratic ranking pays for: the exact
-            // keys are sorted best first in registers, a thread per entry, by
-            // a bitonic network over next_pow2(nc) entries (partners in the
-            // same warp exchange by shuffles, across warps through shared
-            // memory); the low bits of a sort key carry the candidate's slot
-            // next to its id, which keeps the tie order (lower id first).
-            // One scan in rank order then gives the sizes and run lengths
-            // ranked above each entry.
-            __shared__ int s_o0[SEL_FAST];
-            __shared__ unsigned long long s_w64[33];
-            static_assert(SEL_FAST <= 256 && MAX_CMAX <= (1 << 24), "slot and id fit the key's low 32 bits");
-            unsigned long long v = 0;  // below every real key
+        __shared__ unsigned long long s_sv[SEL_FAST];
+        __shared__ int s_pw[SEL_FAST], s_pl[SEL_FAST], s_o0[SEL_FAST];
+        static_assert(SEL_FAST <= 1024 && MAX_CMAX <= (1 << 22), "slot and id fit the value's low 32 bits");
+        const int R = (nc + 31) >> 5;
+        int w = 0, len = 0;
+        unsigned long long v = 0ull;  // below every real value
+        if (warp < R) {
             if (tid < nc) {
                 const unsigned long long k = s_key[tid];
                 s_o0[tid] = o0;
-                v = (k & 0xffffffff00000000ull) | ((unsigned long long)(MAX_CMAX - 1 - key_id(k)) << 8) |
+                v = (k & 0xffffffff00000000ull) | ((unsigned long long)(MAX_CMAX - 1 - key_id(k)) << 10) |
                     (unsigned long long)tid;
             }
-            int npow = 32;
-            while (npow < nc) npow <<= 1;
-            for (int k = 2; k <= npow; k <<= 1) {
-                for (int j = k >> 1; j > 0; j >>= 1) {
-                    unsigned long long o;
-                    if (j >= 32) {  // uniform over the block
-                        s_key[tid] = v;  // each thread read only its own entry above
-                        __syncthreads();
-                        o = s_key[tid ^ j];
-                        __syncthreads();
-                    } else {
-                        o = __shfl_xor_sync(FULL, v, j);
-                    }
-                    const unsigned long long hi = v > o ? v : o, lo = v > o ? o : v;
-                    v = (((tid & k) == 0) == ((tid & j) == 0)) ? hi : lo;
-                }
-            }
-            int w = 0, len = 0, slot = 0;
-            if (tid < nc) {
-                slot = (int)(v & 0xffu);
+            v = warp_sort_desc(v, lane);
+            if (v) {
+                const int slot = (int)(v & 0x3ffu);
                 w = s_w[slot];
                 len = s_len[slot];
             }
-            // sizes and run lengths are each at most T_cap < 2^31: one 64-bit scan
-            const unsigned long long pre =
-                block_exclusive_scan_u64(((unsigned long long)w << 32) | (unsigned)len, s_w64);
-            if (tid < nc) {
-                const int above = (int)(pre >> 32), above_len = (int)(pre & 0xffffffffu);
-                const int id = MAX_CMAX - 1 - (int)((v >> 8) & 0xffffffu);
-                const int o0r = s_o0[slot];
-                in = above + w <= p.budget;
-                s_runs[tid] = (v & 0xffffffff00000000ull) | (unsigned long long)(0xffffffffu - (unsigned)id);
-                s_bsz[tid] = above_len + len;  // inclusive prefix in rank order
-                s_ofs[tid] = o0r;
-                if (in || tid == 0) prefetch_run(p.tok + (size_t)u * p.T_cap + o0r, len);
+            int pw = w, pl = len;  // inclusive prefixes in the run's order
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int yw = __shfl_up_sync(FULL, pw, o), yl = __shfl_up_sync(FULL, pl, o);
+                if (lane >= o) {
+                    pw += yw;
+                    pl += yl;
+                }
             }
+            s_sv[tid] = v;
+            s_pw[tid] = pw;
+            s_pl[tid] = pl;
+        }
+        __syncthreads();
+        bool in = false;
+        if (warp < R && v) {
+            int rank = lane, above = s_pw[tid] - w, above_len = s_pl[tid] - len;
+            for (int r = 0; r < R; ++r) {
+                if (r == warp) continue;
+                const unsigned long long* run = s_sv + (r << 5);
+                int lo = 0;  // entries of run r above v: a prefix of the run
+#pragma unroll
+                for (int step = 16; step >= 1; step >>= 1) lo += run[lo + step - 1] > v ? step : 0;
+                lo += (lo == 31 && run[31] > v) ? 1 : 0;
+                rank += lo;
+                if (lo) {
+                    above += s_pw[(r << 5) + lo - 1];
+                    above_len += s_pl[(r << 5) + lo - 1];
+                }
+            }
+            const int slot = (int)(v & 0x3ffu);
+            const int id = MAX_CMAX - 1 - (int)((v >> 10) & 0x3fffffu);
+            const int o0r = s_o0[slot];
+            in = above + w <= p.budget;
+            s_runs[rank] = (v & 0xffffffff00000000ull) | (unsigned long long)(0xffffffffu - (unsigned)id);
+            s_bsz[rank] = above_len + len;  // inclusive prefix in rank order
+            s_ofs[rank] = o0r;
+            if (in || rank == 0) prefetch_run(p.tok + (size_t)u * p.T_cap + o0r, len);
         }
         kstar = __syncthreads_count(in);
         if (kstar == 0 && nc > 0) kstar = 1;  // the top community alone exceeds the budget: take it
@@ -709,9 +599,9 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         if (tid == 0) s_nc = 0;
         __syncthreads();
         for (int c = tid; c < C; c += nt) {
-            const int w = cn[c];
+            const int w = s_sz[c];
             if (w <= 0) continue;
-            const unsigned long long k = score_key(__ldcg(sc + c), c);
+            const unsigned long long k = score_key(s_ub[c], c);
             if ((int)(k >> (64 - SEL_HBITS)) >= bstar) gk[atomicAdd(&s_nc, 1)] = k;
         }
         __syncthreads();
@@ -735,7 +625,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
                 __syncthreads();
             }
         }
-        for (int i = tid; i < nc; i += nt) gw[i] = cn[key_id(gk[i])];
+        for (int i = tid; i < nc; i += nt) gw[i] = s_sz[key_id(gk[i])];
         __syncthreads();
         block_scan_inplace(gw, nc, s_warp);
         int mine = 0;
@@ -752,7 +642,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         }
     }
 
-    // 4. ranked ids and membership mask
+    // 3a. ranked ids and membership mask
     int32_t* selc = p.sel_comm + (size_t)u * p.Cmax;
     for (int i = tid; i < kstar; i += nt) {
         const int c = key_id(sorted[i]);
@@ -777,6 +667,7 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
         if (i < p.tok_cap) out[i] = i;
         else overflow = true;
     }
+    constexpr int RND = 4;
     if (small) {
         // one token per thread per round: its run is found by binary search in
         // the inclusive run prefix; a round's loads are issued before its stores
@@ -865,49 +756,6 @@ __device__ void select_unit(const SelectParams& p, int u, int C) {
     }
 }
 
-template <typename T, int D, int GQ>
-__global__ void __launch_bounds__(SEL_THREADS) score_kernel(SelectParams p) {
-    pdl_wait();  // q may come from the kernel before
-    const int u = blockIdx.y;
-    const int C = min(p.num_comm[u], p.Cmax);
-    score_rows<T, D, GQ>(p, u, C);
-}
-
-// Thread i < SEL_PREFETCH warms one page the selection of unit u reads or
-// writes after its first loads (token list, members, CSR offsets, ranked
-// ids, sizes, fp32 centres, tail), so the address translations are done
-// before they are needed.  None is written by the scoring kernel: issued
-// before waiting for it, they overlap its last blocks.
-constexpr int SEL_PREFETCH = 11;
-__device__ __forceinline__ void select_prefetch(const SelectParams& p, int u, int i, int D) {
-    const size_t crow = (size_t)u * p.Cmax * D;
-    const void* a = nullptr;
-    switch (i) {
-        case 0: a = p.sel_tok + (size_t)u * p.tok_cap; break;
-        case 1: a = p.tok + (size_t)u * p.T_cap; break;
-        case 2: a = p.tok + (size_t)u * p.T_cap + p.T_cap - 1; break;
-        case 3: a = p.offs + (size_t)u * (p.Cmax + 1); break;
-        case 4: a = p.sel_comm + (size_t)u * p.Cmax; break;
-        case 5: a = p.cnt + (size_t)u * p.Cmax; break;
-        case 6: a = p.cent + crow; break;
-        case 7: a = p.cent + crow + (size_t)(p.Cmax - 1) * D; break;
-        case 8: a = p.max_tail > 0 ? p.tail_tok + (size_t)u * p.max_tail : nullptr; break;
-        case 9: a = p.max_tail > 0 ? p.tail_comm + (size_t)u * p.max_tail : nullptr; break;
-        case 10: a = p.tail_len + u; break;
-        default: break;
-    }
-    if (a) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-}
-
-template <typename T, int D, int GQ>
-__global__ void __launch_bounds__(SEL_THREADS) select_kernel(SelectParams p) {
-    const int u = blockIdx.x;
-    if (threadIdx.x < SEL_PREFETCH) select_prefetch(p, u, threadIdx.x, D);
-    pdl_wait();  // every score and histogram update of the scoring kernel is visible
-    const int C = min(p.num_comm[u], p.Cmax);
-    select_unit<T, D, GQ>(p, u, C);
-}
-
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -920,13 +768,12 @@ static int next_pow2(int x) {
 
 namespace {
 struct SelWs {
-    size_t scores, gkey, gw, total;
+    size_t gkey, gw, total;
 };
 SelWs sel_ws_layout(int U, int Cmax) {
     SelWs l;
     const size_t np = (size_t)next_pow2(Cmax);
-    l.scores = 0;
-    l.gkey = l.scores + align256((size_t)U * Cmax * 4);
+    l.gkey = 0;
     l.gw = l.gkey + align256((size_t)U * np * 8);
     l.total = l.gw + align256((size_t)U * np * 4);
     return l;
@@ -934,11 +781,12 @@ SelWs sel_ws_layout(int U, int Cmax) {
 
 template <typename T, int D, int GQ>
 cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
-    constexpr int rows = ScoreBlockRows<GQ>::v;
-    dim3 grid((p.Cmax + rows - 1) / rows, p.U);
-    cudaError_t e = launch_pdl(KK_SCORE, score_kernel<T, D, GQ>, grid, dim3(SEL_THREADS), 0, st, p);
+    static LaunchCache lc;
+    auto kern = score_select_kernel<T, D, GQ>;
+    const size_t smem = sel_dyn_smem(p.Cmax);
+    cudaError_t e = prepare_launch(kern, lc, smem, SEL_THREADS, nullptr, nullptr);
     if (e != cudaSuccess) return e;
-    return launch_pdl(KK_SELECT, select_kernel<T, D, GQ>, dim3(p.U), dim3(SEL_THREADS), 0, st, p);
+    return launch_pdl(KK_SCORE, kern, dim3(p.U), dim3(SEL_THREADS), smem, st, p);
 }
 }  // namespace
 
@@ -947,6 +795,7 @@ size_t select_ws_bytes(int U, int Cmax) { return sel_ws_layout(U, Cmax).total; }
 cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const void* q, int budget,
                                 const SelView& s, void* ws, cudaStream_t st) {
     const int U = c.B * g.G;
+    if (U <= 0) return cudaSuccess;
     const SelWs l = sel_ws_layout(U, g.Cmax);
     char* w = static_cast<char*>(ws) + ws_head_bytes(c.B, c.Hq);
     SelectParams p{};
@@ -954,8 +803,6 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     p.cent = g.cent;
     p.cent_q = g.cent_q;
     p.cent_qs = g.cent_qs;
-    p.scores = reinterpret_cast<float*>(w + l.scores);
-    p.hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + WS_RESERVED);  // zero on entry
     p.gkey = reinterpret_cast<unsigned long long*>(w + l.gkey);
     p.gw = reinterpret_cast<int32_t*>(w + l.gw);
     p.cnt = g.cnt;
@@ -970,7 +817,6 @@ cudaError_t launch_score_select(const CacheView& c, const GraphView& g, const vo
     p.n_sel = s.n_sel;
     p.sel_tok = s.sel_tok;
     p.n_tok = s.n_tok;
-    p.unit_prefix = s.unit_prefix;
     p.tok_prefix = s.tok_prefix;
     p.tail_sel = s.tail_sel;
     p.Hq = c.Hq;

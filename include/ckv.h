@@ -32,10 +32,10 @@
  *  - No call allocates device memory.  Scratch comes from the caller's
  *    workspace `ws` of `ws_bytes` bytes (256-byte aligned), sized by
  *    ckv_workspace_size(); a smaller workspace returns CKV_ERR_WORKSPACE.
- *    Its head (256 + 16384 * B * Hq bytes: the attention kernels' work
- *    counter and the selection's score histograms) must be zero before the
- *    workspace's first use, e.g. zero-fill the whole workspace once after
- *    allocating it; every call leaves the head zero.  The rest needs no
+ *    Its head (256 + 4 * B * Hq bytes rounded up to a multiple of 256: the
+ *    attention kernels' work counter and one arrival counter per graph unit)
+ *    must be zero before the workspace's first use, e.g. zero-fill the whole
+ *    workspace once after allocating it; every call leaves the head zero.  The rest needs no
  *    initialisation.  Calls sharing a workspace must not overlap on the GPU.
  *  - Host-side checks happen before any launch and return a status without
  *    touching the device; ckv_last_error() then names the failed check.
@@ -66,7 +66,7 @@ extern "C" {
 #define CKV_API
 #endif
 
-#define CKV_ABI_VERSION 5
+#define CKV_ABI_VERSION 6
 #define CKV_NEIGHBOURS 8
 
 typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
@@ -226,10 +226,12 @@ CKV_API ckv_status ckv_build_centroids(const ckv_cache_desc* cache, const int32_
  *           longest ranked prefix whose cnt sum is <= budget, and at least the
  *           top community; the sinks come on top of the budget.
  * Writes every field of `sel`.  budget >= 0.  The pass over all communities
- * reads the int8 copy (cent_q, cent_qs) with a rigorous error bound per score
- * (|q . (cent - s cent_q)| <= s |q|_1 / 2 plus rounding); only the
+ * reads the int8 copy (cent_q, cent_qs) against an exact integer split of q,
+ * with a rigorous error bound per score (|q . (cent - s cent_q)| <=
+ * s |q|_1 / 2, plus the split's and the rounding's share); only the
  * communities whose bound reaches the budget cut are re-scored from the fp32
- * cent, so the selection is the one the fp32 scores give.
+ * cent, so the selection is the one the fp32 scores give.  One kernel
+ * launch.
  */
 CKV_API ckv_status ckv_score_select(const ckv_cache_desc* cache, const ckv_graph_desc* graph,
                             const void* q, int32_t budget, const ckv_selection_desc* sel,
@@ -263,12 +265,14 @@ CKV_API ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q,
  *   - Calls needing more scratch than CKV_NOALLOC_SCRATCH_BYTES return
  *     CKV_ERR_UNSUPPORTED before touching the device.  The need is the size
  *     ckv_workspace_size reports for the attention alone: the head
- *     (256 + 16384 * B * Hq bytes), about 4 * (12288 + 2U) * gq * (d + 2)
- *     bytes of split-K partials (gq query heads per graph, U = B * graphs per
- *     sequence) and 4 * U * sel->tok_cap bytes of neighbour logits.  Per-head
- *     graphs with d = 128 need about 6.4 MiB + the head + the logits;
- *     Hq/Hkv = 8 with d = 128 in per-group mode needs over 32 MiB and is
- *     refused.
+ *     (256 + 4 * B * Hq bytes, rounded up to 256), about
+ *     4 * (12288 + 2U) * gq * (d + 2) bytes of split-K partials (gq query
+ *     heads per graph, U = B * graphs per sequence) and 4 * U * sel->tok_cap
+ *     bytes of neighbour logits.  Per-head graphs with d = 128 need about
+ *     6.4 MiB + the head + the logits; Hq/Hkv = 8 with d = 128 in per-group
+ *     mode needs over 32 MiB and is refused.
+ *   - If a launch fails, the call zeroes the array's head before returning
+ *     (an asynchronous memset on `stream`), so later calls start clean.
  *   - The first call on each device looks up the array's device address
  *     (with that device current); make that first call before any stream
  *     capture.  No call allocates or frees memory.
@@ -357,8 +361,8 @@ CKV_API ckv_status ckv_get_device_error(const ckv_graph_desc* graph, ckv_stream_
  */
 typedef enum {
     CKV_KERNEL_BUILD = 0,      /* the four kernels of ckv_build_centroids, as one */
-    CKV_KERNEL_SCORE = 1,      /* first scoring pass (ckv_score_select) */
-    CKV_KERNEL_SELECT = 2,     /* selection and token list (ckv_score_select) */
+    CKV_KERNEL_SCORE = 1,      /* ckv_score_select: scoring, selection and token list, one kernel */
+    CKV_KERNEL_SELECT = 2,     /* no kernel (kept so the kinds keep their numbers) */
     CKV_KERNEL_ATTENTION = 3,  /* split-K attention (sparse and dense decode) */
     CKV_KERNEL_MERGE = 4,      /* merge, neighbours and fused update */
     CKV_KERNEL_UPDATE = 5      /* ckv_assign_update / ckv_append_assign */
