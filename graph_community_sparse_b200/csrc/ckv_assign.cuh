@@ -94,21 +94,32 @@ inline AssignParams make_assign_params(const CacheView& c, const GraphView& g, i
     return p;
 }
 
+// Shared-memory scratch of one unit's update (the caller provides it: the
+// stand-alone kernel as a shared variable, the attention's merging warp in
+// its own staging ring, which is idle by then).
+template <int D>
+struct AssignScratch {
+    int cand[CKV_NEIGHBOURS];
+    float score[CKV_NEIGHBOURS];
+    int cnt[CKV_NEIGHBOURS];
+    int tl;
+    int pad[3];
+    float row[CKV_NEIGHBOURS][D];  // candidate centres, reused by the update
+};
+
 // The update of unit u by NW warps (thread index tid in [0, 32 NW)), given
 // the unit's 8 neighbour positions (-1: none) in nbrpos, readable by all of
-// them.  sync() is a barrier over exactly these NW warps.  Candidates are
-// scored NW at a time, one warp each, so all their centres are fetched in
-// one or two rounds; warp 0 picks the winner and moves its centre.
+// them.  sync() is a barrier over exactly these NW warps.  Warp w scores
+// candidates w, w + NW, ... with all of their centres requested before any
+// is used; warp 0 picks the winner and moves its centre.
 template <typename T, int D, int NW, typename Sync>
-__device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const int* nbrpos, int tid, Sync sync) {
+__device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const int* nbrpos, int tid,
+                                            AssignScratch<D>& sc, Sync sync) {
     constexpr int E = D / 32;
+    constexpr int PER = CKV_NEIGHBOURS / NW;  // candidates per warp
     static_assert(E == 2 || E == 4, "d is 64 or 128");
-    __shared__ int s_cand[CKV_NEIGHBOURS];
-    __shared__ float s_score[CKV_NEIGHBOURS];
-    __shared__ int s_cnt[CKV_NEIGHBOURS];
-    __shared__ float s_row[CKV_NEIGHBOURS][D];  // candidate centres, reused by the update
-    __shared__ int s_tl;
-    const int lane = tid & 31, warp = tid >> 5;
+    static_assert(CKV_NEIGHBOURS % NW == 0, "whole candidates per warp");
+    const int lane = tid & 31, warp = NW == 1 ? 0 : tid >> 5;
     const int b = u / p.G, g = u - b * p.G;
     const int gq = p.Hq / p.Hkv;
     const int kvh = p.per_head ? g / gq : g;
@@ -132,37 +143,52 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
             const int cc = p.comm_of[(size_t)u * p.T_cap + np];
             if (cc >= 0 && cc < p.Cmax) c = cc;
         }
-        s_cand[tid] = c;
+        sc.cand[tid] = c;
     }
-    if (tid == 0) s_tl = p.tail_len[u];
+    if (tid == 0) sc.tl = p.tail_len[u];
     const T* krow = static_cast<const T*>(p.k) + b * p.sb + kvh * p.sh + lane * E;
     float kx[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) kx[e] = to_f32(krow[e]);
     sync();
 
-    // warp w: scores of candidates w, w + NW, ... (-inf when absent or a repeat)
+    // this warp's candidates (-inf when absent or a repeat): rows first
+    bool use[PER];
+    int ci[PER];
+    float row[PER][E];
 #pragma unroll
-    for (int i = warp; i < CKV_NEIGHBOURS; i += NW) {
-        const int ci = s_cand[i];
-        bool use = ci >= 0;
-        for (int j = 0; j < i; ++j) use = use && s_cand[j] != ci;
-        float s = -INFINITY;
-        if (use) {
-            const float* cr = p.cent + ((size_t)u * p.Cmax + ci) * D + lane * E;
-            if (lane == 0) s_cnt[i] = p.cnt[(size_t)u * p.Cmax + ci];
-            float a = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const float c = cr[e];
-                s_row[i][lane * E + e] = c;
-                a = fmaf(kx[e], c, a);
+    for (int r = 0; r < PER; ++r) {
+        const int i = warp + r * NW;
+        ci[r] = sc.cand[i];
+        use[r] = ci[r] >= 0;
+        for (int j = 0; j < i; ++j) use[r] = use[r] && sc.cand[j] != ci[r];
+        const float* cr = p.cent + ((size_t)u * p.Cmax + max(ci[r], 0)) * D + lane * E;
+        if (use[r]) {
+            if constexpr (E == 4) {
+                const float4 v = *reinterpret_cast<const float4*>(cr);
+                row[r][0] = v.x; row[r][1] = v.y; row[r][2] = v.z; row[r][3] = v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2*>(cr);
+                row[r][0] = v.x; row[r][1] = v.y;
             }
+            if (lane == 0) sc.cnt[i] = p.cnt[(size_t)u * p.Cmax + ci[r]];
+        } else {
 #pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
-            s = a * p.inv_sqrt_d;
+            for (int e = 0; e < E; ++e) row[r][e] = 0.f;
         }
-        if (lane == 0) s_score[i] = use ? s : -INFINITY;
+    }
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+        const int i = warp + r * NW;
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            sc.row[i][lane * E + e] = row[r][e];
+            a = fmaf(kx[e], row[r][e], a);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) a += __shfl_xor_sync(FULL, a, o);
+        if (lane == 0) sc.score[i] = use[r] ? a * p.inv_sqrt_d : -INFINITY;
     }
     sync();
     if (warp != 0) return;  // warp 0 picks the winner and updates its row
@@ -173,15 +199,15 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     // low bits below the id, which is unique among the keys.
     unsigned long long key = 0ull;  // 0: no candidate
     if (lane < CKV_NEIGHBOURS) {
-        const int ci = s_cand[lane];
-        const float sc = s_score[lane];
-        const unsigned same = __match_any_sync(0xffu, ci);  // lanes 0..7 naming the same community
-        if (ci >= 0 && sc != -INFINITY) {
+        const int c = sc.cand[lane];
+        const float s = sc.score[lane];
+        const unsigned same = __match_any_sync(0xffu, c);  // lanes 0..7 naming the same community
+        if (c >= 0 && s != -INFINITY) {
             const unsigned v = p.vote ? (unsigned)__popc(same) : 0u;
-            unsigned b = __float_as_uint(sc + 0.0f);  // -0 ranks as +0
-            b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-            key = ((unsigned long long)v << 60) | ((unsigned long long)b << 16) |
-                  ((unsigned long long)(MAX_CMAX - 1 - ci) << 3) | (unsigned long long)lane;
+            unsigned bits = __float_as_uint(s + 0.0f);  // -0 ranks as +0
+            bits = (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+            key = ((unsigned long long)v << 60) | ((unsigned long long)bits << 16) |
+                  ((unsigned long long)(MAX_CMAX - 1 - c) << 3) | (unsigned long long)lane;
         }
     }
 #pragma unroll
@@ -191,11 +217,12 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     }
     int best = key ? MAX_CMAX - 1 - (int)((key >> 3) & 0x1fffu) : -1;
     const int bi = (int)(key & 7u);
-    if (best >= 0 && s_tl >= p.max_tail) {
+    const int tl = sc.tl;
+    if (best >= 0 && tl >= p.max_tail) {
         if (lane == 0) atomicOr(p.dev_err, CKV_DEVERR_TAIL_FULL);
         best = -1;
     }
-    const int n = best >= 0 ? s_cnt[bi] : 0;  // written by the candidate's warp above
+    const int n = best >= 0 ? sc.cnt[bi] : 0;  // written by the candidate's warp above
     if (lane == 0) {
         int32_t* cpos = p.comm_of + (size_t)u * p.T_cap + p.pos;
         if (best < 0) {
@@ -204,9 +231,9 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
         } else {
             p.cnt[(size_t)u * p.Cmax + best] = n + 1;
             *cpos = best;
-            p.tail_tok[(size_t)u * p.max_tail + s_tl] = p.pos;
-            p.tail_comm[(size_t)u * p.max_tail + s_tl] = best;
-            p.tail_len[u] = s_tl + 1;
+            p.tail_tok[(size_t)u * p.max_tail + tl] = p.pos;
+            p.tail_comm[(size_t)u * p.max_tail + tl] = best;
+            p.tail_len[u] = tl + 1;
             if (p.assigned) p.assigned[u] = best;
         }
     }
@@ -214,9 +241,9 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     // running mean: c <- c + (k - c) / (n + 1) (as (k - c) * (1/(n + 1)) + c,
     // one rounding more than a division), from the copy of the centre
     // taken while scoring
-    const size_t row = (size_t)u * p.Cmax + best;
-    float* cr = p.cent + row * D + lane * E;
-    const float* c0r = s_row[bi] + lane * E;
+    const size_t rowi = (size_t)u * p.Cmax + best;
+    float* cr = p.cent + rowi * D + lane * E;
+    const float* c0r = sc.row[bi] + lane * E;
     const float inv_n1 = __frcp_rn((float)(n + 1));  // one reciprocal, then products
     float c1[E], amax = 0.f;
 #pragma unroll
@@ -229,14 +256,14 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     // the int8 scoring copy follows the centre: new scale, new codes
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-    const float sc = q8_scale(amax), rc = q8_recip(amax);
+    const float scl = q8_scale(amax), rc = q8_recip(amax);
     uint32_t packed = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e) packed |= (uint32_t)(q8_code(c1[e], rc) & 0xff) << (8 * e);
-    int8_t* qr = p.cent_q + row * D + lane * E;
+    int8_t* qr = p.cent_q + rowi * D + lane * E;
     if constexpr (E == 4) *reinterpret_cast<uint32_t*>(qr) = packed;
     else *reinterpret_cast<uint16_t*>(qr) = (uint16_t)packed;
-    if (lane == 0) p.cent_qs[row] = sc;
+    if (lane == 0) p.cent_qs[rowi] = scl;
 }
 
 }  // namespace ckv

@@ -360,7 +360,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
 }
 
 template <typename T, int D, int GQ, bool DENSE>
-__global__ void __launch_bounds__(DEC_WARPS * 32, DecMinBlocks<T, GQ>::v) decode_main(DecodeParams p) {
+__global__ void __launch_bounds__(DEC_WARPS * 32, DecMinBlocks<T, GQ>::v) decode_main(const __grid_constant__ DecodeParams p) {
     extern __shared__ __align__(128) unsigned char smem[];
     pdl_wait();  // the selection comes from the kernel before
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -468,8 +468,9 @@ __device__ __forceinline__ int nbr_pos(unsigned long long k) {
 // neighbour warps (thread xt of 32 NBR_WARPS), given its neighbour positions.
 template <typename T, int D>
 __device__ __forceinline__ void merge_assign(const DecodeParams& p, int u, const int* nbpos, int xt) {
+    __shared__ __align__(16) AssignScratch<D> s_as;
     auto sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory"); };
-    assign_unit<T, D, NBR_WARPS>(p.ap, u, nbpos, xt, sync);
+    assign_unit<T, D, NBR_WARPS>(p.ap, u, nbpos, xt, s_as, sync);
 }
 
 // One block per unit: threads 0..D-1 own one output dimension each (all the
@@ -478,7 +479,7 @@ __device__ __forceinline__ void merge_assign(const DecodeParams& p, int u, const
 // merge: no shared memory and no barriers, so the merge costs about two
 // dependent rounds of loads.
 template <typename T, int D, int GQ, bool DENSE>
-__global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_merge(DecodeParams p) {
+__global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_merge(const __grid_constant__ DecodeParams p) {
     pdl_wait();  // the attention kernel's partials are complete and visible
     const int u = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     // no kernel of this call takes a ticket any more: return it to zero

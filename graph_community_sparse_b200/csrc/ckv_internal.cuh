@@ -252,9 +252,9 @@ struct SelView {
 
 // workspace carving
 // Workspace head, shared by every call on a workspace and zero before its
-// first use: the attention kernels' work ticket (WS_RESERVED bytes), then one
-// arrival counter per possible graph unit (B * Hq ints).  Every call leaves
-// the head zero.  The other parts of each call start after the head.
+// first use: the attention kernels' work ticket.  Every call leaves it zero
+// (the attention's merge returns the ticket).  The other parts of each call
+// start after the head.
 constexpr size_t WS_RESERVED = 256;
 
 struct DecodeWs {
@@ -296,7 +296,7 @@ cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos
                                  const void* v_new, const int32_t* nbr8, int32_t* assigned, cudaStream_t st);
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline size_t ws_head_bytes(int B, int Hq) { return WS_RESERVED + align256((size_t)B * Hq * 4); }
+inline size_t ws_head_bytes(int, int) { return WS_RESERVED; }
 
 // Programmatic dependent launch.  Kernels launched by launch_pdl() start
 // with pdl_wait(), so they read and write nothing before the previous kernel

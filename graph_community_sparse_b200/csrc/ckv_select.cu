@@ -49,7 +49,7 @@ constexpr int SEL_HBINS = 1 << SEL_HBITS;
 constexpr int SEL_FAST = SEL_THREADS;       // candidates ranked in shared memory
 constexpr int SC_LPR = 8;                   // lanes per centre row in the first pass
 constexpr int SC_RPI = 32 / SC_LPR;         // rows per warp instruction
-template <int GQ> struct ScRq { static constexpr int v = GQ == 1 ? 8 : GQ == 2 ? 4 : 2; };  // row groups per lane in flight
+template <int GQ> struct ScRq { static constexpr int v = GQ == 1 ? 4 : GQ == 2 ? 2 : 1; };  // row groups per lane in flight
 // Range of the integer query: q_i ~ sq Q_i with |Q_i| <= 127 * 128, so
 // Q_i = 128 hi_i + lo_i with hi_i in [-127, 127] and lo_i in [-64, 63].
 constexpr int Q_SPLIT = 127 * 128;
@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
     __shared__ __align__(16) float s_qf[GQ][D];
     __shared__ __align__(16) uint32_t s_qw[GQ][2][D / 4];
     __shared__ float s_sq[GQ], s_eb[GQ];
+    __shared__ float s_f[SEL_WARPS][32];  // first-pass sums of a warp's round, before the bounds
 
     constexpr int EW = D / 32;  // q elements per lane
     const int u = blockIdx.x;
@@ -265,6 +266,36 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
         s_cnt = 0;
     }
     pdl_wait();  // q, the centres and the counts may come from the kernels before
+
+    using CP = CodePart<D>;
+    constexpr int W = CP::W;
+    constexpr int RQ = ScRq<GQ>::v;
+    constexpr int STEP = SEL_WARPS * RQ * SC_RPI;  // rows per round of the block
+    const int sub = lane / SC_LPR, lr = lane % SC_LPR;
+    const int8_t* codes = p.cent_q + (size_t)u * p.Cmax * D + lr * (D / SC_LPR);
+    const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
+    // 1. first pass: lane lr of row group `sub` owns D/8 dims of one row; two
+    //    rounds of RQ row groups per warp in flight (the next round's codes are
+    //    requested before the current one is used).  The first round and the
+    //    rows' scales and sizes (to shared memory: s_ub, s_sz; each row's upper
+    //    bound later replaces its scale) are requested before anything else,
+    //    up to Cmax rows (the number present is not known yet)
+    CP cva[RQ], cvb[RQ];
+    auto load_codes = [&](CP (&cv)[RQ], int b0, int lim) {
+#pragma unroll
+        for (int j = 0; j < RQ; ++j) cv[j].load(codes + (size_t)min(b0 + j * SC_RPI + sub, lim - 1) * D);
+    };
+    int base = warp * RQ * SC_RPI;
+    if (base < p.Cmax) load_codes(cva, base, p.Cmax);
+    {
+        const float* scales = p.cent_qs + (size_t)u * p.Cmax;
+        for (int c = tid; c < p.Cmax; c += nt) {
+            cp_async_4(s_ub + c, scales + c);
+            cp_async_4(s_sz + c, cn + c);
+        }
+        cp_async_commit();
+    }
+    const int C = min(p.num_comm[u], p.Cmax);
 
     const int b = u / p.G, g = u - b * p.G;
     const int h0 = p.per_head ? g : g * GQ;
@@ -308,15 +339,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
             s_eb[warp] = fmaf(Q8_BOUND, qn, (127.0f * D * QSPLIT_BOUND) * sq);
         }
     }
+    cp_async_wait<0>();
     __syncthreads();
-    const int C = min(p.num_comm[u], p.Cmax);
-    const int32_t* cn = p.cnt + (size_t)u * p.Cmax;
 
-    // 1. first pass: lane lr of row group `sub` owns D/8 dims of one row
     {
-        using CP = CodePart<D>;
-        constexpr int W = CP::W;
-        const int sub = lane / SC_LPR, lr = lane % SC_LPR;
         constexpr int LG = GQ == 1 ? 0 : GQ == 2 ? 1 : GQ == 4 ? 2 : 3;
         const int hl = lr >> (3 - LG);  // head whose sum this lane ends up with
         const float sq_mine = s_sq[hl];
@@ -336,29 +362,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
                     qreg[h][1][k] = s_qw[h][1][lr * W + k];
                 }
         }
-        const int8_t* codes = p.cent_q + (size_t)u * p.Cmax * D + lr * (D / SC_LPR);
-        // the rows' scales and sizes go to shared memory (s_ub, s_sz) while
-        // the first codes load; each row's upper bound later replaces its scale
-        {
-            const float* scales = p.cent_qs + (size_t)u * p.Cmax;
-            for (int c = tid; c < C; c += nt) {
-                cp_async_4(s_ub + c, scales + c);
-                cp_async_4(s_sz + c, cn + c);
-            }
-            cp_async_commit();
-        }
-        constexpr int RQ = ScRq<GQ>::v;
-        constexpr int STEP = SEL_WARPS * RQ * SC_RPI;
-        CP cv[RQ];
-        auto load_codes = [&](int b0) {
-#pragma unroll
-            for (int j = 0; j < RQ; ++j) cv[j].load(codes + (size_t)min(b0 + j * SC_RPI + sub, C - 1) * D);
-        };
-        int base = warp * RQ * SC_RPI;
-        if (base < C) load_codes(base);
-        cp_async_wait<0>();
-        __syncthreads();
-        for (; base < C; base += STEP) {
+        float* my_f = s_f[warp];
+        // scores of the round's rows: each row group's sum goes to my_f, then
+        // lane i < RQ * SC_RPI finishes row base + i (bounds, histogram)
+        auto score_round = [&](const CP (&cv)[RQ], int b0) {
 #pragma unroll
             for (int j = 0; j < RQ; ++j) {
                 int acc[GQ];
@@ -383,17 +390,28 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
                 float f = (float)rowgroup_reduce_heads<GQ>(acc, lr) * sq_mine;
 #pragma unroll
                 for (int o = SC_LPR >> LG; o < SC_LPR; o <<= 1) f = fmaxf(f, __shfl_xor_sync(FULL, f, o));
-                const int c = base + j * SC_RPI + sub;
-                if (lr == 0 && c < C) {
-                    const float rs = s_ub[c];
-                    const int w = s_sz[c];
-                    const float sc = f * rs * p.inv_sqrt_d;
-                    const float err = fmaf(ebase, rs, Q8_ABS_BOUND);
-                    s_ub[c] = w > 0 ? sc + err : -INFINITY;
-                    if (w > 0) atomicAdd(&s_hist[(int)(score_key(sc - err, c) >> (64 - SEL_HBITS))], w);
-                }
+                if (lr == 0) my_f[j * SC_RPI + sub] = f;
             }
-            if (base + STEP < C) load_codes(base + STEP);
+            __syncwarp();
+            const int c = b0 + lane;
+            if (lane < RQ * SC_RPI && c < C) {
+                const float rs = s_ub[c];
+                const int w = s_sz[c];
+                const float sc = my_f[lane] * rs * p.inv_sqrt_d;
+                const float err = fmaf(ebase, rs, Q8_ABS_BOUND);
+                s_ub[c] = w > 0 ? sc + err : -INFINITY;
+                if (w > 0) atomicAdd(&s_hist[(int)(score_key(sc - err, c) >> (64 - SEL_HBITS))], w);
+            }
+            __syncwarp();
+        };
+        while (base < C) {
+            if (base + STEP < C) load_codes(cvb, base + STEP, C);
+            score_round(cva, base);
+            base += STEP;
+            if (base >= C) break;
+            if (base + STEP < C) load_codes(cva, base + STEP, C);
+            score_round(cvb, base);
+            base += STEP;
         }
     }
     __syncthreads();
@@ -401,7 +419,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
     // exact fp32 scores, from cent, of the n candidates whose keys (built
     // from the upper bounds) are in keys[]: one warp per candidate, RSC
     // candidates' rows in flight per warp; the keys are replaced in place
-    constexpr int RSC = GQ >= 4 ? 4 : 8;
+    constexpr int RSC = GQ >= 4 ? 2 : GQ == 2 ? 4 : 8;
     auto rescore = [&](unsigned long long* keys, int n) {
         for (int i0 = warp; i0 < n; i0 += RSC * nw) {
             float row[RSC][EW];

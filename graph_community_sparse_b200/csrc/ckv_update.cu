@@ -12,11 +12,12 @@ namespace ckv {
 template <typename T, int D>
 __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParams p) {
     __shared__ int s_nbr[CKV_NEIGHBOURS];
+    __shared__ __align__(16) AssignScratch<D> s_scratch;
     pdl_wait();  // everything this kernel reads may come from the kernel before it
     const int u = blockIdx.x;
     if (threadIdx.x < CKV_NEIGHBOURS) s_nbr[threadIdx.x] = p.nbr8[(size_t)u * CKV_NEIGHBOURS + threadIdx.x];
     __syncthreads();
-    assign_unit<T, D, CKV_NEIGHBOURS>(p, u, s_nbr, threadIdx.x, [] { __syncthreads(); });
+    assign_unit<T, D, CKV_NEIGHBOURS>(p, u, s_nbr, threadIdx.x, s_scratch, [] { __syncthreads(); });
 }
 
 cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const void* k_new,

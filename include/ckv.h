@@ -32,8 +32,7 @@
  *  - No call allocates device memory.  Scratch comes from the caller's
  *    workspace `ws` of `ws_bytes` bytes (256-byte aligned), sized by
  *    ckv_workspace_size(); a smaller workspace returns CKV_ERR_WORKSPACE.
- *    Its head (256 + 4 * B * Hq bytes rounded up to a multiple of 256: the
- *    attention kernels' work counter and one arrival counter per graph unit)
+ *    Its first 256 bytes (the head: the attention kernels' work counter)
  *    must be zero before the workspace's first use, e.g. zero-fill the whole
  *    workspace once after allocating it; every call leaves the head zero.  The rest needs no
  *    initialisation.  Calls sharing a workspace must not overlap on the GPU.
@@ -264,8 +263,8 @@ CKV_API ckv_status ckv_sparse_decode(const ckv_cache_desc* cache, const void* q,
  * until the process exits.
  *   - Calls needing more scratch than CKV_NOALLOC_SCRATCH_BYTES return
  *     CKV_ERR_UNSUPPORTED before touching the device.  The need is the size
- *     ckv_workspace_size reports for the attention alone: the head
- *     (256 + 4 * B * Hq bytes, rounded up to 256), about
+ *     ckv_workspace_size reports for the attention alone: the 256-byte
+ *     head, about
  *     4 * (12288 + 2U) * gq * (d + 2) bytes of split-K partials (gq query
  *     heads per graph, U = B * graphs per sequence) and 4 * U * sel->tok_cap
  *     bytes of neighbour logits.  Per-head graphs with d = 128 need about

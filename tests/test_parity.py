@@ -424,6 +424,7 @@ def test_kernel_timing_counts_each_launch():
     t = ckv.ckv_kernel_times()
     for kind in ("score", "attention", "merge"):
         assert t[kind][1] == 1 and t[kind][0] > 0.0, (kind, t[kind])
-    assert t["build"][1] == 0 and t["update"][1] == 0 and t["select"][1] == 0
+    # scoring and selection are one kernel; the update runs in the merge kernel
+    assert all(t[k][1] == 0 for k in ("build", "select", "update"))
     case.st.select(q, wl.budget)
     assert all(v[1] == 0 for v in ckv.ckv_kernel_times().values())
