@@ -38,6 +38,7 @@ import synth  # noqa: E402
 METRIC = "sparse decode steps/s at 128K ctx; achieved HBM GB/s vs B200 peak"
 DEFAULT_WORKLOAD = "qwen3_8b_128k_head"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 # score+select, attention, merge (the update runs inside the merge kernel)
 KERNELS_PER_STEP_UPDATE = 3
 KERNELS_PER_STEP_STATIC = 3
@@ -104,6 +105,14 @@ def csrc_digest() -> str:
         if f.endswith((".cu", ".cuh", ".h")) and f not in ("ckv_api.cu", "ckv_timing.cu"):
             h.update(f.encode() + b"\0" + open(os.path.join(d, f), "rb").read())
     return h.hexdigest()
+
+
+def call_traffic(workload: str):
+    """ncu DRAM bytes of one ckv_sparse_decode(_append) call: its attention
+    and merge kernels' committed figures, while both are current."""
+    a = profile_traffic("decode_main", workload)
+    m = profile_traffic("decode_merge", workload)
+    return a + m if a is not None and m is not None else None
 
 
 def profile_traffic(kernel: str, workload: str):
@@ -362,9 +371,20 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     barrier(device)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    # a longer sample of the same steps (each timed alone, L2 flushed before
+    # each), for the spread of the step time; not part of `value`
+    long_ms = []
+    if args.long_steps > 0:
+        lev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.long_steps)]
+        for j in range(args.long_steps):
+            new_episode_if_due()
+            flush()
+            one_step((W_steps + j) % n_total, lev[j])
+        torch.cuda.synchronize()
+        long_ms = [e[0].elapsed_time(e[1]) for e in lev]
     clk.__exit__()
     clocks = clk.summary()
-    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     total_s = sum(step_ms) / 1e3
     max_total_s = reduce_max(total_s, device)
 
@@ -469,23 +489,22 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         a["bytes"] = float(np.mean(attn_bytes))
         a["GB/s"] = a["bytes"] / (a["ms"] * 1e-3) / 1e9
         a["frac"] = a["GB/s"] / peak
-    dom_kind = max(per_kernel, key=lambda k: per_kernel[k]["ms"]) if per_kernel else None
-    if dom_kind == "attention":
-        a = per_kernel["attention"]
-        roofline = {"kernel": "decode_main (the split-K attention kernel of " + dec_name + ")", "bound": "hbm",
-                    "achieved": a["GB/s"], "peak": peak, "unit": "GB/s", "frac": a["frac"], "peak_source": peak_src,
-                    "traffic": profile_traffic("decode_main", wl.key) if n_layers == 1 else None,
-                    "bytes_per_launch": a["bytes"] / n_layers,
-                    "timing": "CUDA events the library records around each launch (ckv_kernel_timing) on the "
-                              f"launching stream, mean over a pass of {B_steps} steps after the timed ones{per}"}
-    else:
-        dom = max((dec_name, "ckv_score_select"), key=lambda k: kernels[k]["ms"])
-        roofline = {"kernel": dom, "bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": peak, "unit": "GB/s",
-                    "frac": kernels[dom]["GB/s"] / peak, "peak_source": peak_src,
-                    "traffic": profile_traffic(dom, wl.key) if n_layers == 1 else None,
-                    "bytes_per_launch": kernels[dom]["bytes"] / n_layers,
-                    "timing": "CUDA events around the library call on its stream, mean over a pass of "
-                              f"{B_steps} steps right after the timed ones{per}"}
+    # the roofline of the call the target names (ckv_sparse_decode, here with
+    # the fused append when the workload updates): its algorithmic bytes over
+    # its duration, against the measured copy peak and the nominal 8 TB/s;
+    # the attention kernel alone is in per_kernel
+    dk = kernels[dec_name]
+    roofline = {"kernel": dec_name + " (the call: split-K attention kernel, then the merge kernel"
+                          + (" that also runs the update)" if wl.update else ")"),
+                "bound": "hbm", "achieved": dk["GB/s"], "peak": peak, "unit": "GB/s", "frac": dk["GB/s"] / peak,
+                "peak_source": peak_src, "peak_nominal": NOMINAL_HBM_GBS,
+                "frac_nominal": dk["GB/s"] / NOMINAL_HBM_GBS,
+                "traffic": call_traffic(wl.key) if n_layers == 1 else None,
+                "bytes_per_launch": dk["bytes"] / n_layers,
+                "timing": "CUDA events on the launching stream around the call, mean over a pass of "
+                          f"{B_steps} steps right after the timed ones{per}"}
+    if "attention" in per_kernel:
+        per_kernel["attention"]["frac_nominal"] = per_kernel["attention"]["GB/s"] / NOMINAL_HBM_GBS
 
     # dense comparator on the same caches and queries
     dense_out = torch.empty_like(st0.out)
@@ -572,17 +591,25 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
     check_dev_err("host enqueue pass")
 
     value = job_value(n_ranks, K_steps, max_total_s)
+
+    def stats(ms):
+        a = np.asarray(ms, dtype=np.float64)
+        return {"n": int(a.size), "median": float(np.median(a)), "p10": float(np.percentile(a, 10)),
+                "p90": float(np.percentile(a, 90)), "min": float(a.min()), "max": float(a.max())}
+
+    spread = {"timed_steps": stats(step_ms)}
+    if long_ms:
+        spread["long_sample"] = dict(stats(long_ms), steps_per_s=1e3 / float(np.mean(long_ms)),
+                                     note="the same steps, each timed alone after an L2 flush, after the "
+                                          "timed ones; not part of value")
+    if clocks.get("sm_mhz"):
+        spread["median_ms_x_sm_mhz"] = float(np.median(step_ms)) * clocks["sm_mhz"]
     return {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": n_ranks, "steps": K_steps,
         "warmup": W_steps, "ms_per_step": max_total_s * 1e3 / K_steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic",
-        "config": {"workload": wl.key, "title": wl.title, "B_per_gpu": wl.B, "layers": n_layers, "Hq": wl.Hq,
-                   "Hkv": wl.Hkv, "d": wl.d, "ctx": wl.T, "graphs": "per query head" if per_head else "per KV group",
-                   "communities_per_graph": float(ncomm / (U * n_layers)), "budget": budget, "sinks": wl.S,
-                   "update": wl.update, "assign_rule": wl.assign_rule if wl.update else None,
-                   "layout": wl.layout,
-                   "l2": "flushed by a 1 GiB write then a 512 MiB read before every timed step, outside the CUDA events",
-                   "parallelism": f"dp{n_ranks} (independent batches, no collective)"},
+        "config": config_dict(wl, budget, n_layers, float(ncomm / (U * n_layers)), n_ranks),
+        "step_spread": spread,
         "tokens_per_s": value * wl.B,
         "roofline": roofline,
         "kernels": kernels,
@@ -600,6 +627,179 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
         "host_us_per_step_timed_loop": host_s / K_steps * 1e6,
         "episodes": episodes[0],
     }
+
+
+# ----------------------------------------------------------------------------
+# the other 128K / 64K configurations, measured in the same run (N = 1)
+# ----------------------------------------------------------------------------
+
+def measure_point(layers, wl: synth.Workload, budget: int, device, flush, steps: int, warmup: int,
+                  call_steps: int, dense_reps: int, first: int = 0) -> dict:
+    """One (workload, budget) point on already built layers: the step time
+    (`steps` steps, each bracketed by CUDA events after an L2 flush), the two
+    calls' times (events between them, `call_steps` steps), each kernel's time
+    (the library's own launch events, `call_steps` steps) and the dense
+    comparator (`dense_reps` runs)."""
+    import graph_community_sparse_b200 as ckv
+    n_layers = len(layers)
+    esz = 2 if wl.dtype == "bf16" else 4
+    row_bytes = 2 * wl.d * esz
+    T0 = wl.T
+
+    def step(i, ev=None):
+        for li, L in enumerate(layers):
+            if wl.update and L.st.T - T0 >= wl.steps:
+                L.build(T0)
+            q = L.qs[i]
+            if ev:
+                ev[2 * li].record()
+            L.st.select(q, budget)
+            if ev:
+                ev[2 * li + 1].record()
+            if wl.update:
+                k, v = L.news[i]
+                L.st.attend_append(q, k, v)
+            else:
+                L.st.attend(q, want_nbr=False)
+        if ev:
+            ev[-1].record()
+
+    i = first
+    for _ in range(warmup):
+        flush()
+        step(i)
+        i += 1
+    evs = []
+    for _ in range(steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record()
+        step(i)
+        e[1].record()
+        evs.append(e)
+        i += 1
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    # per call, with the rows each step reads
+    cevs, ntok, nsel = [], [], []
+    for _ in range(call_steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_layers + 1)]
+        step(i, e)
+        cevs.append(e)
+        ntok.append(sum(L.st.sel.n_tok.long().sum() for L in layers))
+        nsel.append(sum(L.st.sel.n_sel.long().sum() for L in layers))
+        i += 1
+    torch.cuda.synchronize()
+    sel_ms = [sum(e[2 * li].elapsed_time(e[2 * li + 1]) for li in range(n_layers)) for e in cevs]
+    dec_ms = [sum(e[2 * li + 1].elapsed_time(e[2 * li + 2]) for li in range(n_layers)) for e in cevs]
+    per_layer = None
+    if n_layers > 1:
+        per_layer = {"sel_us": [round(float(np.mean([e[2 * li].elapsed_time(e[2 * li + 1]) for e in cevs])) * 1e3, 2)
+                                for li in range(n_layers)],
+                     "attn_us": [round(float(np.mean([e[2 * li + 1].elapsed_time(e[2 * li + 2]) for e in cevs])) * 1e3,
+                                       2) for li in range(n_layers)]}
+    # per kernel (the library's launch events)
+    ckv.ckv_kernel_times()
+    ckv.ckv_kernel_timing(True)
+    try:
+        for _ in range(call_steps):
+            flush()
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    finally:
+        ckv.ckv_kernel_timing(False)
+    kt = ckv.ckv_kernel_times()
+    for L in layers:
+        err = int(L.st.graph.dev_err.item())
+        if err:
+            raise RuntimeError(f"{wl.key} budget {budget}: device error {err}")
+    ntok = float(np.mean([int(t.item()) for t in ntok]))
+    nsel = float(np.mean([int(t.item()) for t in nsel]))
+    peak, _ = measured_peaks()
+    q_bytes = n_layers * wl.B * wl.Hq * wl.d * esz
+    out_bytes = n_layers * wl.B * wl.Hq * wl.d * 4
+    # per-group graphs: one graph per KV head, so every list entry is a
+    # distinct K/V row
+    attn_bytes = ntok * row_bytes + ntok * 4 + q_bytes + (ntok * 4 if wl.update else 0)
+    dec_bytes = ntok * row_bytes + ntok * 4 + q_bytes + out_bytes
+    attn_ms = kt["attention"][0] / call_steps
+    res = {"budget": budget, "timed_steps": steps, "ms_per_step": float(np.mean(step_ms)),
+           "ms_per_step_median": float(np.median(step_ms)), "steps_per_s": 1e3 / float(np.mean(step_ms)),
+           "tokens_per_step": ntok, "communities_selected_per_step": nsel,
+           "select_ms": float(np.mean(sel_ms)), "decode_call_ms": float(np.mean(dec_ms)),
+           "decode_call_frac": dec_bytes / (float(np.mean(dec_ms)) * 1e-3) / 1e9 / peak,
+           "kernel_ms": {k: v[0] / call_steps for k, v in kt.items() if v[1] and k != "build"},
+           "attention_frac": attn_bytes / (attn_ms * 1e-3) / 1e9 / peak if attn_ms > 0 else None,
+           "per_layer": per_layer}
+    if dense_reps > 0:
+        dense_out = torch.empty_like(layers[0].st.out)
+        dms = []
+        for j in range(dense_reps + 1):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for L in layers:
+                L.st.dense(L.qs[0], dense_out)
+            e1.record()
+            dms.append((e0, e1))
+        torch.cuda.synchronize()
+        dms = [a.elapsed_time(b) for a, b in dms[1:]]
+        dense_bytes = n_layers * wl.B * wl.Hkv * layers[0].st.T * row_bytes + q_bytes + out_bytes
+        res["dense_ms"] = float(np.mean(dms))
+        res["dense_frac"] = dense_bytes / (res["dense_ms"] * 1e-3) / 1e9 / peak
+        res["sparse_step_speedup"] = res["dense_ms"] / res["ms_per_step"]
+    return res
+
+
+def run_sweeps(device, steps: int = 10, warmup: int = 3, call_steps: int = 5) -> dict:
+    """The Zipf budget sweep (128K, B 32, per-group graphs) and one 32-layer
+    Llama-3.1-8B-shaped step (64K, B 16, update), each with the dense
+    comparator, on the same GPU after the headline workload."""
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.float32, device=device)
+    clean_buf = torch.ones(128 * 1024 * 1024, dtype=torch.float32, device=device)
+    sink = torch.zeros((), dtype=torch.float32, device=device)
+
+    def flush():
+        flush_buf.fill_(1.0)
+        torch.sum(clean_buf, dim=0, out=sink)
+
+    out = {"note": f"{steps} timed steps per point after {warmup} warm-up steps, {call_steps} steps for the "
+                   "per-call and per-kernel times; L2 flushed before every step; peak = the measured copy peak"}
+    wl = synth.WORKLOADS["qwen3_8b_128k_zipf"]
+    n = warmup + steps + 2 * call_steps
+    t0 = time.perf_counter()
+    layers = [BenchLayer(wl, 0, device, wl.T, 1, n)]
+    for L in layers:
+        L.build(wl.T)
+    out[wl.key] = {"title": wl.title, "points": [measure_point(layers, wl, b, device, flush, steps, warmup,
+                                                               call_steps, 2) for b in wl.budgets],
+                   "setup_s": None}
+    out[wl.key]["setup_s"] = round(time.perf_counter() - t0, 1)
+    del layers
+    torch.cuda.empty_cache()
+    wl = synth.WORKLOADS["llama31_8b_64k"]
+    t0 = time.perf_counter()
+    layers = [BenchLayer(wl, l, device, wl.T + wl.steps + 8, wl.steps + 8, n) for l in range(wl.layers)]
+    for L in layers:
+        L.build(wl.T)
+    out[wl.key] = dict(title=wl.title, **measure_point(layers, wl, wl.budget, device, flush, steps, warmup,
+                                                        call_steps, 1))
+    out[wl.key]["setup_s"] = round(time.perf_counter() - t0, 1)
+    del layers
+    torch.cuda.empty_cache()
+    return out
+
+
+def config_dict(wl: synth.Workload, budget: int, n_layers: int, comm_per_graph: float, n_ranks: int) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": wl.key, "title": wl.title, "B_per_gpu": wl.B, "layers": n_layers, "Hq": wl.Hq,
+            "Hkv": wl.Hkv, "d": wl.d, "ctx": wl.T, "graphs": "per query head" if wl.mode == "head" else "per KV group",
+            "communities_per_graph": round(comm_per_graph, 3), "budget": budget, "sinks": wl.S,
+            "update": wl.update, "assign_rule": wl.assign_rule if wl.update else None, "layout": wl.layout,
+            "l2": "flushed by a 1 GiB write then a 512 MiB read before every timed step, outside the CUDA events",
+            "parallelism": f"dp{n_ranks} (independent batches, no collective)"}
 
 
 # ----------------------------------------------------------------------------
@@ -691,7 +891,8 @@ def run_reference(args, wl: synth.Workload, device) -> dict:
     return {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.key, "budget": budget},
+            "config": config_dict(wl, budget, wl.layers if args.layers is None else args.layers,
+                                  float(np.mean(draw.labels.max(axis=2) + 1)), 1),
             "cpu_baseline": cb, "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0}}
 
@@ -715,6 +916,10 @@ def parse(argv=None):
     ap.add_argument("--cpu-units", type=int, default=48, help="graph units the CPU baseline times")
     ap.add_argument("--ref-units", type=int, default=4, help="graph units per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--long-steps", type=int, default=300,
+                    help="extra steps timed one by one after the timed ones, for the step-time spread")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the Zipf budget sweep and the 32-layer step run after the headline (N = 1 only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -750,6 +955,9 @@ def main(argv=None):
             torch.cuda.empty_cache()
             res["cpu_baseline"] = cpu_baseline(wl, res["config"]["budget"], device, args.cpu_units,
                                                res["config"]["layers"])
+        if ws == 1 and not args.no_sweeps and args.workload == DEFAULT_WORKLOAD and args.batch is None:
+            torch.cuda.empty_cache()
+            res["sweeps"] = run_sweeps(device)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -30,9 +30,8 @@ __all__ = [
     "NEIGHBOURS",
 ]
 
-# CKV_LIB may name another build of the same library (e.g. one compiled with
-# different tuning constants); by default the in-tree build is loaded.
-LIB_PATH = os.environ.get("CKV_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckv.so")
+# the in-tree build, always: no environment variable selects another library
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckv.so")
 
 DTYPE_F32, DTYPE_BF16 = 0, 1
 PER_GROUP, PER_HEAD = 0, 1

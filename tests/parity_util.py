@@ -113,6 +113,7 @@ class Case:
         self.states: Dict[tuple, O.GraphState] = {}
         self._kv: Dict[tuple, tuple] = {}
         self.step_idx = 0
+        self.T_step = self.st.T
 
     # oracle-side helpers -------------------------------------------------
     def state(self, b: int, g: int) -> O.GraphState:
@@ -121,9 +122,12 @@ class Case:
         (those joins were not checked; later counts and centres are)."""
         if (b, g) not in self.states:
             st = O.GraphState(self.draw.labels[b, g], self.st.cache.T_cap, self.wl.S, self.Cmax)
-            if self.st.T > self.wl.T:
+            # the cache length when the current step began (a fused step has
+            # already appended its own token when the checks run)
+            T_known = min(self.st.T, self.T_step)
+            if T_known > self.wl.T:
                 u = b * self.wl.G + g
-                joined = self.st.graph.comm_of[u, self.wl.T: self.st.T].cpu().numpy()
+                joined = self.st.graph.comm_of[u, self.wl.T: T_known].cpu().numpy()
                 for i, c in enumerate(joined):
                     st.join(self.wl.T + i, int(c))
             self.states[(b, g)] = st
@@ -147,12 +151,26 @@ class Case:
 
     # one step ----------------------------------------------------------------
     def step(self, budget: int, units: Optional[Sequence[tuple]] = None, rep: Optional[Report] = None,
-             update: Optional[bool] = None, check_all_units: bool = True) -> Report:
+             update: Optional[bool] = None, check_all_units: bool = True, fused: bool = False) -> Report:
+        """One decode step, checked.  fused=True runs the attention and the
+        update as the benchmark does (ckv_sparse_decode_append, one call);
+        otherwise ckv_sparse_decode, then ckv_append_assign."""
         wl = self.wl
         rep = rep or Report()
         update = wl.update if update is None else update
+        self.T_step = self.st.T
         q = synth.draw_queries(wl, self.draw, self.step_idx, self.layer_idx)
-        out = self.st.decode(q, budget).clone()
+        fused_assigned = None
+        if fused and update:
+            self.st.select(q, budget)
+            cnt_before = self.st.graph.cnt.clone()  # the update below changes the counts
+            kn, vn = synth.draw_new_tokens(wl, self.draw, self.step_idx, self.layer_idx)
+            pos = self.st.T
+            out = self.st.attend_append(q, kn, vn).clone()
+            fused_assigned = self.st.assigned.clone()
+        else:
+            out = self.st.decode(q, budget).clone()
+            cnt_before = None
         torch.cuda.synchronize()
         sel_comm = self.st.sel.sel_comm.cpu().numpy()
         n_sel = self.st.sel.n_sel.cpu().numpy()
@@ -162,7 +180,7 @@ class Case:
         tok_prefix = self.st.sel.tok_prefix.cpu().numpy()
         tail_sel = self.st.sel.tail_sel.cpu().numpy()
         nbr = self.st.nbr8.cpu().numpy()
-        cnt_gpu = self.st.graph.cnt.cpu().numpy()
+        cnt_gpu = (cnt_before if cnt_before is not None else self.st.graph.cnt).cpu().numpy()
         assert prefix[0] == 0 and np.array_equal(np.diff(prefix), n_tok), "unit_prefix is not the scan of n_tok"
         if check_all_units:
             # cheap invariants on every unit
@@ -213,9 +231,12 @@ class Case:
             cand_cache[(b, g)] = cent
             rep.units_checked += 1
         if update:
-            kn, vn = synth.draw_new_tokens(wl, self.draw, self.step_idx, self.layer_idx)
-            pos = self.st.T
-            assigned = self.st.append(kn, vn).cpu().numpy()
+            if fused_assigned is not None:
+                assigned = fused_assigned.cpu().numpy()
+            else:
+                kn, vn = synth.draw_new_tokens(wl, self.draw, self.step_idx, self.layer_idx)
+                pos = self.st.T
+                assigned = self.st.append(kn, vn).cpu().numpy()
             torch.cuda.synchronize()
             for (b, g) in units:
                 u = b * wl.G + g

@@ -5,8 +5,10 @@ or a decode loop that must not call cudaMalloc because it can synchronise the
 device).  Its scratch is a fixed array inside the library.
 
 Checked through the C ABI against ckv_sparse_decode (the workspace version)
-on two calls in a row, within the parity tolerance; sizes beyond the fixed
-scratch are refused with a clear error before anything runs.  This file is
+on two calls in a row: both run the same kernels in the same order, so the
+outputs and neighbours must be identical bit for bit (which also catches a
+slip in how the fixed scratch is laid out); sizes beyond the fixed scratch
+are refused with a clear error before anything runs.  This file is
 collected last on purpose, and passes alone in a fresh process too.
 """
 import pytest
@@ -42,6 +44,7 @@ def test_noalloc_matches_workspace_decode_twice(key, extra):
         torch.cuda.synchronize()
         assert torch.isfinite(out2).all()
         assert float((out2 - ref_out).abs().max()) <= TOL[wl.dtype]
+        assert torch.equal(out2, ref_out)
         assert torch.equal(nbr2, ref_nbr)
 
 
