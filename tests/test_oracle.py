@@ -224,6 +224,65 @@ def test_centroid_is_running_mean_of_members():
         assert np.allclose(cent, run_c, rtol=0, atol=1e-12)
 
 
+def check_assign_worked(assign) -> bool:
+    """The default update rule on the hand-worked cases."""
+    # tests/golden/worked_examples.json "assign" (worked by hand there)
+    g = GOLDEN["assign"]
+    k, cent = _arr(g["k"]), _arr(g["cent"])
+    return all(assign(k, cent, cand) == expect for cand, expect in g["cases"])
+
+
+def check_graph_logits_worked(graph_logits) -> bool:
+    """Graph logits with their 1/sqrt(d) scale, in the order of the positions given."""
+    # tests/golden/worked_examples.json "graph_logits" (worked by hand there)
+    g = GOLDEN["graph_logits"]
+    lam = graph_logits(_arr(g["q"]), _arr(g["K"]), np.array(g["positions"]))
+    return bool(np.allclose(lam, _arr(g["logits"]), rtol=0, atol=1e-15))
+
+
+def test_assign_worked_examples():
+    assert check_assign_worked(O.assign)
+
+
+def test_graph_logits_worked_example():
+    assert check_graph_logits_worked(O.graph_logits)
+
+
+def _assign_ties_high(k, cent, cand):
+    best, bs = -1, -math.inf
+    for c in sorted(set(cand)):
+        s = float(np.dot(k, cent[c])) / math.sqrt(len(k))
+        if s >= bs:
+            best, bs = c, s
+    return best
+
+
+def _assign_first_candidate(k, cent, cand):
+    return cand[0] if cand else -1
+
+
+def _logits_unscaled(q, K, positions):
+    return (np.asarray(K)[np.asarray(positions)] @ np.asarray(q).T).max(axis=1)
+
+
+def _logits_mean_heads(q, K, positions):
+    return (np.asarray(K)[np.asarray(positions)] @ np.asarray(q).T).mean(axis=1) / math.sqrt(np.asarray(q).shape[1])
+
+
+def _logits_first_head(q, K, positions):
+    return (np.asarray(K)[np.asarray(positions)] @ np.asarray(q)[0]) / math.sqrt(np.asarray(q).shape[1])
+
+
+@pytest.mark.parametrize("mutant", [_assign_ties_high, _assign_first_candidate])
+def test_pins_catch_assign_mutants(mutant):
+    assert not check_assign_worked(mutant)
+
+
+@pytest.mark.parametrize("mutant", [_logits_unscaled, _logits_mean_heads, _logits_first_head])
+def test_pins_catch_graph_logit_mutants(mutant):
+    assert not check_graph_logits_worked(mutant)
+
+
 def test_assign_bruteforce_ties_and_one_update():
     rng = np.random.default_rng(17)
     d, C = 8, 6
