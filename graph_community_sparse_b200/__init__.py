@@ -24,26 +24,30 @@ __all__ = [
     "ckv_sparse_decode_append", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times",
     "KERNEL_KINDS",
     "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
-    "ckv_abi_version", "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
+    "ckv_abi_version", "ckv_debug_build", "load_debug_library", "DEBUG_LIB_PATH",
+    "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "ASSIGN_SCORE", "ASSIGN_VOTE",
-    "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP",
+    "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP", "DEVERR_INDEX",
     "NEIGHBOURS",
 ]
 
 # the in-tree build, always: no environment variable selects another library
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckv.so")
+# the same library built with device-side index checks (build.py --debug); it
+# is loaded only on request (load_debug_library)
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckv_debug.so")
 
 DTYPE_F32, DTYPE_BF16 = 0, 1
 PER_GROUP, PER_HEAD = 0, 1
 ASSIGN_SCORE, ASSIGN_VOTE = 0, 1
-DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP = 1, 2, 4, 8
+DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP, DEVERR_INDEX = 1, 2, 4, 8, 16
 NEIGHBOURS = 8
 KERNEL_KINDS = ("build", "score", "select", "attention", "merge", "update")
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
             "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
             "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times",
             "ckv_dense_decode",
-            "ckv_status_string", "ckv_last_error", "ckv_abi_version")
+            "ckv_status_string", "ckv_last_error", "ckv_abi_version", "ckv_debug_build")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -79,29 +83,58 @@ class SelectionDesc(ctypes.Structure):
 
 
 _P = ctypes.POINTER
-lib.ckv_workspace_size.argtypes = [_P(CacheDesc), _P(GraphDesc), _P(SelectionDesc), _P(_sz)]
-lib.ckv_build_centroids.argtypes = [_P(CacheDesc), _p, _i64, _i32, _P(GraphDesc), _p, _sz, _p]
-lib.ckv_score_select.argtypes = [_P(CacheDesc), _P(GraphDesc), _p, _i32, _P(SelectionDesc), _p, _sz, _p]
-lib.ckv_sparse_decode.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p, _sz, _p]
-lib.ckv_sparse_decode_noalloc.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p]
-lib.ckv_assign_update.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p]
-lib.ckv_append_assign.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p, _p, _p]
-lib.ckv_sparse_decode_append.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _i32, _p,
-                                         _p, _p, _p, _sz, _p]
-lib.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
-lib.ckv_get_device_error.argtypes = [_P(GraphDesc), _p, _P(ctypes.c_int32), _i32]
-lib.ckv_kernel_timing.argtypes = [_i32]
-lib.ckv_kernel_times.argtypes = [_P(ctypes.c_float), _P(ctypes.c_int32), _i32]
-for _f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
-           "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
-           "ckv_dense_decode", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times"):
-    getattr(lib, _f).restype = ctypes.c_int
-lib.ckv_status_string.argtypes = [ctypes.c_int]
-lib.ckv_status_string.restype = ctypes.c_char_p
-lib.ckv_last_error.argtypes = []
-lib.ckv_last_error.restype = ctypes.c_char_p
-lib.ckv_abi_version.argtypes = []
-lib.ckv_abi_version.restype = ctypes.c_int32
+
+
+def _declare(lib_: ctypes.CDLL) -> ctypes.CDLL:
+    """Argument and result types of every entry point of a loaded libckv."""
+    lib_.ckv_workspace_size.argtypes = [_P(CacheDesc), _P(GraphDesc), _P(SelectionDesc), _P(_sz)]
+    lib_.ckv_build_centroids.argtypes = [_P(CacheDesc), _p, _i64, _i32, _P(GraphDesc), _p, _sz, _p]
+    lib_.ckv_score_select.argtypes = [_P(CacheDesc), _P(GraphDesc), _p, _i32, _P(SelectionDesc), _p, _sz, _p]
+    lib_.ckv_sparse_decode.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p, _sz, _p]
+    lib_.ckv_sparse_decode_noalloc.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _p]
+    lib_.ckv_assign_update.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p]
+    lib_.ckv_append_assign.argtypes = [_P(CacheDesc), _P(GraphDesc), _i32, _p, _p, _p, _p, _p]
+    lib_.ckv_sparse_decode_append.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _i32,
+                                              _p, _p, _p, _p, _sz, _p]
+    lib_.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
+    lib_.ckv_get_device_error.argtypes = [_P(GraphDesc), _p, _P(ctypes.c_int32), _i32]
+    lib_.ckv_kernel_timing.argtypes = [_i32]
+    lib_.ckv_kernel_times.argtypes = [_P(ctypes.c_float), _P(ctypes.c_int32), _i32]
+    for f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
+              "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
+              "ckv_dense_decode", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times"):
+        getattr(lib_, f).restype = ctypes.c_int
+    lib_.ckv_status_string.argtypes = [ctypes.c_int]
+    lib_.ckv_status_string.restype = ctypes.c_char_p
+    lib_.ckv_last_error.argtypes = []
+    lib_.ckv_last_error.restype = ctypes.c_char_p
+    lib_.ckv_abi_version.argtypes = []
+    lib_.ckv_abi_version.restype = ctypes.c_int32
+    lib_.ckv_debug_build.argtypes = []
+    lib_.ckv_debug_build.restype = ctypes.c_int32
+    return lib_
+
+
+_declare(lib)
+_debug_lib: Optional[ctypes.CDLL] = None
+
+
+def load_debug_library() -> ctypes.CDLL:
+    """The debug build of the library (libckv_debug.so: every index a
+    caller's array feeds to a kernel is checked on the device), loaded on
+    first use, with the same entry points as `lib`.  Raises ImportError when
+    it has not been built (build.py --debug)."""
+    global _debug_lib
+    if _debug_lib is None:
+        if not os.path.exists(DEBUG_LIB_PATH):
+            raise ImportError(f"libckv_debug.so not built at {DEBUG_LIB_PATH}; run "
+                              "`python graph_community_sparse_b200/build.py --debug`")
+        _debug_lib = _declare(ctypes.CDLL(DEBUG_LIB_PATH))
+    return _debug_lib
+
+
+def ckv_debug_build() -> int:
+    return int(lib.ckv_debug_build())
 
 
 def ckv_status_string(status: int) -> str:

@@ -1,10 +1,14 @@
 """Compile libckv.so in-tree for sm_100a with nvcc (no GPU needed).
 
-    python graph_community_sparse_b200/build.py [-v] [-f]
+    python graph_community_sparse_b200/build.py [-v] [-f] [--debug | --all]
 
 Objects go to graph_community_sparse_b200/_build/, the library to
-graph_community_sparse_b200/libckv.so.  Only the ckv_* C symbols are exported
-(linker version script); the CUDA runtime is linked statically.
+graph_community_sparse_b200/libckv.so.  --debug builds libckv_debug.so
+instead (objects in _build_debug/, compiled with CKV_DEBUG: every index a
+caller's array feeds to a kernel is checked on the device, see
+ckv_debug_build in include/ckv.h); --all builds both.  Only the ckv_* C
+symbols are exported (linker version script); the CUDA runtime is linked
+statically.
 """
 from __future__ import annotations
 
@@ -19,6 +23,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libckv.so")
+BUILD_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libckv_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "-I", os.path.join(ROOT, "include"), "-I", CSRC]
@@ -42,18 +48,20 @@ def _stale(out: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
+def build(verbose: bool = False, force: bool = False, debug: bool = False) -> str:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    out_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    flags = FLAGS + (["-DCKV_DEBUG"] if debug else [])
+    os.makedirs(out_dir, exist_ok=True)
     headers = [os.path.join(ROOT, "include", "ckv.h")] + [
         os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
     objs = []
     jobs = []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [nvcc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+            cmd = [nvcc, *ARCH, *flags, "-c", src, "-o", obj]
             if verbose:
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
@@ -68,15 +76,20 @@ def build(verbose: bool = False, force: bool = False) -> str:
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode:
                 raise RuntimeError("nvcc failed: " + " ".join(cmd))
-    if force or jobs or _stale(LIB, objs):
-        link = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs,
+    if force or jobs or _stale(lib, objs):
+        link = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", lib, *objs,
                 "-Xlinker", "--version-script=" + os.path.join(CSRC, "ckv.map")]
         r = subprocess.run(link, capture_output=True, text=True)
         if r.returncode:
             sys.stderr.write(r.stdout + r.stderr)
             raise RuntimeError("link failed")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv, force="-f" in sys.argv))
+    v, f = "-v" in sys.argv, "-f" in sys.argv
+    if "--all" in sys.argv:
+        print(build(v, f))
+        print(build(v, f, debug=True))
+    else:
+        print(build(v, f, debug="--debug" in sys.argv))

@@ -173,6 +173,8 @@ extern "C" {
 
 int32_t ckv_abi_version(void) { return CKV_ABI_VERSION; }
 
+int32_t ckv_debug_build(void) { return ckv::kDebugChecks ? 1 : 0; }
+
 static_assert(ckv::KK_COUNT == CKV_KERNEL_KINDS && ckv::KK_ATTENTION == CKV_KERNEL_ATTENTION &&
                   ckv::KK_UPDATE == CKV_KERNEL_UPDATE,
               "kernel kinds match the header");

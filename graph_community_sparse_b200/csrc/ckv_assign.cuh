@@ -222,6 +222,10 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
         if (lane == 0) atomicOr(p.dev_err, CKV_DEVERR_TAIL_FULL);
         best = -1;
     }
+    if (best >= 0 && tl < 0) {  // a corrupted tail length: never written through
+        if (lane == 0 && kDebugChecks) atomicOr(p.dev_err, CKV_DEVERR_INDEX);
+        best = -1;
+    }
     const int n = best >= 0 ? sc.cnt[bi] : 0;  // written by the candidate's warp above
     if (lane == 0) {
         int32_t* cpos = p.comm_of + (size_t)u * p.T_cap + p.pos;

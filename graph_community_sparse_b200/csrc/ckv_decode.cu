@@ -118,6 +118,8 @@ struct DecodeParams {
     int32_t* unit_prefix;   // written by block 0 of the attention kernel
     const int32_t* n_tok;
     int T;                  // dense only: tokens per unit
+    int T_cap;              // rows per (sequence, KV head): debug checks of positions
+    int32_t* dev_err;       // the graph's error word (debug checks; NULL for dense)
     float scale_log2;
     DecodeWs ws;
     int W;                  // warps in the grid
@@ -216,6 +218,7 @@ __device__ __forceinline__ void process_segment(const DecodeParams& p, int u, in
                 pos = lo + i;
             } else {
                 pos = __shfl_sync(ckv::FULL, win_cur, ((it & 3) << 3) + 2 * j + half);
+                pos = checked_index(pos, 0, p.T_cap, p.dev_err, 0);
             }
             if (!ALL_VALID) pos = valid ? pos : 0;
             const int64_t off = (int64_t)pos * st;
@@ -377,7 +380,13 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, DecMinBlocks<T, GQ>::v) decode
         const int b0 = min(p.U, (int)threadIdx.x * seg), b1 = min(p.U, b0 + seg);
         int own = 0;
         for (int i = b0; i < b1; ++i) {
-            const int x = p.n_tok[i];
+            int x = p.n_tok[i];
+            if constexpr (kDebugChecks) {
+                if (x < 0 || x > p.tok_cap) {
+                    atomicOr(p.dev_err, CKV_DEVERR_INDEX);
+                    x = max(0, min(x, p.tok_cap));
+                }
+            }
             s_pre[i] = x;
             own += x;
         }
@@ -783,6 +792,8 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
     p.S = g.S;
     p.sel_tok = s.sel_tok;
     p.tok_cap = s.tok_cap;
+    p.T_cap = c.T_cap;
+    p.dev_err = g.dev_err;
     p.unit_prefix = s.unit_prefix;
     p.n_tok = s.n_tok;
     p.scale_log2 = 1.4426950408889634f / sqrtf((float)c.d);

@@ -124,6 +124,7 @@ __device__ __forceinline__ void process_segment_mma(const DecodeParams& p, int u
                     pos = lo + it * MMA_TOK + r;
                 } else {
                     pos = __shfl_sync(FULL, win_cur, ((it & 1) << 4) + r);
+                    pos = checked_index(pos, 0, p.T_cap, p.dev_err, 0);
                 }
                 const bool valid = r < rem;
                 pos = valid ? pos : 0;

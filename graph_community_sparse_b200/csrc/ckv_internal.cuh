@@ -58,6 +58,27 @@ __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // ---------------------------------------------------------------------------
+// Debug builds (CKV_DEBUG) check every index that a caller's array feeds to a
+// kernel before using it; a bad one sets CKV_DEVERR_INDEX in the error word
+// and is replaced by a harmless value.  Release builds compile the checks out.
+// ---------------------------------------------------------------------------
+#ifdef CKV_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+// i if lo <= i < hi; otherwise (debug builds) `fallback`, with the error bit set
+__device__ __forceinline__ int checked_index(int i, int lo, int hi, int32_t* err, int fallback) {
+    if constexpr (kDebugChecks) {
+        if (i < lo || i >= hi) {
+            if (err) atomicOr(err, CKV_DEVERR_INDEX);
+            return fallback;
+        }
+    }
+    return i;
+}
+
+// ---------------------------------------------------------------------------
 // The int8 scoring copy of a centre row: scale s = max_i |c_i| / 127 and code
 // round-half-even(c_i * r) with r = 127 / max_i |c_i| (both divisions IEEE,
 // the product fp32; 0 for an all-zero row).  c_i r is within 127 * 2^-23 of

@@ -104,6 +104,19 @@ __device__ __forceinline__ int key_id(unsigned long long k) {
     return (int)(0xffffffffu - (unsigned)(k & 0xffffffffull));
 }
 
+// Community c's build-time run [o0, o1) in the member list; debug builds
+// check 0 <= o0 <= o1 <= T_cap (an empty run otherwise, with the error bit).
+__device__ __forceinline__ void member_run(const int32_t* of, int c, int T_cap, int32_t* err, int& o0, int& o1) {
+    o0 = of[c];
+    o1 = of[c + 1];
+    if constexpr (kDebugChecks) {
+        if (o0 < 0 || o1 < o0 || o1 > T_cap) {
+            atomicOr(err, CKV_DEVERR_INDEX);
+            o0 = o1 = 0;
+        }
+    }
+}
+
 // In-place inclusive scan of n ints (shared or global memory, visible to the
 // whole block); returns the total.
 __device__ int block_scan_inplace(int* a, int n, int* s_warp) {
@@ -525,8 +538,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
     int o0 = 0, o1 = 0;
     if (tid < min(nc, SEL_FAST)) {
         const int c = key_id(s_key[tid]);
-        o0 = of[c];
-        o1 = of[c + 1];
+        member_run(of, c, p.T_cap, p.dev_err, o0, o1);
     }
     if (nc <= SEL_FAST) {
         rescore(s_key, nc);
@@ -655,8 +667,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
         sorted = gk;
         __syncthreads();
         for (int i = tid; i < kstar; i += nt) {  // gw's weights are no longer needed
-            const int c = key_id(gk[i]);
-            bsz[i] = of[c + 1] - of[c];
+            int r0, r1;
+            member_run(of, key_id(gk[i]), p.T_cap, p.dev_err, r0, r1);
+            bsz[i] = r1 - r0;
         }
     }
 
@@ -731,10 +744,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
         }
     } else {
         for (int k = warp; k < kstar; k += nw) {
-            const int c = key_id(sorted[k]);
-            const int len = of[c + 1] - of[c];
+            int src, r1;
+            member_run(of, key_id(sorted[k]), p.T_cap, p.dev_err, src, r1);
+            const int len = r1 - src;
             const int dst = p.S + bsz[k] - len;
-            const int src = of[c];
             for (int i = lane; i < len; i += 32) {
                 if (dst + i < p.tok_cap) out[dst + i] = tk[src + i];
                 else overflow = true;
@@ -744,7 +757,13 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) score_select_kernel(SelectPara
     {
         // tail members of the selected communities, in tail order: the whole
         // block flags one entry per thread per round and compacts by a scan
-        const int tl = min(p.tail_len[u], p.max_tail);
+        int tl = min(p.tail_len[u], p.max_tail);
+        if constexpr (kDebugChecks) {
+            if (tl < 0) {
+                if (tid == 0) atomicOr(p.dev_err, CKV_DEVERR_INDEX);
+                tl = 0;
+            }
+        }
         const int32_t* tt = p.tail_tok + (size_t)u * p.max_tail;
         const int32_t* tc = p.tail_comm + (size_t)u * p.max_tail;
         int base = p.S + nb;

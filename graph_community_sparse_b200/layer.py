@@ -6,6 +6,7 @@ order.  It computes nothing itself.
 """
 from __future__ import annotations
 
+import contextlib
 from typing import Optional
 
 import torch
@@ -14,6 +15,17 @@ from . import (ASSIGN_SCORE, ASSIGN_VOTE, PER_GROUP, PER_HEAD, Graph, Selection,
                ckv_sparse_decode_append,
                ckv_build_centroids, ckv_dense_decode, ckv_score_select, ckv_sparse_decode,
                ckv_workspace_size, new_graph, new_selection, new_workspace, NEIGHBOURS)
+
+
+@contextlib.contextmanager
+def _range(name: str):
+    """An NVTX range around one library call, so that a profiler's timeline
+    names the step's parts; a no-op when no profiler is attached."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
 
 
 class LayerState:
@@ -53,15 +65,18 @@ class LayerState:
 
     def build(self, labels: torch.Tensor, T: int, stream=None) -> None:
         """labels: int32 [U, >=T] on the device."""
-        ckv_build_centroids(self.cache, labels, T, self.graph, self.ws, stream)
+        with _range("ckv_build_centroids"):
+            ckv_build_centroids(self.cache, labels, T, self.graph, self.ws, stream)
         self.T = T
 
     def select(self, q: torch.Tensor, budget: int, stream=None) -> None:
-        ckv_score_select(self.cache, self.graph, q, budget, self.sel, self.ws, stream)
+        with _range("ckv_score_select"):
+            ckv_score_select(self.cache, self.graph, q, budget, self.sel, self.ws, stream)
 
     def attend(self, q: torch.Tensor, want_nbr: bool = True, stream=None) -> torch.Tensor:
-        ckv_sparse_decode(self.cache, q, self.graph, self.sel, self.out,
-                          self.nbr8 if want_nbr else None, self.ws, stream)
+        with _range("ckv_sparse_decode"):
+            ckv_sparse_decode(self.cache, q, self.graph, self.sel, self.out,
+                              self.nbr8 if want_nbr else None, self.ws, stream)
         return self.out
 
     def decode(self, q: torch.Tensor, budget: int, want_nbr: bool = True, stream=None) -> torch.Tensor:
@@ -72,8 +87,9 @@ class LayerState:
         """attend (neighbours into nbr8) and append in one call: the update
         runs inside the attention's merge kernel."""
         pos = self.T
-        ckv_sparse_decode_append(self.cache, q, self.graph, self.sel, self.out, self.nbr8, pos, k_new.contiguous(),
-                                 v_new.contiguous(), self.assigned, self.ws, stream)
+        with _range("ckv_sparse_decode_append"):
+            ckv_sparse_decode_append(self.cache, q, self.graph, self.sel, self.out, self.nbr8, pos,
+                                     k_new.contiguous(), v_new.contiguous(), self.assigned, self.ws, stream)
         self.T += 1
         return self.out
 
@@ -81,8 +97,9 @@ class LayerState:
         """Write the new token's K/V rows ([B, Hkv, d]) at position T and let
         it join a community: one library call (ckv_append_assign)."""
         pos = self.T
-        ckv_append_assign(self.cache, self.graph, pos, k_new.contiguous(), v_new.contiguous(), self.nbr8,
-                          self.assigned, stream)
+        with _range("ckv_append_assign"):
+            ckv_append_assign(self.cache, self.graph, pos, k_new.contiguous(), v_new.contiguous(), self.nbr8,
+                              self.assigned, stream)
         self.T += 1
         return self.assigned
 
@@ -92,11 +109,13 @@ class LayerState:
         pos = self.T
         self.K[:, :, pos].copy_(k_new)
         self.V[:, :, pos].copy_(v_new)
-        ckv_assign_update(self.cache, self.graph, pos, self.nbr8, self.assigned, stream)
+        with _range("ckv_assign_update"):
+            ckv_assign_update(self.cache, self.graph, pos, self.nbr8, self.assigned, stream)
         self.T += 1
         return self.assigned
 
     def dense(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
         out = torch.empty_like(self.out) if out is None else out
-        ckv_dense_decode(self.cache, q, self.T, out, self.ws, stream)
+        with _range("ckv_dense_decode"):
+            ckv_dense_decode(self.cache, q, self.T, out, self.ws, stream)
         return out

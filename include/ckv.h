@@ -101,6 +101,9 @@ typedef enum { CKV_ASSIGN_SCORE = 0, CKV_ASSIGN_VOTE = 1 } ckv_assign_rule;
 #define CKV_DEVERR_LABEL_RANGE 2  /* a label outside [0, Cmax) at a position >= S      */
 #define CKV_DEVERR_TAIL_FULL 4    /* ckv_assign_update found the tail full; not joined */
 #define CKV_DEVERR_TOKEN_CAP 8    /* a selection longer than tok_cap was truncated     */
+#define CKV_DEVERR_INDEX 16       /* debug builds: an index read from a caller's array
+                                     (a position, a run offset, a token count, a tail
+                                     length) was out of range; the access was skipped */
 
 /*
  * The full KV cache of one layer: K and V are [B, Hkv, T_cap, d] with the d
@@ -369,6 +372,20 @@ typedef enum {
 #define CKV_KERNEL_KINDS 6
 CKV_API ckv_status ckv_kernel_timing(int32_t enable);
 CKV_API ckv_status ckv_kernel_times(float* total_ms, int32_t* launches, int32_t n);
+
+/*
+ * 1 in the debug build of the library (libckv_debug.so, compiled with
+ * CKV_DEBUG), 0 otherwise.  The debug build checks, on the device, every
+ * index that a caller's array feeds to a kernel before using it: the
+ * positions in sel_tok and n_tok against T_cap and tok_cap (attention), the
+ * CSR run offsets against T_cap (selection), the tail length against
+ * [0, max_tail] (selection, update).  A bad one sets CKV_DEVERR_INDEX in
+ * dev_err and the access is skipped or clamped: results are then wrong but
+ * nothing outside the arrays is touched, and no kernel traps.  Arithmetic
+ * and results on valid inputs are those of the release build.  (A negative
+ * tail length skips the join in every build.)
+ */
+CKV_API int32_t ckv_debug_build(void);
 
 CKV_API const char* ckv_status_string(ckv_status status);
 /* Message of the last failed call on this host thread ("" if none). */
