@@ -33,6 +33,10 @@ in that order:
    (ties to the lower id), or, under the other reading (assign_vote), the
    community holding the most of the 8 neighbours, ties to the larger
    k_new . c / sqrt(d) and then the lower id.
+7. At prefill (before decoding), the token graph the partition is computed
+   from: direct edges from a query to the keys it attends most, and
+   co-attention edges between keys attended together, with the sinks kept
+   out (direct_edges, coattention_edges; the partition itself is not built).
 
 Every centre is recomputed from the member lists whenever it is needed; the
 oracle never updates a mean incrementally.  Pins: see tests/test_oracle.py
@@ -216,6 +220,48 @@ def assign_vote(k_new: np.ndarray, cent: np.ndarray, neighbour_comms: Sequence[i
         if best < 0 or key > best_key:
             best, best_key = c, key
     return best
+
+
+# ----------------------------------------------------------------------------
+# the token graph at prefill (the input of the partition, which is not built)
+# ----------------------------------------------------------------------------
+
+def direct_edges(q_heads_seq: np.ndarray, K: np.ndarray, S: int, T: int,
+                 k: int = NEIGHBOURS) -> List[np.ndarray]:
+    """Direct edges of the prefill token graph (rit.work summary, section "A
+    graph of tokens replaces re-clustering", paragraph 3: a query that pays a
+    key much attention links the two; the first tokens are kept out of the
+    graph).  Reading used: for every query position i in [S, T), the k key
+    positions j in [S, i) with the largest graph logit
+    max over the graph's heads of q_{h,i} . k_j / sqrt(d) (the rule of the
+    decode-time neighbours), ties to the lower position, best first.
+    q_heads_seq: [heads, >=T, d] (the graph's query heads over the prefill);
+    K: [>=T, d].  Returns one array per query position, indexed by i - S."""
+    q_heads_seq = np.asarray(q_heads_seq, dtype=np.float64)
+    out = []
+    for i in range(S, T):
+        pos = np.arange(S, i, dtype=np.int64)
+        if len(pos) == 0:
+            out.append(pos)
+            continue
+        lam = graph_logits(q_heads_seq[:, i, :], K, pos)
+        order = np.lexsort((pos, -lam))   # logit descending, then position ascending
+        out.append(pos[order[:k]])
+    return out
+
+
+def coattention_edges(direct: Sequence[np.ndarray]) -> Dict[tuple, int]:
+    """Co-attention edges of the prefill token graph (same paragraph: keys
+    that are looked at together are linked).  Reading used: every pair of
+    keys j < l that appear in the same query's direct edges is linked, with
+    the number of such queries as its weight."""
+    w: Dict[tuple, int] = {}
+    for lst in direct:
+        ps = sorted(int(p) for p in lst)
+        for a in range(len(ps)):
+            for b in range(a + 1, len(ps)):
+                w[(ps[a], ps[b])] = w.get((ps[a], ps[b]), 0) + 1
+    return w
 
 
 # ----------------------------------------------------------------------------

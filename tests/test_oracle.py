@@ -501,3 +501,117 @@ def test_pins_catch_vote_mutants(mutant):
 def test_pins_catch_dropped_sinks(monkeypatch):
     monkeypatch.setattr(O, "token_set", _mut_token_set_no_sinks)
     assert not check_dense_equivalence(O.decode_graph)
+
+
+# ----------------------------------------------------------------------------
+# the token graph at prefill: direct and co-attention edges
+# ----------------------------------------------------------------------------
+
+def check_edges_worked(direct_edges, coattention_edges) -> bool:
+    # tests/golden/worked_examples.json "edges" (worked by hand there)
+    g = GOLDEN["edges"]
+    q = _arr(g["q"])[None]            # one head: [1, T, d]
+    K = _arr(g["K"])
+    d = direct_edges(q, K, g["S"], g["T"], k=g["k"])
+    if [list(map(int, x)) for x in d] != g["direct"]:
+        return False
+    w = coattention_edges(d)
+    return sorted([j, l, c] for (j, l), c in w.items()) == g["coattention"]
+
+
+def _brute_direct(q_heads_seq, K, S, T, k=8):
+    """Per query, the keys before it (sinks excluded) ranked by counting how
+    many beat each one (logit, then lower position), the first k."""
+    out = []
+    for i in range(S, T):
+        pos = list(range(S, i))
+        lam = {p: max(float(np.dot(q_heads_seq[h, i], K[p])) for h in range(q_heads_seq.shape[0])) for p in pos}
+
+        def better(a, b):
+            return lam[a] > lam[b] or (lam[a] == lam[b] and a < b)
+
+        rank = {p: sum(better(o, p) for o in pos) for p in pos}
+        out.append([p for p in sorted(pos, key=lambda p: rank[p]) if rank[p] < k])
+    return out
+
+
+def check_edges_bruteforce(direct_edges, coattention_edges, trials=12, seed=29) -> bool:
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        H, T, S, d = int(rng.integers(1, 4)), int(rng.integers(2, 40)), int(rng.integers(0, 5)), 8
+        S = min(S, T - 1)
+        q = rng.integers(-1, 2, (H, T, d)).astype(np.float64)    # integer data: many ties
+        K = rng.integers(-2, 3, (T, d)).astype(np.float64)
+        K[:S] += 10.0                                             # sinks would win if they were keys
+        got = [list(map(int, x)) for x in direct_edges(q, K, S, T)]
+        if got != _brute_direct(q, K, S, T):
+            return False
+        # co-attention: the weight of each key pair is the number of lists
+        # holding both; their total is the number of pairs over the lists
+        w = coattention_edges([np.array(x) for x in got])
+        for (j, l), c in w.items():
+            if not (j < l and c == sum(1 for x in got if j in x and l in x)):
+                return False
+        if sum(w.values()) != sum(len(x) * (len(x) - 1) // 2 for x in got):
+            return False
+    return True
+
+
+def test_edges_worked_example():
+    assert check_edges_worked(O.direct_edges, O.coattention_edges)
+
+
+def test_edges_bruteforce():
+    assert check_edges_bruteforce(O.direct_edges, O.coattention_edges)
+
+
+def _edges_with_sinks(q, K, S, T, k=8):
+    return O.direct_edges(q, K, 0, T, k)[S:] if S <= T else []
+
+
+def _edges_with_self(q, K, S, T, k=8):
+    out = []
+    for i in range(S, T):
+        pos = np.arange(S, i + 1)
+        lam = O.graph_logits(np.asarray(q)[:, i, :], K, pos)
+        out.append(pos[np.lexsort((pos, -lam))[:k]])
+    return out
+
+
+def _edges_future_keys(q, K, S, T, k=8):
+    out = []
+    for i in range(S, T):
+        pos = np.array([p for p in range(S, T) if p != i], dtype=np.int64)
+        lam = O.graph_logits(np.asarray(q)[:, i, :], K, pos) if len(pos) else np.zeros(0)
+        out.append(pos[np.lexsort((pos, -lam))[:k]] if len(pos) else pos)
+    return out
+
+
+def _edges_ties_high(q, K, S, T, k=8):
+    out = []
+    for i in range(S, T):
+        pos = np.arange(S, i)
+        lam = O.graph_logits(np.asarray(q)[:, i, :], K, pos) if len(pos) else np.zeros(0)
+        out.append(pos[np.lexsort((-pos, -lam))[:k]] if len(pos) else pos)
+    return out
+
+
+def _coattention_ordered(direct):
+    w = {}
+    for lst in direct:
+        for a in lst:
+            for b in lst:
+                if a != b:
+                    w[(int(a), int(b))] = w.get((int(a), int(b)), 0) + 1
+    return {key: c for key, c in w.items()}
+
+
+@pytest.mark.parametrize("mutant", [_edges_with_sinks, _edges_with_self, _edges_future_keys, _edges_ties_high])
+def test_pins_catch_edge_mutants(mutant):
+    assert not (check_edges_worked(mutant, O.coattention_edges)
+                and check_edges_bruteforce(mutant, O.coattention_edges))
+
+
+def test_pins_catch_coattention_mutant():
+    assert not (check_edges_worked(O.direct_edges, _coattention_ordered)
+                and check_edges_bruteforce(O.direct_edges, _coattention_ordered))
