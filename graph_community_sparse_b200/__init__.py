@@ -25,6 +25,7 @@ __all__ = [
     "KERNEL_KINDS",
     "ckv_dense_decode", "ckv_status_string", "ckv_last_error",
     "ckv_abi_version", "ckv_debug_build", "load_debug_library", "DEBUG_LIB_PATH",
+    "ckv_edges_workspace_size", "ckv_build_edges", "Edges", "new_edges", "DEVERR_EDGE_CAP",
     "EXPORTED", "DTYPE_F32", "DTYPE_BF16", "PER_GROUP", "PER_HEAD",
     "ASSIGN_SCORE", "ASSIGN_VOTE",
     "DEVERR_SINK_LABEL", "DEVERR_LABEL_RANGE", "DEVERR_TAIL_FULL", "DEVERR_TOKEN_CAP", "DEVERR_INDEX",
@@ -41,12 +42,14 @@ DTYPE_F32, DTYPE_BF16 = 0, 1
 PER_GROUP, PER_HEAD = 0, 1
 ASSIGN_SCORE, ASSIGN_VOTE = 0, 1
 DEVERR_SINK_LABEL, DEVERR_LABEL_RANGE, DEVERR_TAIL_FULL, DEVERR_TOKEN_CAP, DEVERR_INDEX = 1, 2, 4, 8, 16
+DEVERR_EDGE_CAP = 32
 NEIGHBOURS = 8
-KERNEL_KINDS = ("build", "score", "select", "attention", "merge", "update")
+KERNEL_KINDS = ("build", "score", "select", "attention", "merge", "update", "edges")
 EXPORTED = ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
             "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
             "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times",
             "ckv_dense_decode",
+            "ckv_edges_workspace_size", "ckv_build_edges",
             "ckv_status_string", "ckv_last_error", "ckv_abi_version", "ckv_debug_build")
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -97,12 +100,16 @@ def _declare(lib_: ctypes.CDLL) -> ctypes.CDLL:
     lib_.ckv_sparse_decode_append.argtypes = [_P(CacheDesc), _p, _P(GraphDesc), _P(SelectionDesc), _p, _p, _i32,
                                               _p, _p, _p, _p, _sz, _p]
     lib_.ckv_dense_decode.argtypes = [_P(CacheDesc), _p, _i32, _p, _p, _sz, _p]
+    lib_.ckv_edges_workspace_size.argtypes = [_P(CacheDesc), _i32, _i32, _i32, _P(_sz)]
+    lib_.ckv_build_edges.argtypes = [_P(CacheDesc), _i32, _i32, _p, _i32, _p, _p, _p, _p, _p, _p, _i32, _p, _p, _sz,
+                                     _p]
     lib_.ckv_get_device_error.argtypes = [_P(GraphDesc), _p, _P(ctypes.c_int32), _i32]
     lib_.ckv_kernel_timing.argtypes = [_i32]
     lib_.ckv_kernel_times.argtypes = [_P(ctypes.c_float), _P(ctypes.c_int32), _i32]
     for f in ("ckv_workspace_size", "ckv_build_centroids", "ckv_score_select", "ckv_sparse_decode",
               "ckv_sparse_decode_noalloc", "ckv_assign_update", "ckv_append_assign", "ckv_sparse_decode_append",
-              "ckv_dense_decode", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times"):
+              "ckv_dense_decode", "ckv_get_device_error", "ckv_kernel_timing", "ckv_kernel_times",
+              "ckv_edges_workspace_size", "ckv_build_edges"):
         getattr(lib_, f).restype = ctypes.c_int
     lib_.ckv_status_string.argtypes = [ctypes.c_int]
     lib_.ckv_status_string.restype = ctypes.c_char_p
@@ -374,3 +381,65 @@ def ckv_dense_decode(cache: CacheDesc, q: torch.Tensor, T: int, out: torch.Tenso
     _check(lib.ckv_dense_decode(ctypes.byref(cache), q.data_ptr(), T, out.data_ptr(), ws.data_ptr(),
                                 ws.numel(), _stream(stream)),
            "ckv_dense_decode")
+
+
+# ----------------------------------------------------------------------------
+# the prefill token graph
+# ----------------------------------------------------------------------------
+
+@dataclass
+class Edges:
+    """Outputs of ckv_build_edges for U graph units of a T-token prefill."""
+    nbr: torch.Tensor      # int32 [U, T, 8] direct-edge key positions, best first, -1 padded
+    lam: torch.Tensor      # fp32 [U, T, 8] their graph logits
+    co_src: torch.Tensor   # int32 [U, pair_cap]
+    co_dst: torch.Tensor   # int32 [U, pair_cap]
+    co_w: torch.Tensor     # int32 [U, pair_cap]
+    co_n: torch.Tensor     # int32 [U]
+    dev_err: torch.Tensor  # int32 [1]
+    ws: torch.Tensor
+
+    def pairs(self, u: int):
+        """Unit u's co-attention edges as (src, dst, weight) rows, sorted."""
+        n = min(int(self.co_n[u].item()), self.co_src.shape[1])
+        t = torch.stack([self.co_src[u, :n], self.co_dst[u, :n], self.co_w[u, :n]], dim=1)
+        if n == 0:
+            return t
+        order = torch.argsort(t[:, 0].long() * (1 << 31) + t[:, 1].long())
+        return t[order]
+
+
+def ckv_edges_workspace_size(cache: CacheDesc, mode: int, S: int, T: int) -> int:
+    out = _sz(0)
+    _check(lib.ckv_edges_workspace_size(ctypes.byref(cache), mode, S, T, ctypes.byref(out)),
+           "ckv_edges_workspace_size")
+    return int(out.value)
+
+
+def new_edges(cache: CacheDesc, mode: int, S: int, T: int, pair_cap: Optional[int] = None, device="cuda") -> Edges:
+    """Buffers for ckv_build_edges; pair_cap defaults to 28 (T - S), which can
+    never overflow."""
+    U = cache.B * (cache.Hq if mode == PER_HEAD else cache.Hkv)
+    cap = max(1, 28 * max(T - S, 0)) if pair_cap is None else pair_cap
+    i32 = dict(dtype=torch.int32, device=device)
+    return Edges(nbr=torch.empty((U, T, NEIGHBOURS), **i32),
+                 lam=torch.empty((U, T, NEIGHBOURS), dtype=torch.float32, device=device),
+                 co_src=torch.empty((U, cap), **i32), co_dst=torch.empty((U, cap), **i32),
+                 co_w=torch.empty((U, cap), **i32), co_n=torch.empty((U,), **i32),
+                 dev_err=torch.zeros((1,), **i32),
+                 ws=torch.empty((max(ckv_edges_workspace_size(cache, mode, S, T), 256),), dtype=torch.uint8,
+                                device=device))
+
+
+def ckv_build_edges(cache: CacheDesc, mode: int, S: int, q_prefill: torch.Tensor, T: int, edges: Edges,
+                    stream=None) -> None:
+    """q_prefill: [B, Hq, >=T, d] bf16, contiguous rows; fills `edges`."""
+    if q_prefill.dtype != torch.bfloat16 or q_prefill.dim() != 4 or not q_prefill.is_contiguous():
+        raise ValueError("q_prefill must be a contiguous bf16 [B, Hq, T, d] tensor")
+    if q_prefill.shape[2] != T:
+        raise ValueError("q_prefill's third dimension must be T")
+    _check(lib.ckv_build_edges(ctypes.byref(cache), mode, S, q_prefill.data_ptr(), T, edges.nbr.data_ptr(),
+                               edges.lam.data_ptr(), edges.co_src.data_ptr(), edges.co_dst.data_ptr(),
+                               edges.co_w.data_ptr(), edges.co_n.data_ptr(), edges.co_src.shape[1],
+                               edges.dev_err.data_ptr(), edges.ws.data_ptr(), edges.ws.numel(), _stream(stream)),
+           "ckv_build_edges")

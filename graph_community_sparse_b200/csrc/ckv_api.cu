@@ -176,7 +176,7 @@ int32_t ckv_abi_version(void) { return CKV_ABI_VERSION; }
 int32_t ckv_debug_build(void) { return ckv::kDebugChecks ? 1 : 0; }
 
 static_assert(ckv::KK_COUNT == CKV_KERNEL_KINDS && ckv::KK_ATTENTION == CKV_KERNEL_ATTENTION &&
-                  ckv::KK_UPDATE == CKV_KERNEL_UPDATE,
+                  ckv::KK_UPDATE == CKV_KERNEL_UPDATE && ckv::KK_EDGES == CKV_KERNEL_EDGES,
               "kernel kinds match the header");
 
 ckv_status ckv_kernel_timing(int32_t enable) {
@@ -374,6 +374,39 @@ ckv_status ckv_sparse_decode_append(const ckv_cache_desc* cache, const void* q, 
     return cuda_status(ckv::launch_sparse_decode(cv, gv, sel_view(sel), q, out, nbr8, ws, &ap,
                                                  reinterpret_cast<cudaStream_t>(stream)),
                        "ckv_sparse_decode_append");
+}
+
+ckv_status ckv_edges_workspace_size(const ckv_cache_desc* cache, int32_t mode, int32_t S, int32_t T, size_t* bytes) {
+    if (!bytes) return fail(CKV_ERR_INVALID_ARG, "bytes is NULL");
+    CKV_TRY(check_cache(cache, false));
+    if (mode != CKV_GRAPH_PER_GROUP && mode != CKV_GRAPH_PER_HEAD)
+        return fail(CKV_ERR_INVALID_ARG, "graph mode %d unknown", mode);
+    if (S < 0 || T < S || T > cache->T_cap) return fail(CKV_ERR_INVALID_ARG, "need 0 <= S <= T <= T_cap");
+    const int U = cache->B * (mode == CKV_GRAPH_PER_HEAD ? cache->Hq : cache->Hkv);
+    *bytes = ckv::edges_ws_bytes(U, T, S);
+    return ok();
+}
+
+ckv_status ckv_build_edges(const ckv_cache_desc* cache, int32_t mode, int32_t S, const void* q_prefill, int32_t T,
+                           int32_t* nbr, float* lam, int32_t* co_src, int32_t* co_dst, int32_t* co_w, int32_t* co_n,
+                           int32_t pair_cap, int32_t* dev_err, void* ws, size_t ws_bytes, ckv_stream_t stream) {
+    CKV_TRY(check_cache(cache, true));
+    if (cache->dtype != CKV_DTYPE_BF16) return fail(CKV_ERR_UNSUPPORTED, "ckv_build_edges takes bf16 caches only");
+    if (mode != CKV_GRAPH_PER_GROUP && mode != CKV_GRAPH_PER_HEAD)
+        return fail(CKV_ERR_INVALID_ARG, "graph mode %d unknown", mode);
+    if (S < 0 || T < S) return fail(CKV_ERR_INVALID_ARG, "need 0 <= S <= T");
+    if (T > cache->T_cap) return fail(CKV_ERR_CAPACITY, "T = %d > T_cap = %d", T, cache->T_cap);
+    if (!q_prefill || !nbr || !co_src || !co_dst || !co_w || !co_n || !dev_err)
+        return fail(CKV_ERR_INVALID_ARG, "an output or input pointer is NULL");
+    if (!aligned16(q_prefill)) return fail(CKV_ERR_MISALIGNED, "q_prefill must be 16-byte aligned");
+    if (pair_cap < 1) return fail(CKV_ERR_INVALID_ARG, "pair_cap < 1");
+    const int64_t U = (int64_t)cache->B * (mode == CKV_GRAPH_PER_HEAD ? cache->Hq : cache->Hkv);
+    if (U > ckv::MAX_UNITS || U * (int64_t)T * 8 > (int64_t)1 << 31 || U * (int64_t)pair_cap > (int64_t)1 << 31)
+        return fail(CKV_ERR_UNSUPPORTED, "edge arrays too large");
+    CKV_TRY(check_ws(ws, ws_bytes, ckv::edges_ws_bytes((int)U, T, S)));
+    return cuda_status(ckv::launch_build_edges(cache_view(cache), mode, S, q_prefill, T, nbr, lam, co_src, co_dst, co_w,
+                                               co_n, pair_cap, dev_err, ws, reinterpret_cast<cudaStream_t>(stream)),
+                       "ckv_build_edges");
 }
 
 ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, int32_t T, float* out, void* ws,

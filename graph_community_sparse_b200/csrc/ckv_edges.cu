@@ -1,0 +1,402 @@
+// The prefill token graph for sm_100a: direct and co-attention edges.
+//
+// CommunityKV builds its graph during the prefill pass from the attention
+// scores the model computes anyway: nodes are tokens, a query that pays a key
+// much attention links the two (direct edges), keys that are attended
+// together are linked too (co-attention edges), and the first tokens, which
+// attract attention whatever their meaning, are kept out of the graph
+// (rit.work summary, section "A graph of tokens replaces re-clustering",
+// paragraph 3).  The partition of this graph (Leiden) is not computed here.
+//
+// Reading used (the pages give no thresholds): the direct edges of query i
+// are the 8 key positions j in [S, i) with the largest graph logit
+// lambda_ij = max over the graph's query heads of q_{h,i} . k_j / sqrt(d),
+// ties to the lower position -- the rule of the decode-time neighbours; the
+// co-attention edges are the key pairs j < l found together in one query's
+// direct edges, weighted by the number of such queries.
+//
+//  edges_direct_kernel: the causal Q K^T of every graph unit on the tensor
+//    cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), a dense
+//    contraction: a warp's 16 A rows are 16/GQ queries x the GQ heads of the
+//    graph, so the max over heads is a shuffle over the rows of a query; the
+//    block's 4 warps share 16-key K tiles staged by cp.async; each lane keeps
+//    a running top-8 (logit, position) list for the queries of the rows it
+//    owns; at the end the 4 lanes holding a query's columns merge their lists.
+//  edges_pairs_kernel: one thread per query adds the 28 pairs of its list to
+//    the unit's open-addressing hash table (64-bit keys, integer counts by
+//    atomics: the multiset is exact whatever the order).
+//  edges_compact_kernel: the occupied slots become the unit's (src, dst,
+//    weight) list (unordered), warp-aggregated appends.
+#include <math.h>
+
+#include "ckv_internal.cuh"
+
+namespace ckv {
+
+constexpr int ED_WARPS = 4;
+constexpr int ED_KT = 16;                 // keys per K tile
+constexpr unsigned long long ED_EMPTY = ~0ull;
+
+struct EdgesParams {
+    const __nv_bfloat16* k;     // cache K
+    int64_t sb, sh, st;
+    const __nv_bfloat16* q;     // prefill queries [B, Hq, T, d]
+    int B, Hq, Hkv, G, per_head, S, T, T_cap;
+    float inv_sqrt_d;
+    int32_t* nbr;               // [U, T, 8]
+    float* lam;                 // [U, T, 8] or NULL
+    unsigned long long* hkey;   // [U, hcap]
+    int32_t* hcnt;              // [U, hcap]
+    int hcap_log2;
+    int32_t* co_src;
+    int32_t* co_dst;
+    int32_t* co_w;
+    int32_t* co_n;              // [U]
+    int pair_cap;
+    int32_t* dev_err;
+};
+
+// Order-preserving key of (logit, position): larger is better, equal logits
+// rank the lower position first; 0 is below every real key.
+__device__ __forceinline__ unsigned long long edge_key(float lam, int pos) {
+    unsigned b = __float_as_uint(lam + 0.0f);  // -0 ranks as +0
+    b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    return ((unsigned long long)b << 32) | (unsigned)(0x7fffffff - pos);
+}
+__device__ __forceinline__ int edge_pos(unsigned long long k) { return 0x7fffffff - (int)(unsigned)(k & 0xffffffffu); }
+__device__ __forceinline__ float edge_lam(unsigned long long k) {
+    unsigned b = (unsigned)(k >> 32);
+    b = (b & 0x80000000u) ? (b & 0x7fffffffu) : ~b;
+    return __uint_as_float(b);
+}
+
+// Keep `list` (8 keys, best first) the 8 best of itself and `key`.
+__device__ __forceinline__ void top8_insert(unsigned long long (&list)[8], unsigned long long key) {
+    if (key <= list[7]) return;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        const bool gt = key > list[s];
+        const unsigned long long cur = list[s];
+        list[s] = gt ? key : cur;
+        key = gt ? cur : key;
+    }
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D>
+struct EdGeom {
+    static constexpr int KS = D / 16;        // k-steps
+    static constexpr int ROW = D * 2 + 16;   // padded bytes per staged key row (conflict-free 32-bit reads)
+    static constexpr int TILE = ED_KT * ROW;
+    static constexpr int CH = D / 8;         // 16-byte chunks per row
+};
+
+template <int D, int GQ>
+__global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __grid_constant__ EdgesParams p) {
+    using EG = EdGeom<D>;
+    constexpr int QPW = 16 / GQ;             // queries per warp (16 rows = QPW queries x GQ heads)
+    constexpr int QB = ED_WARPS * QPW;       // queries per block
+    __shared__ __align__(16) unsigned char s_k[2][EG::TILE];
+    __shared__ unsigned long long s_m[ED_WARPS][QPW][32];
+    pdl_wait();
+    const int u = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, tq = lane & 3;
+    const int b = u / p.G, gg = u - b * p.G;
+    const int gq = p.Hq / p.Hkv;
+    const int kvh = p.per_head ? gg / gq : gg;
+    const int h0 = p.per_head ? gg : gg * GQ;
+    const int i_blk = p.S + blockIdx.x * QB;               // the block's first query position
+    const int i_w = i_blk + warp * QPW;                    // the warp's first query position
+    const int j_end = min(i_blk + QB, p.T) - 1;            // keys [S, j_end) reach the block's last query
+
+    // rows of the sinks' outputs: -1 (block 0 of each unit)
+    if (blockIdx.x == 0)
+        for (int x = tid; x < p.S * 8; x += blockDim.x) {
+            p.nbr[((size_t)u * p.T) * 8 + x] = -1;
+            if (p.lam) p.lam[((size_t)u * p.T) * 8 + x] = -INFINITY;
+        }
+
+    // A fragments: row r = query r / GQ of the warp, head r % GQ
+    uint32_t a[EG::KS][4];
+    {
+        auto qrow = [&](int r) -> const __nv_bfloat16* {
+            const int i = i_w + r / GQ;
+            return i < p.T ? p.q + (((size_t)b * p.Hq + h0 + r % GQ) * p.T + i) * D : nullptr;
+        };
+        const __nv_bfloat16* r0 = qrow(g);
+        const __nv_bfloat16* r1 = qrow(g + 8);
+#pragma unroll
+        for (int kk = 0; kk < EG::KS; ++kk) {
+            const int c0 = 16 * kk + 2 * tq;
+            a[kk][0] = r0 ? *reinterpret_cast<const uint32_t*>(r0 + c0) : 0u;
+            a[kk][1] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0) : 0u;
+            a[kk][2] = r0 ? *reinterpret_cast<const uint32_t*>(r0 + c0 + 8) : 0u;
+            a[kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0 + 8) : 0u;
+        }
+    }
+    // this lane's rows g and g + 8 belong to queries qa and qb; a lane whose
+    // row is the first head of its query keeps that query's running list
+    constexpr int LG = GQ == 1 ? 0 : GQ == 2 ? 1 : GQ == 4 ? 2 : 3;
+    const bool own = (g & (GQ - 1)) == 0;
+    const int qa = g >> LG, qb = (g + 8) >> LG;
+    const int ia = i_w + qa, ib = i_w + qb;
+    unsigned long long la[8], lb[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) la[s] = lb[s] = 0ull;
+
+    const __nv_bfloat16* Kb = p.k + b * p.sb + kvh * p.sh;
+    auto stage = [&](int buf, int j0) {
+        for (int x = tid; x < ED_KT * EG::CH; x += blockDim.x) {
+            const int r = x / EG::CH, c = x % EG::CH;
+            const int j = j0 + r;
+            const bool ok = j < j_end;
+            cp_async_16(s_k[buf] + r * EG::ROW + c * 16, Kb + (int64_t)(ok ? j : p.S) * p.st + c * 8, ok);
+        }
+        cp_async_commit();
+    };
+    const int ntile = j_end > p.S ? (j_end - p.S + ED_KT - 1) / ED_KT : 0;
+    if (ntile > 0) stage(0, p.S);
+    for (int t = 0; t < ntile; ++t) {
+        const int j0 = p.S + t * ED_KT;
+        if (t + 1 < ntile) stage((t + 1) & 1, j0 + ED_KT);
+        else cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const unsigned char* kt = s_k[t & 1];
+        float c[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
+            const unsigned char* krow = kt + (8 * n + g) * EG::ROW;  // B column g: key j0 + 8n + g
+#pragma unroll
+            for (int kk = 0; kk < EG::KS; ++kk) {
+                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(krow + (16 * kk + 2 * tq) * 2);
+                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(krow + (16 * kk + 8 + 2 * tq) * 2);
+                mma_bf16(c[n], a[kk], b0, b1);
+            }
+        }
+        // max over the heads of each query (rows of one query differ in the
+        // low LG bits of g, i.e. lane bits 2 .. 1 + LG)
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float v = c[n][e];
+#pragma unroll
+                for (int o = 4; o < (4 << LG); o <<= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
+                c[n][e] = v * p.inv_sqrt_d;
+            }
+        if (own) {
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = j0 + 8 * n + 2 * tq + e;
+                    if (j < ia) top8_insert(la, edge_key(c[n][e], j));
+                    if (j < ib) top8_insert(lb, edge_key(c[n][e + 2], j));
+                }
+        }
+        __syncthreads();  // the tile is read by every warp before it is refilled
+    }
+    cp_async_wait<0>();
+
+    // merge the 4 lists of each query (lanes tq = 0..3 of its owning g)
+    if (own) {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            s_m[warp][qa][tq * 8 + s] = la[s];
+            if (qb != qa) s_m[warp][qb][tq * 8 + s] = lb[s];
+        }
+    }
+    __syncwarp();
+    if (lane < QPW) {
+        const int i = i_w + lane;
+        if (i < p.T) {
+            unsigned long long best[8];
+#pragma unroll
+            for (int s = 0; s < 8; ++s) best[s] = 0ull;
+            for (int x = 0; x < 32; ++x) top8_insert(best, s_m[warp][lane][x]);
+            int32_t* on = p.nbr + ((size_t)u * p.T + i) * 8;
+            float* ol = p.lam ? p.lam + ((size_t)u * p.T + i) * 8 : nullptr;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                on[s] = best[s] ? edge_pos(best[s]) : -1;
+                if (ol) ol[s] = best[s] ? edge_lam(best[s]) : -INFINITY;
+            }
+        }
+    }
+}
+
+__global__ void edges_clear_kernel(EdgesParams p) {
+    pdl_wait();
+    const size_t n = (size_t)p.B * p.G << p.hcap_log2;
+    for (size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (size_t)gridDim.x * blockDim.x) {
+        p.hkey[x] = ED_EMPTY;
+        p.hcnt[x] = 0;
+    }
+    for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < p.B * p.G; x += gridDim.x * blockDim.x) p.co_n[x] = 0;
+}
+
+// The pairs of query i's list, ascending by position, into unit u's table.
+__global__ void __launch_bounds__(256) edges_pairs_kernel(EdgesParams p) {
+    pdl_wait();
+    const int u = blockIdx.y;
+    const int i = p.S + blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= p.T) return;
+    const int32_t* in = p.nbr + ((size_t)u * p.T + i) * 8;
+    int v[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) v[s] = in[s];
+    // ascending by position, -1 (no entry) last
+#pragma unroll
+    for (int x = 1; x < 8; ++x)
+#pragma unroll
+        for (int y = x; y > 0; --y) {
+            const unsigned a = (unsigned)v[y - 1], c = (unsigned)v[y];  // -1 is the largest unsigned
+            const bool sw = c < a;
+            v[y - 1] = sw ? (int)c : (int)a;
+            v[y] = sw ? (int)a : (int)c;
+        }
+    const unsigned mask = (1u << p.hcap_log2) - 1u;
+    unsigned long long* tk = p.hkey + ((size_t)u << p.hcap_log2);
+    int32_t* tc = p.hcnt + ((size_t)u << p.hcap_log2);
+    for (int x = 0; x < 8; ++x) {
+        if (v[x] < 0) break;
+        for (int y = x + 1; y < 8; ++y) {
+            if (v[y] < 0) break;
+            const unsigned long long key = ((unsigned long long)(unsigned)v[x] << 32) | (unsigned)v[y];
+            unsigned h = (unsigned)((key * 0x9E3779B97F4A7C15ull) >> 32) & mask;
+            // linear probing; the table is at most half full, so the probe
+            // ends long before it could wrap around
+            for (unsigned probe = 0; probe <= mask; ++probe) {
+                const unsigned long long old = atomicCAS(tk + h, ED_EMPTY, key);
+                if (old == ED_EMPTY || old == key) {
+                    atomicAdd(tc + h, 1);
+                    break;
+                }
+                h = (h + 1) & mask;
+            }
+        }
+    }
+}
+
+// Occupied slots of unit blockIdx.y's table become its (src, dst, weight)
+// list, a warp-aggregated append per 32 slots.
+__global__ void __launch_bounds__(256) edges_compact_kernel(EdgesParams p) {
+    pdl_wait();
+    const int u = blockIdx.y, lane = threadIdx.x & 31;
+    const int n = 1 << p.hcap_log2;
+    const unsigned long long* tk = p.hkey + ((size_t)u << p.hcap_log2);
+    const int32_t* tc = p.hcnt + ((size_t)u << p.hcap_log2);
+    bool over = false;
+    for (int base = blockIdx.x * blockDim.x; base < n; base += gridDim.x * blockDim.x) {
+        const int x = base + threadIdx.x;
+        unsigned long long key = ED_EMPTY;
+        if (x < n) key = tk[x];
+        const bool occ = key != ED_EMPTY;
+        const unsigned m = __ballot_sync(FULL, occ);
+        int first = 0;
+        if (lane == 0 && m) first = atomicAdd(p.co_n + u, __popc(m));
+        first = __shfl_sync(FULL, first, 0);
+        if (occ) {
+            const int at = first + __popc(m & ((1u << lane) - 1u));
+            if (at < p.pair_cap) {
+                const size_t o = (size_t)u * p.pair_cap + at;
+                p.co_src[o] = (int32_t)(key >> 32);
+                p.co_dst[o] = (int32_t)(key & 0xffffffffu);
+                p.co_w[o] = tc[x];
+            } else {
+                over = true;
+            }
+        }
+    }
+    if (over) atomicOr(p.dev_err, CKV_DEVERR_EDGE_CAP);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+int edges_hcap_log2(int T, int S) {
+    // 28 pairs per query at most; the table keeps the load factor <= 1/2
+    const long long need = 2LL * 28 * (long long)(T - S > 0 ? T - S : 1);
+    int l = 6;
+    while ((1LL << l) < need) ++l;
+    return l;
+}
+
+size_t edges_ws_bytes(int U, int T, int S) {
+    const size_t cap = (size_t)1 << edges_hcap_log2(T, S);
+    return align256((size_t)U * cap * 8) + align256((size_t)U * cap * 4);
+}
+
+namespace {
+template <int D, int GQ>
+cudaError_t launch_direct(const EdgesParams& p, cudaStream_t st) {
+    constexpr int QB = ED_WARPS * (16 / GQ);
+    const dim3 grid((p.T - p.S + QB - 1) / QB > 0 ? (p.T - p.S + QB - 1) / QB : 1, p.B * p.G);
+    return launch_pdl(KK_EDGES, edges_direct_kernel<D, GQ>, grid, dim3(ED_WARPS * 32), 0, st, p);
+}
+}  // namespace
+
+cudaError_t launch_build_edges(const CacheView& c, int mode, int S, const void* q, int T, int32_t* nbr, float* lam,
+                               int32_t* co_src, int32_t* co_dst, int32_t* co_w, int32_t* co_n, int pair_cap,
+                               int32_t* dev_err, void* ws, cudaStream_t st) {
+    EdgesParams p{};
+    p.k = static_cast<const __nv_bfloat16*>(c.k);
+    p.sb = c.sb;
+    p.sh = c.sh;
+    p.st = c.st;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.B = c.B;
+    p.Hq = c.Hq;
+    p.Hkv = c.Hkv;
+    p.per_head = mode == CKV_GRAPH_PER_HEAD;
+    p.G = p.per_head ? c.Hq : c.Hkv;
+    p.S = S;
+    p.T = T;
+    p.T_cap = c.T_cap;
+    p.inv_sqrt_d = 1.0f / sqrtf((float)c.d);
+    p.nbr = nbr;
+    p.lam = lam;
+    p.hcap_log2 = edges_hcap_log2(T, S);
+    const int U = c.B * p.G;
+    const size_t cap = (size_t)1 << p.hcap_log2;
+    p.hkey = reinterpret_cast<unsigned long long*>(ws);
+    p.hcnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align256((size_t)U * cap * 8));
+    p.co_src = co_src;
+    p.co_dst = co_dst;
+    p.co_w = co_w;
+    p.co_n = co_n;
+    p.pair_cap = pair_cap;
+    p.dev_err = dev_err;
+    const int gq = p.per_head ? 1 : c.Hq / c.Hkv;
+
+    cudaError_t e = launch_pdl(KK_EDGES, edges_clear_kernel, dim3(296), dim3(256), 0, st, p);
+    if (e != cudaSuccess) return e;
+#define CKV_ED_CASE(DD, GG) \
+    if (c.d == DD && gq == GG) e = launch_direct<DD, GG>(p, st); else
+    CKV_ED_CASE(128, 1) CKV_ED_CASE(128, 2) CKV_ED_CASE(128, 4) CKV_ED_CASE(128, 8)
+    CKV_ED_CASE(64, 1) CKV_ED_CASE(64, 2) CKV_ED_CASE(64, 4) CKV_ED_CASE(64, 8)
+    e = cudaErrorInvalidValue;
+#undef CKV_ED_CASE
+    if (e != cudaSuccess) return e;
+    if (T > S) {
+        const dim3 pg((T - S + 255) / 256, U);
+        e = launch_pdl(KK_EDGES, edges_pairs_kernel, pg, dim3(256), 0, st, p);
+        if (e != cudaSuccess) return e;
+    }
+    const int nchunk = (int)((cap + 255) / 256);
+    const dim3 cg(nchunk < 64 ? nchunk : 64, U);
+    return launch_pdl(KK_EDGES, edges_compact_kernel, cg, dim3(256), 0, st, p);
+}
+
+}  // namespace ckv

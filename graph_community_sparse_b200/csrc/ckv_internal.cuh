@@ -307,6 +307,13 @@ cudaError_t launch_sparse_decode(const CacheView& c, const GraphView& g, const S
                                  cudaStream_t st);
 cudaError_t launch_dense_decode(const CacheView& c, const void* q, int T, float* out, void* ws,
                                 cudaStream_t st);
+// The prefill token graph (ckv_build_edges): its hash tables' size and the
+// launch of its four kernels.
+int edges_hcap_log2(int T, int S);
+size_t edges_ws_bytes(int U, int T, int S);
+cudaError_t launch_build_edges(const CacheView& c, int mode, int S, const void* q, int T, int32_t* nbr, float* lam,
+                               int32_t* co_src, int32_t* co_dst, int32_t* co_w, int32_t* co_n, int pair_cap,
+                               int32_t* dev_err, void* ws, cudaStream_t st);
 // Device address and size of the library's own decode scratch (looked up once
 // per device, with that device current).
 cudaError_t static_decode_scratch(void** ptr, size_t* bytes);
@@ -333,7 +340,7 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 // launch is bracketed by two CUDA events on its stream, and the durations are
 // summed per kind when they are read (ckv_kernel_times).  Off by default; the
 // events also cost the programmatic overlap between a call's kernels.
-enum KernelKind { KK_BUILD = 0, KK_SCORE, KK_SELECT, KK_ATTENTION, KK_MERGE, KK_UPDATE, KK_COUNT };
+enum KernelKind { KK_BUILD = 0, KK_SCORE, KK_SELECT, KK_ATTENTION, KK_MERGE, KK_UPDATE, KK_EDGES, KK_COUNT };
 bool timing_enabled();
 cudaError_t timing_mark(int kind, bool start, cudaStream_t st);
 void timing_set(bool on);

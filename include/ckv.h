@@ -65,7 +65,7 @@ extern "C" {
 #define CKV_API
 #endif
 
-#define CKV_ABI_VERSION 6
+#define CKV_ABI_VERSION 7
 #define CKV_NEIGHBOURS 8
 
 typedef struct CUstream_st* ckv_stream_t; /* the same handle as cudaStream_t */
@@ -101,6 +101,7 @@ typedef enum { CKV_ASSIGN_SCORE = 0, CKV_ASSIGN_VOTE = 1 } ckv_assign_rule;
 #define CKV_DEVERR_LABEL_RANGE 2  /* a label outside [0, Cmax) at a position >= S      */
 #define CKV_DEVERR_TAIL_FULL 4    /* ckv_assign_update found the tail full; not joined */
 #define CKV_DEVERR_TOKEN_CAP 8    /* a selection longer than tok_cap was truncated     */
+#define CKV_DEVERR_EDGE_CAP 32    /* ckv_build_edges: more co-attention pairs than pair_cap */
 #define CKV_DEVERR_INDEX 16       /* debug builds: an index read from a caller's array
                                      (a position, a run offset, a token count, a tail
                                      length) was out of range; the access was skipped */
@@ -341,6 +342,40 @@ CKV_API ckv_status ckv_dense_decode(const ckv_cache_desc* cache, const void* q, 
                             void* ws, size_t ws_bytes, ckv_stream_t stream);
 
 /*
+ * The token graph of a prefill pass, the input of the community partition
+ * ([R-A] paragraph 3: nodes are tokens; a query that pays a key much
+ * attention links the two, keys attended together are linked too, and the
+ * first tokens stay out of the graph).  The partition itself is not computed
+ * here.  For every graph unit u = b * G + g (G by `mode` as in
+ * ckv_graph_desc) and every query position i in [S, T):
+ *   direct edges  the 8 key positions j in [S, i) with the largest graph
+ *                 logit lambda_ij = max over the graph's query heads of
+ *                 q_{h,i} . k_j / sqrt(d), ties to the lower position (the
+ *                 rule of the decode-time neighbours): nbr int32 [U, T, 8],
+ *                 best first, -1 padded (rows i < S all -1); lam fp32
+ *                 [U, T, 8] their logits (-inf where -1), or NULL;
+ *   co-attention  every pair of keys j < l found together in one query's
+ *   edges         direct edges, weighted by the number of such queries:
+ *                 co_src, co_dst, co_w int32 [U, pair_cap], co_n int32 [U]
+ *                 the number of pairs; the order of a unit's pairs is
+ *                 unspecified.  A unit with more than pair_cap pairs writes
+ *                 pair_cap of them and sets CKV_DEVERR_EDGE_CAP in *dev_err
+ *                 (co_n still counts them all); pair_cap >= 28 (T - S) can
+ *                 never overflow.
+ *   q_prefill     [B, Hq, T, d] bf16 (the prefill queries), contiguous.
+ * The keys are K's rows [0, T) of the cache.  bf16 caches only
+ * (CKV_ERR_UNSUPPORTED otherwise); S <= T <= T_cap; the workspace is sized by
+ * ckv_edges_workspace_size (an open-addressing table per unit) and needs no
+ * initialisation.  The Q K^T products run on the tensor cores.
+ */
+CKV_API ckv_status ckv_edges_workspace_size(const ckv_cache_desc* cache, int32_t mode, int32_t S, int32_t T,
+                                            size_t* bytes);
+CKV_API ckv_status ckv_build_edges(const ckv_cache_desc* cache, int32_t mode, int32_t S, const void* q_prefill,
+                                   int32_t T, int32_t* nbr, float* lam, int32_t* co_src, int32_t* co_dst,
+                                   int32_t* co_w, int32_t* co_n, int32_t pair_cap, int32_t* dev_err, void* ws,
+                                   size_t ws_bytes, ckv_stream_t stream);
+
+/*
  * Reads the graph's device error word (ckv_graph_desc.dev_err, an OR of
  * CKV_DEVERR_* bits) after everything queued on `stream` so far: the one
  * call that synchronises (it waits for the stream).  *code receives the
@@ -367,9 +402,10 @@ typedef enum {
     CKV_KERNEL_SELECT = 2,     /* no kernel (kept so the kinds keep their numbers) */
     CKV_KERNEL_ATTENTION = 3,  /* split-K attention (sparse and dense decode) */
     CKV_KERNEL_MERGE = 4,      /* merge, neighbours and fused update */
-    CKV_KERNEL_UPDATE = 5      /* ckv_assign_update / ckv_append_assign */
+    CKV_KERNEL_UPDATE = 5,     /* ckv_assign_update / ckv_append_assign */
+    CKV_KERNEL_EDGES = 6       /* the four kernels of ckv_build_edges, as one */
 } ckv_kernel_kind;
-#define CKV_KERNEL_KINDS 6
+#define CKV_KERNEL_KINDS 7
 CKV_API ckv_status ckv_kernel_timing(int32_t enable);
 CKV_API ckv_status ckv_kernel_times(float* total_ms, int32_t* launches, int32_t n);
 

@@ -237,17 +237,17 @@ def direct_edges(q_heads_seq: np.ndarray, K: np.ndarray, S: int, T: int,
     decode-time neighbours), ties to the lower position, best first.
     q_heads_seq: [heads, >=T, d] (the graph's query heads over the prefill);
     K: [>=T, d].  Returns one array per query position, indexed by i - S."""
-    q_heads_seq = np.asarray(q_heads_seq, dtype=np.float64)
-    out = []
-    for i in range(S, T):
-        pos = np.arange(S, i, dtype=np.int64)
-        if len(pos) == 0:
-            out.append(pos)
-            continue
-        lam = graph_logits(q_heads_seq[:, i, :], K, pos)
-        order = np.lexsort((pos, -lam))   # logit descending, then position ascending
-        out.append(pos[order[:k]])
-    return out
+    return [direct_edges_at(q_heads_seq, K, S, i, k) for i in range(S, T)]
+
+
+def direct_edges_at(q_heads_seq: np.ndarray, K: np.ndarray, S: int, i: int, k: int = NEIGHBOURS) -> np.ndarray:
+    """The direct edges of query position i alone (see direct_edges)."""
+    pos = np.arange(S, i, dtype=np.int64)
+    if len(pos) == 0:
+        return pos
+    lam = graph_logits(np.asarray(q_heads_seq, dtype=np.float64)[:, i, :], K, pos)
+    order = np.lexsort((pos, -lam))   # logit descending, then position ascending
+    return pos[order[:k]]
 
 
 def coattention_edges(direct: Sequence[np.ndarray]) -> Dict[tuple, int]:

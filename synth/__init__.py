@@ -26,7 +26,10 @@ Recipe (all draws seeded; see `Workload`):
 * keys: K[t] = mu_{label(t)} + 0.3 N(0, I) with centres mu_c ~ N(0, I); sink
   keys N(0, I); values N(0, I);
 * queries: q_h = 0.5 mu_{c_h} + N(0, I), c_h uniform per head and step;
-* new tokens: k = mu_c + 0.3 N(0, I) with c uniform, v ~ N(0, I).
+* new tokens: k = mu_c + 0.3 N(0, I) with c uniform, v ~ N(0, I);
+* prefill queries (the token graph's input): q_{h,i} = 0.5 mu_{label(i)} +
+  N(0, I), the label that of position i's key in its KV head's clustering,
+  and N(0, I) at the sinks.
 
 In per-head mode the first head of each GQA group owns the partition the keys
 are clustered by; the other heads of the group get independent partitions
@@ -43,7 +46,7 @@ import torch
 
 __all__ = ["Workload", "WORKLOADS", "community_sizes", "graph_labels",
            "sequence_labels", "CacheDraw", "draw_cache", "draw_queries",
-           "draw_new_tokens", "torch_dtype"]
+           "draw_new_tokens", "draw_prefill_queries", "torch_dtype"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -265,3 +268,20 @@ def draw_new_tokens(wl: Workload, draw: CacheDraw, step: int, layer: int = 0):
     v = torch.randn((wl.B, wl.Hkv, wl.d), generator=gen, device=dev)
     dt = torch_dtype(wl.dtype)
     return k.to(dt).contiguous(), v.to(dt).contiguous()
+
+
+def draw_prefill_queries(wl: Workload, draw: CacheDraw, layer: int = 0) -> torch.Tensor:
+    """The queries of the prefill tokens: [B, Hq, T, d] in the cache dtype.
+    Query i of a head leans towards the centre of the cluster its own key was
+    drawn from (so attention is strongest within a community), sinks are
+    N(0, I)."""
+    dev = draw.mu.device
+    gen = _gen(dev, 3_000_017 * wl.index + 104_711 * layer + 13)
+    gq = wl.Hq // wl.Hkv
+    q = torch.randn((wl.B, wl.Hq, wl.T, wl.d), generator=gen, device=dev)
+    for b in range(wl.B):
+        for h in range(wl.Hkv):
+            lab = torch.from_numpy(draw.labels[b, cluster_graph(wl, h), wl.S:].astype(np.int64)).to(dev)
+            centre = draw.mu[b, h].index_select(0, lab)                       # [T - S, d]
+            q[b, h * gq:(h + 1) * gq, wl.S:] += 0.5 * centre[None]
+    return q.to(torch_dtype(wl.dtype)).contiguous()

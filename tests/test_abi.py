@@ -114,6 +114,20 @@ def _call_decode(cache, graph, sel, q=FAKE, out=FAKE, nbr=FAKE, ws=FAKE, ws_byte
                                      ws, ws_bytes, None)
 
 
+def _call_edges(cache, mode=0, S=4, T=4096, q=FAKE, nbr=FAKE, pair_cap=1024, ws=FAKE, ws_bytes=1 << 40):
+    return ckv.lib.ckv_build_edges(ctypes.byref(cache), mode, S, q, T, nbr, None, FAKE, FAKE, FAKE, FAKE,
+                                   pair_cap, FAKE, ws, ws_bytes, None)
+
+
+def test_edges_workspace_size_is_host_only():
+    out = ctypes.c_size_t(0)
+    assert ckv.lib.ckv_edges_workspace_size(ctypes.byref(_cache()), 0, 4, 1000, ctypes.byref(out)) == OK
+    small = out.value
+    assert ckv.lib.ckv_edges_workspace_size(ctypes.byref(_cache()), 1, 4, 4000, ctypes.byref(out)) == OK
+    assert out.value > small > 0
+    assert ckv.lib.ckv_edges_workspace_size(ctypes.byref(_cache()), 0, 4, 5000, ctypes.byref(out)) == INVALID
+
+
 CASES = [
     ("dtype", lambda: _call_build(_cache(dtype=7), _graph()), UNSUPPORTED),
     ("head dim", lambda: _call_build(_cache(d=80), _graph()), UNSUPPORTED),
@@ -188,6 +202,14 @@ CASES = [
     ("device error null code", lambda: ckv.lib.ckv_get_device_error(ctypes.byref(_graph()), None, None, 0), INVALID),
     ("device error null word", lambda: ckv.lib.ckv_get_device_error(ctypes.byref(_graph(dev_err=None)), None,
                                                                      ctypes.byref(ctypes.c_int32()), 0), INVALID),
+    ("edges: fp32 cache", lambda: _call_edges(_cache(dtype=0)), UNSUPPORTED),
+    ("edges: T above T_cap", lambda: _call_edges(_cache(), T=5000), CAPACITY),
+    ("edges: T below S", lambda: _call_edges(_cache(), S=8, T=4), INVALID),
+    ("edges: graph mode", lambda: _call_edges(_cache(), mode=3), INVALID),
+    ("edges: null nbr", lambda: _call_edges(_cache(), nbr=None), INVALID),
+    ("edges: misaligned q", lambda: _call_edges(_cache(), q=FAKE + 4), MISALIGNED),
+    ("edges: pair_cap 0", lambda: _call_edges(_cache(), pair_cap=0), INVALID),
+    ("edges: small workspace", lambda: _call_edges(_cache(), ws_bytes=1024), WORKSPACE),
 ]
 
 
