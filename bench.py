@@ -95,14 +95,15 @@ def measured_peaks():
 
 
 def csrc_digest() -> str:
-    """sha256 over the library's kernel sources (every .cu and .cuh file but
+    """sha256 over the decode kernels' sources (every .cu and .cuh file but
     the host-only ckv_api.cu (argument checks) and ckv_timing.cu (diagnostic
-    events); names and contents, in name order): any kernel or launch change
-    alters it."""
+    events), and ckv_edges.cu, the prefill token graph's own translation unit,
+    which no decode kernel includes; names and contents, in name order): any
+    decode kernel or launch change alters it."""
     d = os.path.join(ROOT, "graph_community_sparse_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")) and f not in ("ckv_api.cu", "ckv_timing.cu"):
+        if f.endswith((".cu", ".cuh", ".h")) and f not in ("ckv_api.cu", "ckv_timing.cu", "ckv_edges.cu"):
             h.update(f.encode() + b"\0" + open(os.path.join(d, f), "rb").read())
     return h.hexdigest()
 
@@ -505,6 +506,12 @@ def run_cuda(args, wl: synth.Workload, rank: int, n_ranks: int, device) -> dict:
                           f"{B_steps} steps right after the timed ones{per}"}
     if "attention" in per_kernel:
         per_kernel["attention"]["frac_nominal"] = per_kernel["attention"]["GB/s"] / NOMINAL_HBM_GBS
+    if n_layers == 1:
+        # the committed ncu DRAM bytes per launch, beside the algorithmic ones
+        kernels["ckv_score_select"]["traffic"] = profile_traffic("score_select_kernel", wl.key)
+        for name, kern in (("attention", "decode_main"), ("merge", "decode_merge")):
+            if name in per_kernel:
+                per_kernel[name]["traffic"] = profile_traffic(kern, wl.key)
 
     # dense comparator on the same caches and queries
     dense_out = torch.empty_like(st0.out)
@@ -753,6 +760,55 @@ def measure_point(layers, wl: synth.Workload, budget: int, device, flush, steps:
     return res
 
 
+def measured_bf16_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            return float(json.load(open(p))["bf16_tflops"]), "measured"
+        except Exception:
+            pass
+    return 1590.0, "fallback"
+
+
+def measure_edges(device, T: int = 32768, reps: int = 3) -> dict:
+    """The prefill token graph (ckv_build_edges) of one Qwen3-8B-shaped layer
+    at T tokens (one sequence, per-group graphs): call time, and the causal
+    Q K^T's FLOPs (2 Hq d (T - S)(T - S - 1) / 2) over it against the measured
+    dense bf16 peak."""
+    import graph_community_sparse_b200 as ckv
+    wl = synth.WORKLOADS["qwen3_8b_32k"].replace(key="prefill_edges", index=78, T=T, budgets=(2048,))
+    draw = synth.draw_cache(wl, device=device)
+    q = synth.draw_prefill_queries(wl, draw)
+    cache = ckv.cache_desc(draw.K, draw.V, wl.Hq)
+    e = ckv.new_edges(cache, ckv.PER_GROUP, wl.S, wl.T, device=device)
+    ckv.ckv_build_edges(cache, ckv.PER_GROUP, wl.S, q, wl.T, e)
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ckv.ckv_build_edges(cache, ckv.PER_GROUP, wl.S, q, wl.T, e)
+        e1.record()
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    if int(e.dev_err.item()):
+        raise RuntimeError("ckv_build_edges reported a device error")
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    n = wl.T - wl.S
+    flop = 2.0 * wl.B * wl.Hq * wl.d * n * (n - 1) / 2
+    peak, src = measured_bf16_tflops()
+    tf = flop / (ms * 1e-3) / 1e12
+    return {"title": f"prefill token graph, Qwen3-8B-shaped layer, {T} tokens, one sequence, per-group graphs",
+            "ms": ms, "reps": reps, "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                                                 "frac": tf / peak, "peak_source": peak_src_note(src),
+                                                 "flop": flop},
+            "co_attention_pairs_per_graph": float(e.co_n.float().mean().item())}
+
+
+def peak_src_note(src: str) -> str:
+    return "measured dense bf16 (cuBLAS)" if src == "measured" else "fallback bf16 figure"
+
+
 def run_sweeps(device, steps: int = 10, warmup: int = 3, call_steps: int = 5) -> dict:
     """The Zipf budget sweep (128K, B 32, per-group graphs) and one 32-layer
     Llama-3.1-8B-shaped step (64K, B 16, update), each with the dense
@@ -788,6 +844,8 @@ def run_sweeps(device, steps: int = 10, warmup: int = 3, call_steps: int = 5) ->
                                                         call_steps, 1))
     out[wl.key]["setup_s"] = round(time.perf_counter() - t0, 1)
     del layers
+    torch.cuda.empty_cache()
+    out["prefill_edges"] = measure_edges(device)
     torch.cuda.empty_cache()
     return out
 
@@ -918,6 +976,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--long-steps", type=int, default=300,
                     help="extra steps timed one by one after the timed ones, for the step-time spread")
+    ap.add_argument("--edges-only", type=int, default=None, metavar="T",
+                    help="measure only the prefill token graph (ckv_build_edges) at T tokens and print its line")
     ap.add_argument("--no-sweeps", action="store_true",
                     help="skip the Zipf budget sweep and the 32-layer step run after the headline (N = 1 only)")
     args = ap.parse_args(argv)
@@ -944,6 +1004,10 @@ def main(argv=None):
         raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.edges_only is not None:
+        if rank == 0:
+            print(json.dumps({"prefill_edges": measure_edges(device, T=args.edges_only)}), flush=True)
+        return 0
     if ws > 1:
         import datetime
 
