@@ -107,12 +107,35 @@ struct AssignScratch {
     float row[CKV_NEIGHBOURS][D];  // candidate centres, reused by the update
 };
 
+// Fused append: the first graph of each (sequence, KV head) copies the
+// caller's new K and V rows into the cache at pos (threads t of nthr, one
+// 16-byte vector each per step).
+__device__ __forceinline__ void append_rows(const AssignParams& p, int u, int t, int nthr) {
+    if (!p.k_dst) return;
+    const int b = u / p.G, g = u - b * p.G;
+    const int gq = p.Hq / p.Hkv;
+    if (p.per_head && g % gq != 0) return;
+    const int kvh = p.per_head ? g / gq : g;
+    const uint4* ks = static_cast<const uint4*>(p.k_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
+    const uint4* vs = static_cast<const uint4*>(p.v_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
+    const size_t eoff = (size_t)(b * p.csb + kvh * p.csh);  // elements
+    const size_t esz = p.row_vec * 16 / (size_t)p.d;
+    uint4* kd = reinterpret_cast<uint4*>(static_cast<char*>(p.k_dst) + eoff * esz);
+    uint4* vd = reinterpret_cast<uint4*>(static_cast<char*>(p.v_dst) + eoff * esz);
+    for (int i = t; i < p.row_vec; i += nthr) {
+        kd[i] = ks[i];
+        vd[i] = vs[i];
+    }
+}
+
 // The update of unit u by NW warps (thread index tid in [0, 32 NW)), given
 // the unit's 8 neighbour positions (-1: none) in nbrpos, readable by all of
 // them.  sync() is a barrier over exactly these NW warps.  Warp w scores
 // candidates w, w + NW, ... with all of their centres requested before any
-// is used; warp 0 picks the winner and moves its centre.
-template <typename T, int D, int NW, typename Sync>
+// is used; warp 0 picks the winner and moves its centre.  APPEND: the last
+// warp also writes the new K/V rows (append_rows; the attention's merge
+// kernel does that itself, off the update's path).
+template <typename T, int D, int NW, bool APPEND, typename Sync>
 __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const int* nbrpos, int tid,
                                             AssignScratch<D>& sc, Sync sync) {
     constexpr int E = D / 32;
@@ -123,19 +146,7 @@ __device__ __forceinline__ void assign_unit(const AssignParams& p, int u, const 
     const int b = u / p.G, g = u - b * p.G;
     const int gq = p.Hq / p.Hkv;
     const int kvh = p.per_head ? g / gq : g;
-    if (p.k_dst && (!p.per_head || g % gq == 0) && warp == NW - 1) {
-        // the first graph of each (sequence, KV head) appends its K and V rows
-        const uint4* ks = static_cast<const uint4*>(p.k_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
-        const uint4* vs = static_cast<const uint4*>(p.v_new) + ((size_t)b * p.Hkv + kvh) * p.row_vec;
-        const size_t eoff = (size_t)(b * p.csb + kvh * p.csh);  // elements
-        const size_t esz = p.row_vec * 16 / (size_t)p.d;
-        uint4* kd = reinterpret_cast<uint4*>(static_cast<char*>(p.k_dst) + eoff * esz);
-        uint4* vd = reinterpret_cast<uint4*>(static_cast<char*>(p.v_dst) + eoff * esz);
-        for (int i = lane; i < p.row_vec; i += 32) {
-            kd[i] = ks[i];
-            vd[i] = vs[i];
-        }
-    }
+    if (APPEND && warp == NW - 1) append_rows(p, u, lane, 32);
     if (tid < CKV_NEIGHBOURS) {
         int c = -1;
         const int np = nbrpos[tid];

@@ -479,7 +479,7 @@ template <typename T, int D>
 __device__ __forceinline__ void merge_assign(const DecodeParams& p, int u, const int* nbpos, int xt) {
     __shared__ __align__(16) AssignScratch<D> s_as;
     auto sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(NBR_THREADS) : "memory"); };
-    assign_unit<T, D, NBR_WARPS>(p.ap, u, nbpos, xt, s_as, sync);
+    assign_unit<T, D, NBR_WARPS, false>(p.ap, u, nbpos, xt, s_as, sync);
 }
 
 // One block per unit: threads 0..D-1 own one output dimension each (all the
@@ -506,6 +506,9 @@ __global__ void __launch_bounds__(D + (DENSE ? 0 : 32 * NBR_WARPS), 2) decode_me
         total = p.unit_prefix[p.U];
     }
     float* outu = p.out + ((size_t)b * p.Hq + h0) * D;
+    // the new K/V rows go into the cache first, by the output threads (off
+    // the neighbour search and update, which wait on more round trips)
+    if (!DENSE && p.append && t < D) append_rows(p.ap, u, t, D);
     if (uend <= ubeg) {
         for (int i = t; i < GQ * D; i += blockDim.x) outu[i] = 0.f;
         if (!DENSE && p.want_nbr && p.nbr8 && t < 8) p.nbr8[(size_t)u * 8 + t] = -1;

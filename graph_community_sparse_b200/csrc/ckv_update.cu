@@ -17,7 +17,7 @@ __global__ void __launch_bounds__(CKV_NEIGHBOURS * 32) assign_kernel(AssignParam
     const int u = blockIdx.x;
     if (threadIdx.x < CKV_NEIGHBOURS) s_nbr[threadIdx.x] = p.nbr8[(size_t)u * CKV_NEIGHBOURS + threadIdx.x];
     __syncthreads();
-    assign_unit<T, D, CKV_NEIGHBOURS>(p, u, s_nbr, threadIdx.x, s_scratch, [] { __syncthreads(); });
+    assign_unit<T, D, CKV_NEIGHBOURS, true>(p, u, s_nbr, threadIdx.x, s_scratch, [] { __syncthreads(); });
 }
 
 cudaError_t launch_assign_update(const CacheView& c, const GraphView& g, int pos, const void* k_new,
