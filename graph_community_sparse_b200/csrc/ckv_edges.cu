@@ -98,13 +98,53 @@ struct EdGeom {
     static constexpr int CH = D / 8;         // 16-byte chunks per row
 };
 
+// ldmatrix of four 8x8 b16 matrices (the B fragments of two k-steps)
+__device__ __forceinline__ void ed_ldsm_x4(unsigned addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+// A running top-8 list with the logit of its 8th entry (-inf while it is not
+// full): a logit below it cannot enter, so most values cost one comparison.
+struct Top8 {
+    unsigned long long key[8];
+    float th;
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) key[s] = 0ull;
+        th = -INFINITY;
+    }
+    __device__ __forceinline__ void offer(float lam, int pos) {
+        if (lam < th) return;
+        top8_insert(key, edge_key(lam, pos));
+        th = key[7] ? edge_lam(key[7]) : -INFINITY;
+    }
+};
+
+// Rows of the A operand: with one head per graph the 16 rows are 16
+// queries; otherwise rows g and g + 8 (the two rows of one accumulator
+// thread) are two heads of one query, so the max over heads starts inside
+// the thread, and the GQ / 2 row pairs of a query sit in lanes that differ in
+// lane bits 2 .. LG.
+template <int GQ>
+struct EdRows {
+    static constexpr int LG = GQ == 1 ? 0 : GQ == 2 ? 1 : GQ == 4 ? 2 : 3;
+    static constexpr int QPW = 16 / GQ;                 // queries per warp
+    static constexpr int NSH = GQ == 1 ? 1 : GQ / 2;    // lanes sharing a query's columns
+    static constexpr int MLEN = GQ == 1 ? 32 : 16 * GQ; // list entries merged per query
+    __device__ static int query(int r) { return GQ == 1 ? r : (r & 7) >> (LG - 1); }
+    __device__ static int head(int r) { return GQ == 1 ? 0 : (((r & 7) & (NSH - 1)) << 1) | (r >> 3); }
+};
+
 template <int D, int GQ>
 __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __grid_constant__ EdgesParams p) {
     using EG = EdGeom<D>;
-    constexpr int QPW = 16 / GQ;             // queries per warp (16 rows = QPW queries x GQ heads)
+    using ER = EdRows<GQ>;
+    constexpr int QPW = ER::QPW;
     constexpr int QB = ED_WARPS * QPW;       // queries per block
+    constexpr int LG = ER::LG, NSH = ER::NSH;
     __shared__ __align__(16) unsigned char s_k[2][EG::TILE];
-    __shared__ unsigned long long s_m[ED_WARPS][QPW][32];
+    __shared__ unsigned long long s_m[ED_WARPS][QPW][ER::MLEN];
     pdl_wait();
     const int u = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tq = lane & 3;
@@ -123,12 +163,12 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
             if (p.lam) p.lam[((size_t)u * p.T) * 8 + x] = -INFINITY;
         }
 
-    // A fragments: row r = query r / GQ of the warp, head r % GQ
+    // A fragments of rows g and g + 8
     uint32_t a[EG::KS][4];
     {
         auto qrow = [&](int r) -> const __nv_bfloat16* {
-            const int i = i_w + r / GQ;
-            return i < p.T ? p.q + (((size_t)b * p.Hq + h0 + r % GQ) * p.T + i) * D : nullptr;
+            const int i = i_w + ER::query(r);
+            return i < p.T ? p.q + (((size_t)b * p.Hq + h0 + ER::head(r)) * p.T + i) * D : nullptr;
         };
         const __nv_bfloat16* r0 = qrow(g);
         const __nv_bfloat16* r1 = qrow(g + 8);
@@ -141,15 +181,15 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
             a[kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0 + 8) : 0u;
         }
     }
-    // this lane's rows g and g + 8 belong to queries qa and qb; a lane whose
-    // row is the first head of its query keeps that query's running list
-    constexpr int LG = GQ == 1 ? 0 : GQ == 2 ? 1 : GQ == 4 ? 2 : 3;
-    const bool own = (g & (GQ - 1)) == 0;
-    const int qa = g >> LG, qb = (g + 8) >> LG;
+    // the lane's lists: one head per graph, queries g (la) and g + 8 (lb);
+    // otherwise query g >> (LG - 1) (la), whose keys this lane's sub-index
+    // among the NSH lanes sharing them takes a share of
+    const int qa = ER::query(g), qb = ER::query(g + 8);
     const int ia = i_w + qa, ib = i_w + qb;
-    unsigned long long la[8], lb[8];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) la[s] = lb[s] = 0ull;
+    const int sub = g & (NSH - 1);
+    Top8 la, lb;
+    la.init();
+    lb.init();
 
     const __nv_bfloat16* Kb = p.k + b * p.sb + kvh * p.sh;
     auto stage = [&](int buf, int j0) {
@@ -161,6 +201,9 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         }
         cp_async_commit();
     };
+    // ldmatrix lane address inside a tile: matrix lane >> 3 is (k-step 2 kp +
+    // (lane >> 4), dims half (lane >> 3) & 1) of key row lane & 7
+    const int lm_off = (lane & 7) * EG::ROW + (lane >> 3) * 16;
     const int ntile = j_end > p.S ? (j_end - p.S + ED_KT - 1) / ED_KT : 0;
     if (ntile > 0) stage(0, p.S);
     for (int t = 0; t < ntile; ++t) {
@@ -169,52 +212,68 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         else cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();
-        const unsigned char* kt = s_k[t & 1];
+        const unsigned kbase = static_cast<unsigned>(__cvta_generic_to_shared(s_k[t & 1]));
         float c[2][4];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
-            const unsigned char* krow = kt + (8 * n + g) * EG::ROW;  // B column g: key j0 + 8n + g
 #pragma unroll
-            for (int kk = 0; kk < EG::KS; ++kk) {
-                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(krow + (16 * kk + 2 * tq) * 2);
-                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(krow + (16 * kk + 8 + 2 * tq) * 2);
-                mma_bf16(c[n], a[kk], b0, b1);
+            for (int kp = 0; kp < EG::KS / 2; ++kp) {
+                uint32_t b0, b1, b2, b3;
+                ed_ldsm_x4(kbase + 8 * n * EG::ROW + lm_off + kp * 64, b0, b1, b2, b3);
+                mma_bf16(c[n], a[2 * kp], b0, b1);
+                mma_bf16(c[n], a[2 * kp + 1], b2, b3);
             }
         }
-        // max over the heads of each query (rows of one query differ in the
-        // low LG bits of g, i.e. lane bits 2 .. 1 + LG)
-#pragma unroll
-        for (int n = 0; n < 2; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float v = c[n][e];
-#pragma unroll
-                for (int o = 4; o < (4 << LG); o <<= 1) v = fmaxf(v, __shfl_xor_sync(FULL, v, o));
-                c[n][e] = v * p.inv_sqrt_d;
-            }
-        if (own) {
+        if constexpr (GQ == 1) {
+            // rows g and g + 8 are queries qa and qb: keys j0 + 8n + 2tq + e
 #pragma unroll
             for (int n = 0; n < 2; ++n)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int j = j0 + 8 * n + 2 * tq + e;
-                    if (j < ia) top8_insert(la, edge_key(c[n][e], j));
-                    if (j < ib) top8_insert(lb, edge_key(c[n][e + 2], j));
+                    if (j < ia) la.offer(c[n][e] * p.inv_sqrt_d, j);
+                    if (j < ib) lb.offer(c[n][e + 2] * p.inv_sqrt_d, j);
+                }
+        } else {
+            // max over the query's heads: its two rows here, then the NSH
+            // lanes holding its other row pairs
+            float v[2][2];
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float x = fmaxf(c[n][e], c[n][e + 2]);
+#pragma unroll
+                    for (int o = 4; o < (4 << (LG - 1)); o <<= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
+                    v[n][e] = x * p.inv_sqrt_d;
+                }
+            // this lane's share of the query's 4 keys: all (NSH 1), key
+            // pair n = sub (NSH 2), or key (sub >> 1, sub & 1) (NSH 4)
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool mine = NSH == 1 || (NSH == 2 ? n == sub : (2 * n + e) == sub);
+                    const int j = j0 + 8 * n + 2 * tq + e;
+                    if (mine && j < ia) la.offer(v[n][e], j);
                 }
         }
         __syncthreads();  // the tile is read by every warp before it is refilled
     }
     cp_async_wait<0>();
 
-    // merge the 4 lists of each query (lanes tq = 0..3 of its owning g)
-    if (own) {
+    // merge each query's lists (its 4 column lanes x NSH row-pair lanes)
+    if constexpr (GQ == 1) {
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
-            s_m[warp][qa][tq * 8 + s] = la[s];
-            if (qb != qa) s_m[warp][qb][tq * 8 + s] = lb[s];
+            s_m[warp][qa][tq * 8 + s] = la.key[s];
+            s_m[warp][qb][tq * 8 + s] = lb.key[s];
         }
+    } else {
+#pragma unroll
+        for (int s = 0; s < 8; ++s) s_m[warp][qa][(tq * NSH + sub) * 8 + s] = la.key[s];
     }
     __syncwarp();
     if (lane < QPW) {
@@ -223,7 +282,7 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
             unsigned long long best[8];
 #pragma unroll
             for (int s = 0; s < 8; ++s) best[s] = 0ull;
-            for (int x = 0; x < 32; ++x) top8_insert(best, s_m[warp][lane][x]);
+            for (int x = 0; x < ER::MLEN; ++x) top8_insert(best, s_m[warp][lane][x]);
             int32_t* on = p.nbr + ((size_t)u * p.T + i) * 8;
             float* ol = p.lam ? p.lam + ((size_t)u * p.T + i) * 8 : nullptr;
 #pragma unroll
