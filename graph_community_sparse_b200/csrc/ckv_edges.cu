@@ -18,10 +18,15 @@
 //  edges_direct_kernel: the causal Q K^T of every graph unit on the tensor
 //    cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), a dense
 //    contraction: a warp's 16 A rows are 16/GQ queries x the GQ heads of the
-//    graph, so the max over heads is a shuffle over the rows of a query; the
-//    block's 4 warps share 16-key K tiles staged by cp.async; each lane keeps
-//    a running top-8 (logit, position) list for the queries of the rows it
-//    owns; at the end the 4 lanes holding a query's columns merge their lists.
+//    graph, placed so that an accumulator thread's two rows (g, g + 8) are
+//    two heads of one query: the max over heads is one comparison in the
+//    thread plus a shuffle per further pair.  The block's 4 warps share
+//    32-key K tiles staged by cp.async into padded rows and read as B
+//    fragments by ldmatrix.  Each lane keeps a running top-8 (logit,
+//    position) list for its share of its query's keys, with the 8th logit as
+//    a threshold; insertions run in a warp-uniform branch taken only when
+//    some lane has one, so most tiles cost the products, the max and one
+//    comparison per value.  At the end a query's lists are merged.
 //  edges_pairs_kernel: one thread per query adds the 28 pairs of its list to
 //    the unit's open-addressing hash table (64-bit keys, integer counts by
 //    atomics: the multiset is exact whatever the order).
@@ -34,7 +39,7 @@
 namespace ckv {
 
 constexpr int ED_WARPS = 4;
-constexpr int ED_KT = 16;                 // keys per K tile
+constexpr int ED_KT = 32;                 // keys per K tile
 constexpr unsigned long long ED_EMPTY = ~0ull;
 
 struct EdgesParams {
@@ -114,8 +119,9 @@ struct Top8 {
         for (int s = 0; s < 8; ++s) key[s] = 0ull;
         th = -INFINITY;
     }
-    __device__ __forceinline__ void offer(float lam, int pos) {
-        if (lam < th) return;
+    // may (lam, pos) enter?  (a logit equal to the 8th's needs the key)
+    __device__ __forceinline__ bool wants(float lam) const { return lam >= th; }
+    __device__ __forceinline__ void insert(float lam, int pos) {
         top8_insert(key, edge_key(lam, pos));
         th = key[7] ? edge_lam(key[7]) : -INFINITY;
     }
@@ -143,8 +149,12 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
     constexpr int QPW = ER::QPW;
     constexpr int QB = ED_WARPS * QPW;       // queries per block
     constexpr int LG = ER::LG, NSH = ER::NSH;
-    __shared__ __align__(16) unsigned char s_k[2][EG::TILE];
-    __shared__ unsigned long long s_m[ED_WARPS][QPW][ER::MLEN];
+    // the two K tiles, and after the last tile the lists to merge
+    constexpr int SK_BYTES = 2 * EG::TILE;
+    constexpr int SM_BYTES = ED_WARPS * QPW * ER::MLEN * 8;
+    __shared__ __align__(16) unsigned char s_raw[SK_BYTES > SM_BYTES ? SK_BYTES : SM_BYTES];
+    unsigned char (*s_k)[EG::TILE] = reinterpret_cast<unsigned char (*)[EG::TILE]>(s_raw);
+    unsigned long long (*s_m)[QPW][ER::MLEN] = reinterpret_cast<unsigned long long (*)[QPW][ER::MLEN]>(s_raw);
     pdl_wait();
     const int u = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tq = lane & 3;
@@ -192,12 +202,18 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
     lb.init();
 
     const __nv_bfloat16* Kb = p.k + b * p.sb + kvh * p.sh;
+    // this thread's 16-byte chunks of a K tile: rows r0 + i RSTEP, chunk c0
+    constexpr int NCHT = ED_KT * EG::CH / (ED_WARPS * 32);  // chunks per thread
+    constexpr int RSTEP = ED_WARPS * 32 / EG::CH;
+    static_assert(NCHT * ED_WARPS * 32 == ED_KT * EG::CH, "whole chunks per thread");
+    const int r0 = tid / EG::CH, c0 = tid % EG::CH;
+    const __nv_bfloat16* kc = Kb + c0 * 8;
     auto stage = [&](int buf, int j0) {
-        for (int x = tid; x < ED_KT * EG::CH; x += blockDim.x) {
-            const int r = x / EG::CH, c = x % EG::CH;
-            const int j = j0 + r;
+#pragma unroll
+        for (int i = 0; i < NCHT; ++i) {
+            const int j = j0 + r0 + i * RSTEP;
             const bool ok = j < j_end;
-            cp_async_16(s_k[buf] + r * EG::ROW + c * 16, Kb + (int64_t)(ok ? j : p.S) * p.st + c * 8, ok);
+            cp_async_16(s_k[buf] + (r0 + i * RSTEP) * EG::ROW + c0 * 16, kc + (int64_t)(ok ? j : p.S) * p.st, ok);
         }
         cp_async_commit();
     };
@@ -213,9 +229,10 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         cp_async_wait<1>();
         __syncthreads();
         const unsigned kbase = static_cast<unsigned>(__cvta_generic_to_shared(s_k[t & 1]));
-        float c[2][4];
+        constexpr int NT = ED_KT / 8;  // n-tiles of 8 keys
+        float c[NT][4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n) {
+        for (int n = 0; n < NT; ++n) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
 #pragma unroll
@@ -227,21 +244,36 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
             }
         }
         if constexpr (GQ == 1) {
-            // rows g and g + 8 are queries qa and qb: keys j0 + 8n + 2tq + e
+            // rows g and g + 8 are queries qa and qb: keys j0 + 8n + 2tq + e;
+            // the insertions run only when some lane has one (a warp-uniform
+            // branch: most tiles have none)
+            float va[NT][2], vb[NT][2];
+            bool any = false;
 #pragma unroll
-            for (int n = 0; n < 2; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int j = j0 + 8 * n + 2 * tq + e;
-                    if (j < ia) la.offer(c[n][e] * p.inv_sqrt_d, j);
-                    if (j < ib) lb.offer(c[n][e + 2] * p.inv_sqrt_d, j);
+                    va[n][e] = c[n][e] * p.inv_sqrt_d;
+                    vb[n][e] = c[n][e + 2] * p.inv_sqrt_d;
+                    any |= (j < ia && la.wants(va[n][e])) || (j < ib && lb.wants(vb[n][e]));
                 }
+            if (__any_sync(FULL, any)) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int j = j0 + 8 * n + 2 * tq + e;
+                        if (j < ia && la.wants(va[n][e])) la.insert(va[n][e], j);
+                        if (j < ib && lb.wants(vb[n][e])) lb.insert(vb[n][e], j);
+                    }
+            }
         } else {
             // max over the query's heads: its two rows here, then the NSH
             // lanes holding its other row pairs
-            float v[2][2];
+            float v[NT][2];
 #pragma unroll
-            for (int n = 0; n < 2; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float x = fmaxf(c[n][e], c[n][e + 2]);
@@ -249,20 +281,33 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                     for (int o = 4; o < (4 << (LG - 1)); o <<= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
                     v[n][e] = x * p.inv_sqrt_d;
                 }
-            // this lane's share of the query's 4 keys: all (NSH 1), key
-            // pair n = sub (NSH 2), or key (sub >> 1, sub & 1) (NSH 4)
+            // this lane's share of the query's 2 NT keys here: value 2n + e
+            // belongs to the lane whose sub-index is its remainder modulo NSH;
+            // the insertions run only when some lane has one
+            bool any = false;
 #pragma unroll
-            for (int n = 0; n < 2; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const bool mine = NSH == 1 || (NSH == 2 ? n == sub : (2 * n + e) == sub);
+                    const bool mine = ((2 * n + e) & (NSH - 1)) == sub;
                     const int j = j0 + 8 * n + 2 * tq + e;
-                    if (mine && j < ia) la.offer(v[n][e], j);
+                    any |= mine && j < ia && la.wants(v[n][e]);
                 }
+            if (__any_sync(FULL, any)) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool mine = ((2 * n + e) & (NSH - 1)) == sub;
+                        const int j = j0 + 8 * n + 2 * tq + e;
+                        if (mine && j < ia && la.wants(v[n][e])) la.insert(v[n][e], j);
+                    }
+            }
         }
         __syncthreads();  // the tile is read by every warp before it is refilled
     }
     cp_async_wait<0>();
+    __syncthreads();  // no warp reads a K tile any more: the lists take its space
 
     // merge each query's lists (its 4 column lanes x NSH row-pair lanes)
     if constexpr (GQ == 1) {
