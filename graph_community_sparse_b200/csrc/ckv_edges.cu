@@ -33,6 +33,7 @@
 //  edges_compact_kernel: the occupied slots become the unit's (src, dst,
 //    weight) list (unordered), warp-aggregated appends.
 #include <math.h>
+#include <type_traits>
 
 #include "ckv_internal.cuh"
 
@@ -220,29 +221,10 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
     // ldmatrix lane address inside a tile: matrix lane >> 3 is (k-step 2 kp +
     // (lane >> 4), dims half (lane >> 3) & 1) of key row lane & 7
     const int lm_off = (lane & 7) * EG::ROW + (lane >> 3) * 16;
-    const int ntile = j_end > p.S ? (j_end - p.S + ED_KT - 1) / ED_KT : 0;
-    if (ntile > 0) stage(0, p.S);
-    for (int t = 0; t < ntile; ++t) {
-        const int j0 = p.S + t * ED_KT;
-        if (t + 1 < ntile) stage((t + 1) & 1, j0 + ED_KT);
-        else cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const unsigned kbase = static_cast<unsigned>(__cvta_generic_to_shared(s_k[t & 1]));
-        constexpr int NT = ED_KT / 8;  // n-tiles of 8 keys
-        float c[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
-#pragma unroll
-            for (int kp = 0; kp < EG::KS / 2; ++kp) {
-                uint32_t b0, b1, b2, b3;
-                ed_ldsm_x4(kbase + 8 * n * EG::ROW + lm_off + kp * 64, b0, b1, b2, b3);
-                mma_bf16(c[n], a[2 * kp], b0, b1);
-                mma_bf16(c[n], a[2 * kp + 1], b2, b3);
-            }
-        }
+    constexpr int NT = ED_KT / 8;  // n-tiles of 8 keys per K tile
+    // a tile's logits into the lists (MASK: test each key against the query)
+    auto epilogue = [&](float (&c)[NT][4], int j0, auto mask_tag) {
+        constexpr bool MASK = decltype(mask_tag)::value;
         if constexpr (GQ == 1) {
             // rows g and g + 8 are queries qa and qb: keys j0 + 8n + 2tq + e;
             // the insertions run only when some lane has one (a warp-uniform
@@ -256,7 +238,7 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                     const int j = j0 + 8 * n + 2 * tq + e;
                     va[n][e] = c[n][e] * p.inv_sqrt_d;
                     vb[n][e] = c[n][e + 2] * p.inv_sqrt_d;
-                    any |= (j < ia && la.wants(va[n][e])) || (j < ib && lb.wants(vb[n][e]));
+                    any |= ((!MASK || j < ia) && la.wants(va[n][e])) || ((!MASK || j < ib) && lb.wants(vb[n][e]));
                 }
             if (__any_sync(FULL, any)) {
 #pragma unroll
@@ -264,9 +246,34 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int j = j0 + 8 * n + 2 * tq + e;
-                        if (j < ia && la.wants(va[n][e])) la.insert(va[n][e], j);
-                        if (j < ib && lb.wants(vb[n][e])) lb.insert(vb[n][e], j);
+                        if ((!MASK || j < ia) && la.wants(va[n][e])) la.insert(va[n][e], j);
+                        if ((!MASK || j < ib) && lb.wants(vb[n][e])) lb.insert(vb[n][e], j);
                     }
+            }
+        } else if constexpr (NSH == 2) {
+            // four heads: the two lanes holding a query's columns split them,
+            // this lane keeping column e = sub of each n-tile; each lane maxes
+            // its two rows (two heads) for both columns and sends its partner
+            // the column the partner keeps
+            float v[NT];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const float x0 = fmaxf(c[n][0], c[n][2]), x1 = fmaxf(c[n][1], c[n][3]);
+                const float keep = sub ? x1 : x0, give = sub ? x0 : x1;
+                v[n] = fmaxf(keep, __shfl_xor_sync(FULL, give, 4)) * p.inv_sqrt_d;
+            }
+            bool any = false;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int j = j0 + 8 * n + 2 * tq + sub;
+                any |= (!MASK || j < ia) && la.wants(v[n]);
+            }
+            if (__any_sync(FULL, any)) {
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const int j = j0 + 8 * n + 2 * tq + sub;
+                    if ((!MASK || j < ia) && la.wants(v[n])) la.insert(v[n], j);
+                }
             }
         } else {
             // max over the query's heads: its two rows here, then the NSH
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                 for (int e = 0; e < 2; ++e) {
                     const bool mine = ((2 * n + e) & (NSH - 1)) == sub;
                     const int j = j0 + 8 * n + 2 * tq + e;
-                    any |= mine && j < ia && la.wants(v[n][e]);
+                    any |= mine && (!MASK || j < ia) && la.wants(v[n][e]);
                 }
             if (__any_sync(FULL, any)) {
 #pragma unroll
@@ -300,10 +307,36 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                     for (int e = 0; e < 2; ++e) {
                         const bool mine = ((2 * n + e) & (NSH - 1)) == sub;
                         const int j = j0 + 8 * n + 2 * tq + e;
-                        if (mine && j < ia && la.wants(v[n][e])) la.insert(v[n][e], j);
+                        if (mine && (!MASK || j < ia) && la.wants(v[n][e])) la.insert(v[n][e], j);
                     }
             }
         }
+    };
+    const int ntile = j_end > p.S ? (j_end - p.S + ED_KT - 1) / ED_KT : 0;
+    if (ntile > 0) stage(0, p.S);
+    for (int t = 0; t < ntile; ++t) {
+        const int j0 = p.S + t * ED_KT;
+        if (t + 1 < ntile) stage((t + 1) & 1, j0 + ED_KT);
+        else cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const unsigned kbase = static_cast<unsigned>(__cvta_generic_to_shared(s_k[t & 1]));
+        float c[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < EG::KS / 2; ++kp) {
+                uint32_t b0, b1, b2, b3;
+                ed_ldsm_x4(kbase + 8 * n * EG::ROW + lm_off + kp * 64, b0, b1, b2, b3);
+                mma_bf16(c[n], a[2 * kp], b0, b1);
+                mma_bf16(c[n], a[2 * kp + 1], b2, b3);
+            }
+        }
+        // keys of this tile all below the warp's first query: no causal test
+        if (j0 + ED_KT <= i_w) epilogue(c, j0, std::false_type{});
+        else epilogue(c, j0, std::true_type{});
         __syncthreads();  // the tile is read by every warp before it is refilled
     }
     cp_async_wait<0>();
