@@ -35,6 +35,7 @@ SHAPES = [
     shape("edges_group_gq2_d64", 73, Hq=4, Hkv=2, d=64, T=900, B=2),
     shape("edges_group_gq1", 74, Hq=2, Hkv=2, T=333),
     shape("edges_no_sinks", 75, Hq=8, Hkv=2, S=0, T=517),
+    shape("edges_group_gq4_d64", 79, Hq=8, Hkv=2, d=64, T=777),
 ]
 
 
