@@ -114,17 +114,20 @@ __device__ __forceinline__ void ed_ldsm_x4(unsigned addr, uint32_t& r0, uint32_t
 // full): a logit below it cannot enter, so most values cost one comparison.
 struct Top8 {
     unsigned long long key[8];
-    float th;
+    float th;   // this list's 8th logit
+    float cut;  // a logit below which no key can be in the query's top 8:
+                // the largest 8th logit among the lists sharing the query
     __device__ __forceinline__ void init() {
 #pragma unroll
         for (int s = 0; s < 8; ++s) key[s] = 0ull;
-        th = -INFINITY;
+        th = cut = -INFINITY;
     }
-    // may (lam, pos) enter?  (a logit equal to the 8th's needs the key)
-    __device__ __forceinline__ bool wants(float lam) const { return lam >= th; }
+    // may (lam, pos) enter?  (a logit equal to the cut needs the key)
+    __device__ __forceinline__ bool wants(float lam) const { return lam >= cut; }
     __device__ __forceinline__ void insert(float lam, int pos) {
         top8_insert(key, edge_key(lam, pos));
         th = key[7] ? edge_lam(key[7]) : -INFINITY;
+        cut = fmaxf(cut, th);
     }
 };
 
@@ -337,6 +340,26 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         // keys of this tile all below the warp's first query: no causal test
         if (j0 + ED_KT <= i_w) epilogue(c, j0, std::false_type{});
         else epilogue(c, j0, std::true_type{});
+        // a query's lists are spread over its 4 column lanes (lane bits 0-1)
+        // and, with several heads, its NSH row-pair lanes (bits 2 ..): a list
+        // holds 8 keys at or above its 8th logit, so the largest such logit
+        // among them bounds the query's 8th best from below and prunes all
+        // of them (a list of its own sees only a share of the keys and would
+        // admit many more)
+        {
+            float ca = la.th, cb = lb.th;
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1) {
+                ca = fmaxf(ca, __shfl_xor_sync(FULL, ca, o));
+                if constexpr (GQ == 1) cb = fmaxf(cb, __shfl_xor_sync(FULL, cb, o));
+            }
+            if constexpr (GQ > 1) {
+#pragma unroll
+                for (int o = 4; o < 4 * NSH; o <<= 1) ca = fmaxf(ca, __shfl_xor_sync(FULL, ca, o));
+            }
+            la.cut = fmaxf(la.cut, ca);
+            if constexpr (GQ == 1) lb.cut = fmaxf(lb.cut, cb);
+        }
         __syncthreads();  // the tile is read by every warp before it is refilled
     }
     cp_async_wait<0>();
