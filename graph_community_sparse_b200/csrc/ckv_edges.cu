@@ -26,7 +26,8 @@
 //    position) list for its share of its query's keys, with the 8th logit as
 //    a threshold; insertions run in a warp-uniform branch taken only when
 //    some lane has one, so most tiles cost the products, the max and one
-//    comparison per value.  At the end a query's lists are merged.
+//    comparison per value.  At the end the lists of each query are merged
+//    by the lanes that share it, pairwise over shuffles.
 //  edges_pairs_kernel: one thread per query adds the 28 pairs of its list to
 //    the unit's open-addressing hash table (64-bit keys, integer counts by
 //    atomics: the multiset is exact whatever the order).
@@ -377,13 +378,43 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         for (int s = 0; s < 8; ++s) s_m[warp][qa][(tq * NSH + sub) * 8 + s] = la.key[s];
     }
     __syncwarp();
-    if (lane < QPW) {
-        const int i = i_w + lane;
-        if (i < p.T) {
-            unsigned long long best[8];
+    // a query's MLEN / 8 sorted lists, merged by LPQ = 32 / QPW lanes: lane
+    // (query lane / LPQ, part lane % LPQ) takes its part's lists in turn, then
+    // the parts merge pairwise over shuffles (the best 8 of two sorted lists
+    // of 8: the pairwise larger of one list and the other reversed is
+    // bitonic, and a 12-exchange network sorts it)
+    constexpr int LPQ = 32 / QPW;              // lanes per query
+    constexpr int LPL = ER::MLEN / 8 / LPQ;    // lists per lane
+    static_assert(LPL >= 1 && LPL * LPQ * 8 == ER::MLEN, "whole lists per lane");
+    const int mq = lane / LPQ, mp = lane % LPQ;
+    unsigned long long best[8];
 #pragma unroll
-            for (int s = 0; s < 8; ++s) best[s] = 0ull;
-            for (int x = 0; x < ER::MLEN; ++x) top8_insert(best, s_m[warp][lane][x]);
+    for (int s = 0; s < 8; ++s) best[s] = s_m[warp][mq][mp * LPL * 8 + s];
+#pragma unroll
+    for (int l = 1; l < LPL; ++l)
+#pragma unroll
+        for (int s = 0; s < 8; ++s) top8_insert(best, s_m[warp][mq][(mp * LPL + l) * 8 + s]);
+#pragma unroll
+    for (int o = 1; o < LPQ; o <<= 1) {
+        unsigned long long other[8];
+#pragma unroll
+        for (int s = 0; s < 8; ++s) other[s] = __shfl_xor_sync(FULL, best[s], o);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) best[s] = best[s] > other[7 - s] ? best[s] : other[7 - s];
+        // bitonic (rising then falling, or the reverse): sort descending
+#pragma unroll
+        for (int h = 4; h >= 1; h >>= 1)
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                if ((s & h) == 0) {
+                    const unsigned long long x = best[s], y = best[s + h];
+                    best[s] = x > y ? x : y;
+                    best[s + h] = x > y ? y : x;
+                }
+    }
+    if (mp == 0) {
+        const int i = i_w + mq;
+        if (i < p.T) {
             int32_t* on = p.nbr + ((size_t)u * p.T + i) * 8;
             float* ol = p.lam ? p.lam + ((size_t)u * p.T + i) * 8 : nullptr;
 #pragma unroll
