@@ -23,10 +23,11 @@
 //    thread plus a shuffle per further pair.  The block's 4 warps share
 //    32-key K tiles staged by cp.async into padded rows and read as B
 //    fragments by ldmatrix.  Each lane keeps a running top-8 (logit,
-//    position) list for its share of its query's keys, with the 8th logit as
-//    a threshold; insertions run in a warp-uniform branch taken only when
-//    some lane has one, so most tiles cost the products, the max and one
-//    comparison per value.  At the end the lists of each query are merged
+//    position) list for its share of its query's keys; after every tile the
+//    lists of a query share the largest of their 8th logits as a pruning
+//    cut (a lower bound of the query's 8th best); insertions run in a
+//    warp-uniform branch taken only when some lane has one, so most tiles
+//    cost the products, the max and one comparison per value.  At the end the lists of each query are merged
 //    by the lanes that share it, pairwise over shuffles.
 //  edges_pairs_kernel: one thread per query adds the 28 pairs of its list to
 //    the unit's open-addressing hash table (64-bit keys, integer counts by
