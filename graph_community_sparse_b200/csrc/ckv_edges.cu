@@ -20,7 +20,8 @@
 //    contraction: a warp's 16 A rows are 16/GQ queries x the GQ heads of the
 //    graph, placed so that an accumulator thread's two rows (g, g + 8) are
 //    two heads of one query: the max over heads is one comparison in the
-//    thread plus a shuffle per further pair.  The block's 4 warps share
+//    thread plus a shuffle per further pair.  With several heads a warp
+//    holds two such 16-row tiles, so each K fragment feeds two products.  The block's 4 warps share
 //    32-key K tiles staged by cp.async into padded rows and read as B
 //    fragments by ldmatrix.  Each lane keeps a running top-8 (logit,
 //    position) list for its share of its query's keys; after every tile the
@@ -43,6 +44,7 @@ namespace ckv {
 
 constexpr int ED_WARPS = 4;
 constexpr int ED_KT = 32;                 // keys per K tile
+constexpr int ED_RT = 2;                  // 16-row A tiles per warp (several heads per graph)
 constexpr unsigned long long ED_EMPTY = ~0ull;
 
 struct EdgesParams {
@@ -141,7 +143,9 @@ struct Top8 {
 template <int GQ>
 struct EdRows {
     static constexpr int LG = GQ == 1 ? 0 : GQ == 2 ? 1 : GQ == 4 ? 2 : 3;
-    static constexpr int QPW = 16 / GQ;                 // queries per warp
+    static constexpr int RT = GQ == 1 ? 1 : ED_RT;      // A row tiles per warp
+    static constexpr int QPW0 = 16 / GQ;                // queries per row tile
+    static constexpr int QPW = RT * QPW0;               // queries per warp
     static constexpr int NSH = GQ == 1 ? 1 : GQ / 2;    // lanes sharing a query's columns
     static constexpr int MLEN = GQ == 1 ? 32 : 16 * GQ; // list entries merged per query
     __device__ static int query(int r) { return GQ == 1 ? r : (r & 7) >> (LG - 1); }
@@ -179,11 +183,14 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
             if (p.lam) p.lam[((size_t)u * p.T) * 8 + x] = -INFINITY;
         }
 
-    // A fragments of rows g and g + 8
-    uint32_t a[EG::KS][4];
-    {
+    // A fragments of rows g and g + 8 of each row tile (row tile t holds the
+    // warp's queries t QPW0 ..)
+    constexpr int RT = ER::RT;
+    uint32_t a[RT][EG::KS][4];
+#pragma unroll
+    for (int t = 0; t < RT; ++t) {
         auto qrow = [&](int r) -> const __nv_bfloat16* {
-            const int i = i_w + ER::query(r);
+            const int i = i_w + t * ER::QPW0 + ER::query(r);
             return i < p.T ? p.q + (((size_t)b * p.Hq + h0 + ER::head(r)) * p.T + i) * D : nullptr;
         };
         const __nv_bfloat16* r0 = qrow(g);
@@ -191,16 +198,17 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
 #pragma unroll
         for (int kk = 0; kk < EG::KS; ++kk) {
             const int c0 = 16 * kk + 2 * tq;
-            a[kk][0] = r0 ? *reinterpret_cast<const uint32_t*>(r0 + c0) : 0u;
-            a[kk][1] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0) : 0u;
-            a[kk][2] = r0 ? *reinterpret_cast<const uint32_t*>(r0 + c0 + 8) : 0u;
-            a[kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0 + 8) : 0u;
+            a[t][kk][0] = r0 ? *reinterpret_cast<const uint32_t*>(r0 + c0) : 0u;
+            a[t][kk][1] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0) : 0u;
+            a[t][kk][2] = r0 ? *reinterpret_cast<const uint32_t*>(r0 + c0 + 8) : 0u;
+            a[t][kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(r1 + c0 + 8) : 0u;
         }
     }
     // the lane's lists: one head per graph, queries g (la) and g + 8 (lb);
-    // otherwise query g >> (LG - 1) (la), whose keys this lane's sub-index
-    // among the NSH lanes sharing them takes a share of
-    const int qa = ER::query(g), qb = ER::query(g + 8);
+    // otherwise query g >> (LG - 1) of each row tile (la, and lb for the
+    // second), whose keys this lane's sub-index among the NSH lanes sharing
+    // them takes a share of
+    const int qa = ER::query(g), qb = RT == 2 ? qa + ER::QPW0 : ER::query(g + 8);
     const int ia = i_w + qa, ib = i_w + qb;
     const int sub = g & (NSH - 1);
     Top8 la, lb;
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
     const int lm_off = (lane & 7) * EG::ROW + (lane >> 3) * 16;
     constexpr int NT = ED_KT / 8;  // n-tiles of 8 keys per K tile
     // a tile's logits into the lists (MASK: test each key against the query)
-    auto epilogue = [&](float (&c)[NT][4], int j0, auto mask_tag) {
+    auto epilogue = [&](float (&c)[NT][4], int j0, auto mask_tag, Top8& L, const int iq) {
         constexpr bool MASK = decltype(mask_tag)::value;
         if constexpr (GQ == 1) {
             // rows g and g + 8 are queries qa and qb: keys j0 + 8n + 2tq + e;
@@ -271,13 +279,13 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
                 const int j = j0 + 8 * n + 2 * tq + sub;
-                any |= (!MASK || j < ia) && la.wants(v[n]);
+                any |= (!MASK || j < iq) && L.wants(v[n]);
             }
             if (__any_sync(FULL, any)) {
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     const int j = j0 + 8 * n + 2 * tq + sub;
-                    if ((!MASK || j < ia) && la.wants(v[n])) la.insert(v[n], j);
+                    if ((!MASK || j < iq) && L.wants(v[n])) L.insert(v[n], j);
                 }
             }
         } else {
@@ -303,7 +311,7 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                 for (int e = 0; e < 2; ++e) {
                     const bool mine = ((2 * n + e) & (NSH - 1)) == sub;
                     const int j = j0 + 8 * n + 2 * tq + e;
-                    any |= mine && (!MASK || j < ia) && la.wants(v[n][e]);
+                    any |= mine && (!MASK || j < iq) && L.wants(v[n][e]);
                 }
             if (__any_sync(FULL, any)) {
 #pragma unroll
@@ -312,7 +320,7 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                     for (int e = 0; e < 2; ++e) {
                         const bool mine = ((2 * n + e) & (NSH - 1)) == sub;
                         const int j = j0 + 8 * n + 2 * tq + e;
-                        if (mine && (!MASK || j < ia) && la.wants(v[n][e])) la.insert(v[n][e], j);
+                        if (mine && (!MASK || j < iq) && L.wants(v[n][e])) L.insert(v[n][e], j);
                     }
             }
         }
@@ -326,22 +334,32 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         cp_async_wait<1>();
         __syncthreads();
         const unsigned kbase = static_cast<unsigned>(__cvta_generic_to_shared(s_k[t & 1]));
-        float c[NT][4];
+        float c[RT][NT][4];
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) c[n][e] = 0.f;
+            for (int t = 0; t < RT; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c[t][n][e] = 0.f;
 #pragma unroll
             for (int kp = 0; kp < EG::KS / 2; ++kp) {
                 uint32_t b0, b1, b2, b3;
                 ed_ldsm_x4(kbase + 8 * n * EG::ROW + lm_off + kp * 64, b0, b1, b2, b3);
-                mma_bf16(c[n], a[2 * kp], b0, b1);
-                mma_bf16(c[n], a[2 * kp + 1], b2, b3);
+#pragma unroll
+                for (int t = 0; t < RT; ++t) {
+                    mma_bf16(c[t][n], a[t][2 * kp], b0, b1);
+                    mma_bf16(c[t][n], a[t][2 * kp + 1], b2, b3);
+                }
             }
         }
         // keys of this tile all below the warp's first query: no causal test
-        if (j0 + ED_KT <= i_w) epilogue(c, j0, std::false_type{});
-        else epilogue(c, j0, std::true_type{});
+        if (j0 + ED_KT <= i_w) {
+            epilogue(c[0], j0, std::false_type{}, la, ia);
+            if constexpr (RT == 2) epilogue(c[1], j0, std::false_type{}, lb, ib);
+        } else {
+            epilogue(c[0], j0, std::true_type{}, la, ia);
+            if constexpr (RT == 2) epilogue(c[1], j0, std::true_type{}, lb, ib);
+        }
         // a query's lists are spread over its 4 column lanes (lane bits 0-1)
         // and, with several heads, its NSH row-pair lanes (bits 2 ..): a list
         // holds 8 keys at or above its 8th logit, so the largest such logit
@@ -356,11 +374,18 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
                 if constexpr (GQ == 1) cb = fmaxf(cb, __shfl_xor_sync(FULL, cb, o));
             }
             if constexpr (GQ > 1) {
+                if constexpr (RT == 2) {
 #pragma unroll
-                for (int o = 4; o < 4 * NSH; o <<= 1) ca = fmaxf(ca, __shfl_xor_sync(FULL, ca, o));
+                    for (int o = 1; o < 4; o <<= 1) cb = fmaxf(cb, __shfl_xor_sync(FULL, cb, o));
+                }
+#pragma unroll
+                for (int o = 4; o < 4 * NSH; o <<= 1) {
+                    ca = fmaxf(ca, __shfl_xor_sync(FULL, ca, o));
+                    if constexpr (RT == 2) cb = fmaxf(cb, __shfl_xor_sync(FULL, cb, o));
+                }
             }
             la.cut = fmaxf(la.cut, ca);
-            if constexpr (GQ == 1) lb.cut = fmaxf(lb.cut, cb);
+            if constexpr (GQ == 1 || RT == 2) lb.cut = fmaxf(lb.cut, cb);
         }
         __syncthreads();  // the tile is read by every warp before it is refilled
     }
@@ -376,7 +401,10 @@ __global__ void __launch_bounds__(ED_WARPS * 32) edges_direct_kernel(const __gri
         }
     } else {
 #pragma unroll
-        for (int s = 0; s < 8; ++s) s_m[warp][qa][(tq * NSH + sub) * 8 + s] = la.key[s];
+        for (int s = 0; s < 8; ++s) {
+            s_m[warp][qa][(tq * NSH + sub) * 8 + s] = la.key[s];
+            if constexpr (RT == 2) s_m[warp][qb][(tq * NSH + sub) * 8 + s] = lb.key[s];
+        }
     }
     __syncwarp();
     // a query's MLEN / 8 sorted lists, merged by LPQ = 32 / QPW lanes: lane
@@ -533,7 +561,7 @@ size_t edges_ws_bytes(int U, int T, int S) {
 namespace {
 template <int D, int GQ>
 cudaError_t launch_direct(const EdgesParams& p, cudaStream_t st) {
-    constexpr int QB = ED_WARPS * (16 / GQ);
+    constexpr int QB = ED_WARPS * EdRows<GQ>::QPW;
     const dim3 grid((p.T - p.S + QB - 1) / QB > 0 ? (p.T - p.S + QB - 1) / QB : 1, p.B * p.G);
     return launch_pdl(KK_EDGES, edges_direct_kernel<D, GQ>, grid, dim3(ED_WARPS * 32), 0, st, p);
 }
